@@ -1,0 +1,417 @@
+"""Plain fp64 CPU oracle for the FlexAttention forward pass and BlockMask.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import or run this module.
+The CUDA library never calls it, and it shares no code, constants or tables
+with the CUDA library: mask and score kinds here are strings, interpreted
+below from the pages' formulas.
+
+Sources ("page" = the web page, cited by its title and section):
+
+* "flexattention-score-mod-block-mask" (charlestar.github.io), sections
+  "What one connection goes through" (the semantic definition of s_ij,
+  s~_ij and o_i), "score_mod changes the score, and the order changes the
+  result" (cap-then-bias combination, masking after the score transform),
+  "mask_mod defines legal connections, BlockMask defines block work"
+  (empty / full / partial tiles), "A call example pinned to one version"
+  (window 0 <= p_i - p_j < W), "Packing" (same document), "At decode,
+  q_idx = 0 is not position 0" (logical query position), "Correctness
+  checks come before performance" (fully masked rows).
+* "PyTorch Flex Attention complete guide" (2kiu.com), sections 1.2
+  (score_mod receives the *query* head), 2 (lse output), 3.1 (a block is
+  sparse only if all its elements are masked), 3.2 (dense reconstruction of
+  the ordered block lists), 4.1 (create_block_mask pipeline: dense mask,
+  pad, per-block reduction, separate full blocks), 6.1 (GQA broadcast),
+  6.2 (default scale 1/sqrt(E)).
+* "Attention expressions" (docs.tensorcad.dev), section "Examples" (prefix-LM,
+  sinks, chunked attention, ALiBi slope, Gemma-2 soft-cap).
+* "Causal Mask" (quant67.com, Transformer series no. 17), section 4
+  "query shorter than key: bottom-right alignment" and section 7 "-inf,
+  finfo.min and fully masked rows".
+
+Readings taken where the pages leave a step open (each is listed in the
+design notes too):
+
+* Query positions are logical: q_pos = i + (S_b - L), S_b the valid KV
+  length of sequence b (S when none is given).  All mask and score rules see
+  q_pos; key positions are kv = j.  Keys j >= S_b are never visible.
+* A fully masked row (no visible key, or every visible score mapped to -inf
+  by the score rule) gives output 0 and lse = -inf, never NaN.
+* lse is the natural-log log-sum-exp of the transformed, scaled scores over
+  the visible keys.
+* GQA maps query head h to KV head h // (Hq // Hkv); the score rule sees the
+  query head.
+* ALiBi / distance slope for head h is 2^(-8 (h + 1) / H), h from 0.
+* Tiles at a ragged edge are classified over their in-range cells only.
+  Index lists are ascending; unused slots hold 0.
+
+Rows are computed in groups of whole rows purely to bound memory; every row
+is evaluated in full, exactly as the definition states.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+MASK_KINDS = ("none", "causal", "sliding_window", "document", "prefix_lm", "chunked", "dense")
+SCORE_KINDS = ("none", "softcap", "alibi", "cap_then_bias")
+
+
+# ---------------------------------------------------------------------------
+# Positions
+# ---------------------------------------------------------------------------
+
+def query_positions(L, S_b):
+    """Logical query positions q_pos = i + (S_b - L) (bottom-right alignment).
+
+    "Causal Mask" (quant67.com) section 4: with L < S the r-th query sees the
+    first S - L + r + 1 keys; "flexattention-score-mod-block-mask" section
+    "At decode, q_idx = 0 is not position 0": q_position = q_idx + q_offset.
+    """
+    return np.arange(L, dtype=np.int64) + (int(S_b) - int(L))
+
+
+def _row_for_batch(arr, b):
+    """Row b of a (B, S) array, or its only row when it broadcasts (1, S) / (S,)."""
+    arr = np.asarray(arr)
+    if arr.ndim == 1:
+        return arr
+    return arr[b] if arr.shape[0] > 1 else arr[0]
+
+
+def doc_positions_from_ids(doc_row):
+    """Position of each token inside its own document (restarting at 0).
+
+    "flexattention-score-mod-block-mask" section "Packing": the in-segment
+    position column of the packing table restarts at 0 for every sample.
+    """
+    doc_row = np.asarray(doc_row)
+    pos = np.zeros(len(doc_row), dtype=np.int64)
+    for t in range(1, len(doc_row)):
+        pos[t] = pos[t - 1] + 1 if doc_row[t] == doc_row[t - 1] else 0
+    return pos
+
+
+# ---------------------------------------------------------------------------
+# mask_mod: visibility M(b, h, q_pos, kv)
+# ---------------------------------------------------------------------------
+
+def visible(mask, b, h, qp, kv, S_b):
+    """Boolean visibility for query positions ``qp`` (column) x keys ``kv`` (row).
+
+    ``mask`` is a dict with ``kind`` in MASK_KINDS:
+
+    * none -- every in-range key (the noop mask; guide section 4.4).
+    * causal -- kv <= q.
+    * sliding_window -- kv <= q and (q - kv < W or kv < n_sink): window of W
+      keys including the query itself ("flexattention-score-mod-block-mask",
+      "A call example pinned to one version": 0 <= p_i - p_j < W), plus sink
+      tokens ("Attention expressions", Examples: q - kv < W or kv < 4 with
+      causal on).
+    * document -- kv <= q and doc[q] == doc[kv] ("flexattention-score-mod-
+      block-mask", "Packing"; "Causal Mask" section 3, intra-document causal).
+    * prefix_lm -- kv <= q or kv < P, causal off ("Attention expressions",
+      Examples; "Causal Mask" section 3, Prefix LM).
+    * chunked -- kv <= q and floor(q / C) == floor(kv / C)
+      ("Attention expressions", Examples, causal on).
+    * dense -- an explicit (L, S) boolean matrix (oracle-only, for the pages'
+      key-padding example).
+
+    Keys at or beyond the valid length S_b are invisible under every kind.
+    """
+    qp = np.asarray(qp, dtype=np.int64)[:, None]
+    kv = np.asarray(kv, dtype=np.int64)[None, :]
+    kind = mask["kind"]
+    in_range = kv < S_b
+    causal = kv <= qp
+    if kind == "none":
+        m = np.ones(np.broadcast(qp, kv).shape, dtype=bool)
+    elif kind == "causal":
+        m = causal
+    elif kind == "sliding_window":
+        W, n_sink = int(mask["window"]), int(mask.get("n_sink", 0))
+        m = causal & (((qp - kv) < W) | (kv < n_sink))
+    elif kind == "document":
+        doc_b = _row_for_batch(mask["doc_id"], b)
+        qi = np.clip(qp, 0, len(doc_b) - 1)
+        ki = np.clip(kv, 0, len(doc_b) - 1)
+        m = causal & (qp >= 0) & (doc_b[qi] == doc_b[ki])
+    elif kind == "prefix_lm":
+        P = int(mask["prefix"])
+        m = causal | (kv < P)
+    elif kind == "chunked":
+        C = int(mask["chunk"])
+        m = causal & (np.floor_divide(qp, C) == np.floor_divide(kv, C))
+    elif kind == "dense":
+        m = np.asarray(mask["matrix"], dtype=bool)
+        rows = mask.get("rows")
+        m = m if rows is None else m[np.asarray(rows)]
+    else:
+        raise ValueError(f"unknown mask kind {kind!r}")
+    return np.broadcast_to(m, np.broadcast(qp, kv).shape) & in_range
+
+
+# ---------------------------------------------------------------------------
+# score_mod: g(s, b, h, q_pos, kv)
+# ---------------------------------------------------------------------------
+
+def distance_slope(h, H):
+    """2^(-8 (h+1) / H) ("Attention expressions", Examples: ALiBi)."""
+    return 2.0 ** (-8.0 * (h + 1) / H)
+
+
+def score_mod(score, s, b, h, qp, kv, Hq):
+    """Apply the score transform g to the scaled scores ``s`` (rows qp, cols kv).
+
+    * none -- g = s.
+    * softcap -- g = c tanh(s / c) ("flexattention-score-mod-block-mask",
+      "score_mod changes the score"; "Attention expressions", Gemma 2's cap).
+    * alibi -- g = s - slope_h (q - kv) ("Attention expressions", Examples).
+    * cap_then_bias -- g = c tanh(s / c) + slope_h (p_kv - p_q): cap first,
+      then the distance bias ("flexattention-score-mod-block-mask", "score_mod
+      changes the score": the bias-then-cap form is a different rule).  p is
+      the in-document position when ``pos == 'in_doc'`` (computed here from
+      the document ids), else the global position.
+    """
+    kind = score["kind"]
+    if kind == "none":
+        return s
+    if kind == "softcap":
+        c = float(score["cap"])
+        return c * np.tanh(s / c)
+    H = int(score.get("slope_heads") or Hq)
+    slope = distance_slope(h, H)
+    qp = np.asarray(qp, dtype=np.int64)[:, None]
+    kv = np.asarray(kv, dtype=np.int64)[None, :]
+    if kind == "alibi":
+        return s - slope * (qp - kv).astype(np.float64)
+    if kind == "cap_then_bias":
+        c = float(score["cap"])
+        if score.get("pos", "global") == "in_doc":
+            doc_b = _row_for_batch(score["doc_id"], b)
+            p = doc_positions_from_ids(doc_b)
+            pq = p[np.clip(qp, 0, len(p) - 1)]
+            pk = p[np.clip(kv, 0, len(p) - 1)]
+        else:
+            pq, pk = qp, kv
+        return c * np.tanh(s / c) + slope * (pk - pq).astype(np.float64)
+    raise ValueError(f"unknown score kind {kind!r}")
+
+
+# ---------------------------------------------------------------------------
+# Forward
+# ---------------------------------------------------------------------------
+
+def _as_f64(x):
+    if hasattr(x, "detach"):  # a torch tensor: upcast exactly
+        import torch
+        return x.detach().to(torch.float64).cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def attention_rows(q_rows, k, v, scale, mask, score, b, h, qp, S_b, Hq):
+    """Output rows and lse for one (b, h) and a set of query positions.
+
+    The definition in "flexattention-score-mod-block-mask", "What one
+    connection goes through": s_ij = scale q_i . k_j; s~_ij = g(s_ij, ...) where
+    M_ij, -inf elsewhere; o_i = sum_j softmax_j(s~_ij) v_j.  The score rule is
+    applied first and the mask second (section "score_mod changes the score").
+    """
+    S = k.shape[0]
+    kv = np.arange(S, dtype=np.int64)
+    s = scale * (q_rows @ k.T)                      # full score rows
+    g = score_mod(score, s, b, h, qp, kv, Hq)       # transform everywhere
+    vis = visible(mask, b, h, qp, kv, S_b)
+    bad = vis & (np.isnan(g) | (g == np.inf))
+    assert not bad.any(), "score rule produced NaN or +inf on a visible cell"
+    st = np.where(vis, g, NEG_INF)                  # mask after the transform
+    m = st.max(axis=1)
+    out = np.zeros((q_rows.shape[0], v.shape[1]), dtype=np.float64)
+    lse = np.full(q_rows.shape[0], NEG_INF)
+    live = m > NEG_INF
+    if live.any():
+        p = np.exp(st[live] - m[live, None])
+        l = p.sum(axis=1)
+        out[live] = (p @ v) / l[:, None]
+        lse[live] = m[live] + np.log(l)
+    return out, lse
+
+
+def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, row_group=512):
+    """fp64 FlexAttention forward: returns (out (B,Hq,L,Ev), lse (B,Hq,L)).
+
+    q (B,Hq,L,E), k (B,Hkv,S,E), v (B,Hkv,S,Ev); numpy arrays or torch
+    tensors (upcast exactly).  ``scale`` defaults to 1/sqrt(E) (guide section
+    6.2).  GQA broadcasts KV head h // (Hq // Hkv) (guide section 6.1).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, L, E = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if Hq != Hkv:
+        assert enable_gqa and Hq % Hkv == 0, "Hq != Hkv needs enable_gqa and Hq % Hkv == 0"
+    G = Hq // Hkv
+    mask = mask or {"kind": "none"}
+    score = score or {"kind": "none"}
+    scale = 1.0 / math.sqrt(E) if scale is None else float(scale)
+    out = np.zeros((B, Hq, L, v.shape[3]))
+    lse = np.full((B, Hq, L), NEG_INF)
+    for b in range(B):
+        S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
+        qp_all = query_positions(L, S_b)
+        for h in range(Hq):
+            hk = h // G
+            for r0 in range(0, L, row_group):
+                r1 = min(L, r0 + row_group)
+                mk = dict(mask)
+                if mask["kind"] == "dense":
+                    mk["rows"] = np.arange(r0, r1)
+                o, ls = attention_rows(q[b, h, r0:r1], k[b, hk], v[b, hk], scale, mk, score, b, h,
+                                       qp_all[r0:r1], S_b, Hq)
+                out[b, h, r0:r1] = o
+                lse[b, h, r0:r1] = ls
+    return out, lse
+
+
+def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False):
+    """Output and lse for sampled (b, h, row) triples; returns (out[n,Ev], lse[n]).
+
+    Used on workloads too large for :func:`forward`: each sampled row is
+    computed in full by :func:`attention_rows`.
+    """
+    Bq, Hq, L, E = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    mask = mask or {"kind": "none"}
+    score = score or {"kind": "none"}
+    scale = 1.0 / math.sqrt(E) if scale is None else float(scale)
+    outs, lses = [], []
+    for (b, h, r) in samples:
+        S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
+        qp = query_positions(L, S_b)[r:r + 1]
+        qrow = _as_f64(q[b, h, r:r + 1])
+        kk = _as_f64(k[b, h // G])
+        vv = _as_f64(v[b, h // G])
+        o, ls = attention_rows(qrow, kk, vv, scale, mask, score, b, h, qp, S_b, Hq)
+        outs.append(o[0])
+        lses.append(ls[0])
+    return np.stack(outs), np.array(lses)
+
+
+# ---------------------------------------------------------------------------
+# BlockMask
+# ---------------------------------------------------------------------------
+
+def block_mask(mask, B, H, L, S, BM, BN, kv_len=None):
+    """Brute-force BlockMask: classify every (m, n) tile as empty / full / partial.
+
+    "flexattention-score-mod-block-mask", "mask_mod defines legal
+    connections": an all-invisible tile is skipped, an all-visible tile is
+    full (no element mask, score_mod still runs), anything else is partial.
+    Guide section 3.1: a block is sparse only when *all* its elements are
+    masked.  Guide section 4.1: the dense mask is evaluated, reduced per
+    block, and full blocks are stored separately from partial ones.
+
+    Returns int32 arrays kv_num_blocks (B,H,Mb), kv_indices (B,H,Mb,Nb) of the
+    partial tiles, full_kv_num_blocks (B,H,Mb), full_kv_indices (B,H,Mb,Nb),
+    indices ascending, unused slots 0.  Tiles at a ragged edge are classified
+    over their in-range cells only.  The menu's masks do not depend on the
+    head, so every head row is the same.
+    """
+    Mb, Nb = -(-L // BM), -(-S // BN)
+    kv_num = np.zeros((B, H, Mb), np.int32)
+    kv_idx = np.zeros((B, H, Mb, Nb), np.int32)
+    full_num = np.zeros((B, H, Mb), np.int32)
+    full_idx = np.zeros((B, H, Mb, Nb), np.int32)
+    kv = np.arange(S, dtype=np.int64)
+    for b in range(B):
+        S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
+        qp_all = query_positions(L, S_b)
+        for h in range(H):
+            for mt in range(Mb):
+                r0, r1 = mt * BM, min(L, (mt + 1) * BM)
+                mk = dict(mask)
+                if mask["kind"] == "dense":
+                    mk["rows"] = np.arange(r0, r1)
+                vis = visible(mk, b, h, qp_all[r0:r1], kv, S_b)
+                nf = npart = 0
+                for nt in range(Nb):
+                    c0, c1 = nt * BN, min(S, (nt + 1) * BN)
+                    cell = vis[:, c0:c1]
+                    if cell.all():
+                        full_idx[b, h, mt, nf] = nt
+                        nf += 1
+                    elif cell.any():
+                        kv_idx[b, h, mt, npart] = nt
+                        npart += 1
+                kv_num[b, h, mt] = npart
+                full_num[b, h, mt] = nf
+    return dict(kv_num_blocks=kv_num, kv_indices=kv_idx,
+                full_kv_num_blocks=full_num, full_kv_indices=full_idx, Mb=Mb, Nb=Nb)
+
+
+def block_map(bm, b=0, h=0):
+    """Dense tile map from the ordered lists: 'F' full, 'P' partial, '0' empty.
+
+    Guide section 3.2: the dense form is rebuilt by walking each row's first
+    num_blocks indices.
+    """
+    Mb, Nb = bm["Mb"], bm["Nb"]
+    grid = [["0"] * Nb for _ in range(Mb)]
+    for mt in range(Mb):
+        for i in range(int(bm["kv_num_blocks"][b, h, mt])):
+            grid[mt][int(bm["kv_indices"][b, h, mt, i])] = "P"
+        for i in range(int(bm["full_kv_num_blocks"][b, h, mt])):
+            grid[mt][int(bm["full_kv_indices"][b, h, mt, i])] = "F"
+    return grid
+
+
+def sparsity(bm, b=0, h=0):
+    """Percentage of tiles that are skipped (guide section 3.3, sparsity())."""
+    grid = block_map(bm, b, h)
+    cells = [c for row in grid for c in row]
+    return 100.0 * sum(c == "0" for c in cells) / len(cells)
+
+
+# ---------------------------------------------------------------------------
+# Split-KV partials and their combination
+# ---------------------------------------------------------------------------
+
+def split_partials(q_rows, k, v, scale, mask, score, b, h, qp, S_b, Hq, bounds):
+    """Per-split (o_s, lse_s) over key ranges [bounds[i], bounds[i+1]).
+
+    Each split is the same definition restricted to its key range: keys
+    outside it are treated as invisible.
+    """
+    parts = []
+    S = k.shape[0]
+    kv = np.arange(S, dtype=np.int64)
+    base = visible(mask, b, h, qp, kv, S_b)
+    for lo, hi in zip(bounds[:-1], bounds[1:]):
+        sub = dict(kind="dense", matrix=base & ((kv >= lo) & (kv < hi))[None, :])
+        o, ls = attention_rows(q_rows, k, v, scale, sub, score, b, h, qp, S_b, Hq)
+        parts.append((o, ls))
+    return parts
+
+
+def combine(parts):
+    """Merge split results: lse = ln sum_s e^{lse_s}; o = sum_s e^{lse_s - lse} o_s.
+
+    Follows from the lse definition (guide section 2): the softmax over the
+    union of disjoint key sets is the lse-weighted mixture of the per-set
+    softmaxes.  All-empty rows stay (0, -inf).
+    """
+    lses = np.stack([p[1] for p in parts])          # (n_split, rows)
+    outs = np.stack([p[0] for p in parts])          # (n_split, rows, Ev)
+    m = lses.max(axis=0)
+    out = np.zeros(outs.shape[1:])
+    lse = np.full(lses.shape[1], NEG_INF)
+    live = m > NEG_INF
+    w = np.exp(lses[:, live] - m[live])
+    tot = w.sum(axis=0)
+    out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]
+    lse[live] = m[live] + np.log(tot)
+    return out, lse

@@ -1,0 +1,418 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each check takes the oracle module and raises AssertionError when the oracle
+disagrees with: a worked example printed on the pages (fixtures under
+tests/golden/, each citing its page and section), a closed form, an invariant
+of the definition, a library routine (torch's SDPA on the CPU in fp64), or
+brute force (the scalar restatement in oracle/scalar_reference.py).
+
+The same checks are run against deliberately broken copies of the oracle in
+test_oracle_mutations.py, to show that each plausible mistake is caught.
+"""
+
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+from _golden import floats, ints, load
+
+RNG = np.random.default_rng(12345)
+
+
+def _scalar():
+    import oracle.scalar_reference as sr
+    return sr
+
+
+# ---------------------------------------------------------------------------
+# Worked examples printed on the pages
+# ---------------------------------------------------------------------------
+
+def check_m1_six_token_tiles(o):
+    g = load("m1_causal_len6_tile2.txt")
+    n, t = int(g["length"]), int(g["tile"])
+    bm = o.block_mask({"kind": "causal"}, 1, 1, n, n, t, t)
+    grid = ["".join(r) for r in o.block_map(bm)]
+    assert grid == g["block_map"].split(), grid
+    flat = "".join(grid)
+    assert flat.count("F") == int(g["count_F"]) and flat.count("P") == int(g["count_P"])
+    assert flat.count("0") == int(g["count_0"])
+    vis = o.visible({"kind": "causal"}, 0, 0, o.query_positions(n, n), np.arange(n), n)
+    assert vis.size == int(g["pairs"]) and int(vis.sum()) == int(g["visible_pairs"])
+    visited = (flat.count("F") + flat.count("P")) * t * t
+    assert visited == int(g["visited_cells"])
+    hidden = 0
+    for mt, row in enumerate(grid):
+        for nt, c in enumerate(row):
+            if c != "0":
+                hidden += int((~vis[mt * t:(mt + 1) * t, nt * t:(nt + 1) * t]).sum())
+    assert hidden == int(g["masked_cells_in_visited_tiles"])
+
+
+def check_m6_packed_documents(o):
+    g = load("m6_packed_docs_len16_block4.txt")
+    n, blk = int(g["n"]), int(g["block"])
+    lens = ints(g["doc_lengths"])
+    doc = np.repeat(np.arange(len(lens)), lens)
+    for kind, key in (({"kind": "causal"}, "causal"), ({"kind": "document", "doc_id": doc}, "doc_causal")):
+        bm = o.block_mask(kind, 1, 1, n, n, blk, blk)
+        dense = ["".join("0" if c == "0" else "1" for c in row) for row in o.block_map(bm)]
+        assert dense == g[f"{key}_map"].split(), (key, dense)
+        assert abs(o.sparsity(bm) - float(g[f"{key}_sparsity"])) < 5e-3
+    # every visited tile of the document mask straddles a boundary or the diagonal
+    bm = o.block_mask({"kind": "document", "doc_id": doc}, 1, 1, n, n, blk, blk)
+    assert int(bm["full_kv_num_blocks"].sum()) == 0 and int(bm["kv_num_blocks"].sum()) == 7
+
+
+def check_m2_softcap_after_mask(o):
+    g = load("m2_softcap_trap.txt")
+    cap = float(g["cap"])
+    # two keys with raw score 0 (q = 0); the first query of a 2x2 causal
+    # attention sees key 0 only, as in the page's allow = [True, False]
+    q = np.zeros((1, 1, 2, 4))
+    k = RNG.standard_normal((1, 1, 2, 4))
+    v = np.eye(2).reshape(1, 1, 2, 2)
+    out, _ = o.forward(q, k, v, 0.5, {"kind": "causal"}, {"kind": "softcap", "cap": cap})
+    assert np.allclose(out[0, 0, 0], floats(g["correct"]), atol=0, rtol=0), out[0, 0, 0]
+    # the wrong order, written out here, reproduces the page's printed numbers
+    wrong = [cap * math.tanh(s / cap) for s in (0.0, -math.inf)]
+    mx = max(wrong)
+    w = [math.exp(x - mx) for x in wrong]
+    w = [x / sum(w) for x in w]
+    assert [round(x, 6) for x in w] == floats(g["incorrect_rounded6"])
+
+
+def check_m3_decode_offset(o):
+    g = load("m3_decode_offset.txt")
+    cap, valid, W = int(g["capacity"]), int(g["valid_length"]), int(g["window"])
+    qp = o.query_positions(1, valid)
+    assert int(qp[0]) == int(g["q_idx"]) + int(g["q_offset"])
+    vis = o.visible({"kind": "sliding_window", "window": W, "n_sink": 0}, 0, 0, qp, np.arange(cap), valid)
+    assert np.flatnonzero(vis[0]).tolist() == ints(g["visible"])
+
+
+def check_m4_bottom_right(o):
+    g = load("m4_bottom_right.txt")
+    L, S, E = int(g["L"]), int(g["S"]), int(g["E"])
+    q = np.ones((1, 1, L, E))
+    k = np.ones((1, 1, S, E))
+    v = np.eye(S).reshape(1, 1, S, S)
+    out, lse = o.forward(q, k, v, None, {"kind": "causal"}, None)
+    assert np.allclose(out[0, 0, 0], floats(g["bottom_right"]), atol=1e-15)
+    assert not np.allclose(out[0, 0, 0], floats(g["top_left"]))
+    assert abs(lse[0, 0, 0] - (E / math.sqrt(E) + math.log(S))) < 1e-12
+
+
+def check_m5_left_padding(o):
+    g = load("m5_left_padding.txt")
+    causal = np.tril(np.ones((3, 3), bool))
+    pad = np.array([True, False, False])
+    vis = causal & ~pad[None, :]
+    q = np.zeros((1, 1, 3, 2))
+    k = RNG.standard_normal((1, 1, 3, 2))
+    v = np.eye(3).reshape(1, 1, 3, 3)
+    out, lse = o.forward(q, k, v, 1.0, {"kind": "dense", "matrix": vis}, None)
+    assert np.allclose(out[0, 0, 1], floats(g["row1"]), atol=1e-15)
+    assert np.allclose(out[0, 0, 2], floats(g["row2"]), atol=1e-15)
+    # the library's convention for the fully masked row 0: zeros and -inf
+    assert np.all(out[0, 0, 0] == 0.0) and lse[0, 0, 0] == -np.inf
+    assert not np.isnan(out).any()
+
+
+# ---------------------------------------------------------------------------
+# Closed forms
+# ---------------------------------------------------------------------------
+
+def check_causal_block_fraction(o):
+    """(T+1)/2T of the tiles are computed ("Causal Mask" section 7)."""
+    for T in (1, 2, 3, 4, 16, 33):
+        bm = o.block_mask({"kind": "causal"}, 1, 1, 4 * T, 4 * T, 4, 4)
+        full = int(bm["full_kv_num_blocks"].sum())
+        part = int(bm["kv_num_blocks"].sum())
+        assert Fraction(full + part, T * T) == Fraction(T + 1, 2 * T)
+        assert part == T and full == T * (T - 1) // 2
+
+
+def check_window_count(o):
+    """Visible pairs of a causal window W: exact sum vs the page's W - W^2/2T.
+
+    "Attention expressions" (docs.tensorcad.dev), "What the engine does with
+    them": a causal window keeps W - W^2/2T keys per query on average once the
+    sequence outgrows it.  The exact mean is W - W^2/2T + W/2T; the page's
+    form is its continuum limit.
+    """
+    for T, W, n_sink in ((64, 16, 0), (257, 32, 0), (300, 40, 4), (129, 128, 3)):
+        vis = o.visible({"kind": "sliding_window", "window": W, "n_sink": n_sink}, 0, 0,
+                        o.query_positions(T, T), np.arange(T), T)
+        total = int(vis.sum())
+        exact = W * (W + 1) // 2 + (T - W) * W + sum(min(n_sink, q - W + 1) for q in range(W, T))
+        assert total == exact, (T, W, n_sink, total, exact)
+        if n_sink == 0:
+            mean = Fraction(total, T)
+            assert mean == Fraction(W) - Fraction(W * W, 2 * T) + Fraction(W, 2 * T)
+
+
+def check_single_visible_key(o):
+    """A row with one visible key returns that key's value; lse = its score."""
+    B, H, L, E = 1, 3, 9, 5
+    q = RNG.standard_normal((B, H, L, E))
+    k = RNG.standard_normal((B, H, L, E))
+    v = RNG.standard_normal((B, H, L, E))
+    score = {"kind": "cap_then_bias", "cap": 7.0, "slope_heads": 3, "pos": "global"}
+    out, lse = o.forward(q, k, v, 0.3, {"kind": "causal"}, score)
+    for h in range(H):
+        assert np.array_equal(out[0, h, 0], v[0, h, 0])
+        s = 0.3 * float(q[0, h, 0] @ k[0, h, 0])
+        assert abs(lse[0, h, 0] - 7.0 * math.tanh(s / 7.0)) < 1e-12
+    # first token of every packed document sees only itself
+    doc = np.array([0, 0, 1, 1, 1, 2, 2, 2, 2])
+    out, lse = o.forward(q, k, v, 0.3, {"kind": "document", "doc_id": doc}, None)
+    for start in (0, 2, 5):
+        assert np.array_equal(out[0, 1, start], v[0, 1, start])
+
+
+def check_equal_scores(o):
+    """q = 0: every visible key weighs the same; o = mean, lse = ln(count)."""
+    B, H, L, S, E = 2, 2, 7, 11, 3
+    q = np.zeros((B, H, L, E))
+    k = RNG.standard_normal((B, H, S, E))
+    v = RNG.standard_normal((B, H, S, 4))
+    kv_len = np.array([11, 8])
+    for mask in ({"kind": "causal"}, {"kind": "prefix_lm", "prefix": 3},
+                 {"kind": "sliding_window", "window": 3, "n_sink": 1}, {"kind": "chunked", "chunk": 4}):
+        out, lse = o.forward(q, k, v, 1.0, mask, None, kv_len=kv_len)
+        for b in range(B):
+            S_b = int(kv_len[b])
+            vis = o.visible(mask, b, 0, o.query_positions(L, S_b), np.arange(S), S_b)
+            for i in range(L):
+                n = int(vis[i].sum())
+                if n == 0:
+                    assert lse[b, 0, i] == -np.inf and np.all(out[b, 0, i] == 0)
+                    continue
+                assert np.allclose(out[b, 0, i], v[b, 0, vis[i]].mean(axis=0), atol=1e-13)
+                assert abs(lse[b, 0, i] - math.log(n)) < 1e-13
+
+
+def check_alibi_geometric(o):
+    """Equal raw scores under ALiBi: causal weights form a geometric sequence.
+
+    With g = -slope_h (q - kv), softmax over keys 0..i gives weights
+    proportional to e^{-slope_h (i - j)}: consecutive keys differ by the
+    factor e^{slope_h}, the nearest key weighs most ("flexattention-score-mod-
+    block-mask": the distance term biases far history negatively).  For 8
+    heads the slopes are 1/2, 1/4, ..., 1/256, the textbook ALiBi set.
+    """
+    H, L = 8, 6
+    q = np.zeros((1, H, L, 2))
+    k = RNG.standard_normal((1, H, L, 2))
+    v = np.eye(L)[None, None].repeat(H, axis=1)
+    out, _ = o.forward(q, k, v, 1.0, {"kind": "causal"}, {"kind": "alibi", "slope_heads": H})
+    for h in range(H):
+        w = out[0, h, L - 1]
+        ratio = w[1:] / w[:-1]
+        assert np.allclose(ratio, math.exp(2.0 ** -(h + 1)), rtol=1e-12), (h, ratio)
+
+
+def check_softcap_limits(o):
+    """c -> infinity: the soft-cap is the identity; a cap bounds scores in (-c, c)."""
+    q = RNG.standard_normal((1, 2, 6, 4))
+    k = RNG.standard_normal((1, 2, 6, 4))
+    v = RNG.standard_normal((1, 2, 6, 4))
+    a, la = o.forward(q, k, v, 2.0, {"kind": "causal"}, {"kind": "softcap", "cap": 1e9})
+    b, lb = o.forward(q, k, v, 2.0, {"kind": "causal"}, None)
+    assert np.allclose(a, b, atol=1e-12) and np.allclose(la, lb, atol=1e-12)
+    _, lc = o.forward(q * 50, k, v, 2.0, {"kind": "none"}, {"kind": "softcap", "cap": 1.5})
+    assert np.all(lc < 1.5 + math.log(6) + 1e-12)
+
+
+def check_cap_then_bias_order(o):
+    """cap-then-bias differs from bias-then-cap, and equals its two parts.
+
+    "flexattention-score-mod-block-mask", "score_mod changes the score":
+    c tanh(s/c) + a(p_j - p_i) is the rule; c tanh((s + a(p_j - p_i))/c) is
+    another.  With c -> infinity both reduce to ALiBi, and with a single
+    head of slope 2^-8 the bias part is tiny but nonzero.
+    """
+    q = RNG.standard_normal((1, 1, 5, 3)) * 3
+    k = RNG.standard_normal((1, 1, 5, 3)) * 3
+    v = RNG.standard_normal((1, 1, 5, 3))
+    big = o.forward(q, k, v, 1.0, {"kind": "causal"}, {"kind": "cap_then_bias", "cap": 1e9, "slope_heads": 1})
+    ali = o.forward(q, k, v, 1.0, {"kind": "causal"}, {"kind": "alibi", "slope_heads": 1})
+    assert np.allclose(big[0], ali[0], atol=1e-9) and np.allclose(big[1], ali[1], atol=1e-9)
+    # q = 0: g = slope (kv - q) exactly, whatever the cap
+    z = np.zeros_like(q)
+    _, l1 = o.forward(z, k, v, 1.0, {"kind": "none"}, {"kind": "cap_then_bias", "cap": 0.01, "slope_heads": 1})
+    i = np.arange(5)[:, None]
+    j = np.arange(5)[None, :]
+    ref = np.log(np.exp(2.0 ** -8 * (j - i)).sum(axis=1))
+    assert np.allclose(l1[0, 0], ref, atol=1e-13)
+
+
+def check_convex_combination(o):
+    """Each output is a convex combination of visible values; lse >= max score."""
+    B, H, L, S, E = 1, 2, 13, 17, 4
+    q = RNG.standard_normal((B, H, L, E))
+    k = RNG.standard_normal((B, H, S, E))
+    v = RNG.standard_normal((B, H, S, E))
+    mask = {"kind": "sliding_window", "window": 5, "n_sink": 2}
+    out, lse = o.forward(q, k, v, 0.5, mask, {"kind": "softcap", "cap": 2.0})
+    vis = o.visible(mask, 0, 0, o.query_positions(L, S), np.arange(S), S)
+    for h in range(H):
+        s = 2.0 * np.tanh(0.5 * (q[0, h] @ k[0, h].T) / 2.0)
+        for i in range(L):
+            vv = v[0, h, vis[i]]
+            assert np.all(out[0, h, i] >= vv.min(axis=0) - 1e-12)
+            assert np.all(out[0, h, i] <= vv.max(axis=0) + 1e-12)
+            assert lse[0, h, i] >= s[i, vis[i]].max() - 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Library routine and brute force
+# ---------------------------------------------------------------------------
+
+def check_against_torch_sdpa(o):
+    """No score rule + a boolean mask = torch's SDPA (CPU, fp64, explicit mask)."""
+    import torch
+    import torch.nn.functional as F
+    B, H, L, S, E = 2, 3, 19, 23, 8
+    q = RNG.standard_normal((B, H, L, E))
+    k = RNG.standard_normal((B, H, S, E))
+    v = RNG.standard_normal((B, H, S, 6))
+    kv_len = np.array([23, 20])
+    masks = ({"kind": "causal"}, {"kind": "sliding_window", "window": 6, "n_sink": 2},
+             {"kind": "prefix_lm", "prefix": 5}, {"kind": "chunked", "chunk": 7},
+             {"kind": "document", "doc_id": np.repeat(np.arange(4), [5, 9, 3, 6])}, {"kind": "none"})
+    for mask in masks:
+        out, lse = o.forward(q, k, v, 0.37, mask, None, kv_len=kv_len)
+        for b in range(B):
+            S_b = int(kv_len[b])
+            vis = o.visible(mask, b, 0, o.query_positions(L, S_b), np.arange(S), S_b)
+            live = vis.any(axis=1)
+            ref = F.scaled_dot_product_attention(
+                torch.from_numpy(q[b:b + 1, :, live]), torch.from_numpy(k[b:b + 1]),
+                torch.from_numpy(v[b:b + 1]), attn_mask=torch.from_numpy(vis[live]), scale=0.37)
+            assert np.allclose(out[b][:, live], ref[0].numpy(), atol=1e-12), mask["kind"]
+
+
+def _tiny_case(seed, L, S, E, Ev, B=2, Hq=2, Hkv=1):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((B, Hq, L, E)), r.standard_normal((B, Hkv, S, E)),
+            r.standard_normal((B, Hkv, S, Ev)))
+
+
+TINY_MASKS = (
+    {"kind": "none"}, {"kind": "causal"}, {"kind": "sliding_window", "window": 3, "n_sink": 1},
+    {"kind": "sliding_window", "window": 2, "n_sink": 0}, {"kind": "prefix_lm", "prefix": 2},
+    {"kind": "chunked", "chunk": 3}, {"kind": "document", "doc_id": [[0, 0, 0, 1, 1, 2, 2, 2], [0, 1, 1, 1, 1, 1, 2, 2]]},
+)
+TINY_SCORES = (
+    {"kind": "none"}, {"kind": "softcap", "cap": 1.5}, {"kind": "alibi", "slope_heads": 2},
+    {"kind": "cap_then_bias", "cap": 2.0, "slope_heads": 0, "pos": "global"},
+    {"kind": "cap_then_bias", "cap": 2.5, "slope_heads": 4, "pos": "in_doc",
+     "doc_id": [[0, 0, 0, 1, 1, 2, 2, 2], [0, 1, 1, 1, 1, 1, 2, 2]]},
+)
+
+
+def check_against_scalar_loops(o):
+    """numpy oracle == pure-Python triple loops on tiny shapes, every mask and score kind."""
+    sr = _scalar()
+    seed = 0
+    for mask in TINY_MASKS:
+        for score in TINY_SCORES:
+            for (L, S, kv_len) in ((8, 8, None), (3, 8, [8, 6]), (8, 8, [8, 5])):
+                seed += 1
+                q, k, v = _tiny_case(seed, L, S, 3, 2)
+                out, lse = o.forward(q, k, v, 0.7, mask, score, kv_len=kv_len, enable_gqa=True)
+                so, sl = sr.forward_scalar(q.tolist(), k.tolist(), v.tolist(), 0.7, mask, score, kv_len)
+                so, sl = np.array(so), np.array(sl)
+                assert np.allclose(out, so, atol=1e-12, rtol=0), (mask, score, L, S)
+                fin = np.isfinite(sl)
+                assert np.array_equal(fin, np.isfinite(lse)) and np.allclose(lse[fin], sl[fin], atol=1e-12)
+
+
+def check_block_mask_against_scalar(o):
+    """Oracle tile classes == a cell-by-cell scalar visit, ragged shapes included."""
+    sr = _scalar()
+    doc = [0] * 7 + [1] * 3 + [2] * 11 + [3] * 2
+    cases = [({"kind": "causal"}, 23, 23, 4, 4, None), ({"kind": "causal"}, 9, 23, 4, 8, [23]),
+             ({"kind": "sliding_window", "window": 5, "n_sink": 2}, 23, 23, 4, 3, None),
+             ({"kind": "prefix_lm", "prefix": 6}, 23, 23, 8, 4, None),
+             ({"kind": "chunked", "chunk": 6}, 23, 23, 4, 4, None),
+             ({"kind": "document", "doc_id": doc}, 23, 23, 4, 4, None),
+             ({"kind": "none"}, 5, 23, 2, 8, [17]), ({"kind": "causal"}, 23, 19, 8, 8, [11])]
+    for mask, L, S, BM, BN, kv_len in cases:
+        bm = o.block_mask(mask, 1, 1, L, S, BM, BN, kv_len=kv_len)
+        ref = sr.tile_classes_scalar(mask, L, S, BM, BN, 0, kv_len)
+        assert o.block_map(bm) == ref, (mask, L, S, BM, BN)
+        # ordering and padding convention
+        for mt in range(bm["Mb"]):
+            for name, cnt in (("kv_indices", "kv_num_blocks"), ("full_kv_indices", "full_kv_num_blocks")):
+                n = int(bm[cnt][0, 0, mt])
+                idx = bm[name][0, 0, mt]
+                assert list(idx[:n]) == sorted(idx[:n]) and np.all(idx[n:] == 0)
+
+
+def check_split_combine(o):
+    """Split-KV partials merged by lse weights equal the unsplit result."""
+    L, S, E = 6, 40, 5
+    q, k, v = _tiny_case(7, L, S, E, 3, B=1, Hq=1, Hkv=1)
+    mask = {"kind": "causal"}
+    score = {"kind": "softcap", "cap": 3.0}
+    qp = o.query_positions(L, S)
+    full_o, full_l = o.attention_rows(q[0, 0], k[0, 0], v[0, 0], 0.4, mask, score, 0, 0, qp, S, 1)
+    for bounds in ([0, 40], [0, 13, 40], [0, 1, 2, 17, 36, 40], [0, 10, 20, 30, 40]):
+        parts = o.split_partials(q[0, 0], k[0, 0], v[0, 0], 0.4, mask, score, 0, 0, qp, S, 1, bounds)
+        co, cl = o.combine(parts)
+        assert np.allclose(co, full_o, atol=1e-12) and np.allclose(cl, full_l, atol=1e-12)
+
+
+def check_gqa_is_broadcast(o):
+    """GQA equals explicitly repeating each KV head for its group of query heads."""
+    q, k, v = _tiny_case(3, 5, 7, 4, 3, B=1, Hq=6, Hkv=2)
+    a = o.forward(q, k, v, 0.5, {"kind": "causal"}, {"kind": "alibi"}, enable_gqa=True)
+    b = o.forward(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), 0.5, {"kind": "causal"}, {"kind": "alibi"})
+    assert np.allclose(a[0], b[0], atol=1e-14) and np.allclose(a[1], b[1], atol=1e-14)
+
+
+def check_workload_tile_counts(o):
+    """Tile counts of the causal 2048/128 and window+sink 16384/128 workloads.
+
+    Causal with T tiles per side: T(T+1)/2 visited, T(T-1)/2 full, T partial.
+    Window W=1024 with 4 sinks, tiles of 128: counted here tile by tile from
+    the interval of keys each query row sees (not cell by cell).
+    """
+    bm = o.block_mask({"kind": "causal"}, 1, 1, 2048, 2048, 128, 128)
+    assert int(bm["full_kv_num_blocks"].sum()) == 120 and int(bm["kv_num_blocks"].sum()) == 16
+    T, W, ns, t = 16384, 1024, 4, 128
+    nb = T // t
+    full = part = 0
+    for m in range(nb):
+        rows = np.arange(m * t, (m + 1) * t)
+        lo = np.maximum(rows - W + 1, 0)
+        for n in range(nb):
+            c0, c1 = n * t, (n + 1) * t - 1
+            win = np.clip(np.minimum(rows, c1) - np.maximum(lo, c0) + 1, 0, None)
+            sink_hi = np.minimum(ns - 1, np.minimum(rows, c1))
+            sink = np.clip(np.minimum(sink_hi, lo - 1) - c0 + 1, 0, None)
+            cnt = win + sink
+            if np.all(cnt == t):
+                full += 1
+            elif np.any(cnt > 0):
+                part += 1
+    assert (full, part) == (868, 367), (full, part)
+    bm = o.block_mask({"kind": "sliding_window", "window": W, "n_sink": ns}, 1, 1, T, T, t, t)
+    assert int(bm["full_kv_num_blocks"].sum()) == full and int(bm["kv_num_blocks"].sum()) == part
+
+
+ALL_CHECKS = [
+    check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
+    check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
+    check_causal_block_fraction, check_window_count, check_single_visible_key, check_equal_scores,
+    check_alibi_geometric, check_softcap_limits, check_cap_then_bias_order, check_convex_combination,
+    check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
+    check_split_combine, check_gqa_is_broadcast,
+]
+SLOW_CHECKS = [check_workload_tile_counts]

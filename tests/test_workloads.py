@@ -1,0 +1,49 @@
+"""The seeded input recipes produce the documented shapes and draws."""
+import numpy as np
+import torch
+
+import workloads as w
+
+
+def test_packed_doc_lengths_seed0():
+    lens = w.doc_lengths(8192, 128, 2048, seed=0)
+    assert lens == [1762, 1351, 1109, 646, 719, 206, 272, 159, 464, 1504]
+    assert sum(lens) == 8192
+    ids = w.doc_ids_from_lengths(lens)
+    pos = w.in_doc_positions(lens)
+    assert ids.shape == (8192,) and pos.shape == (8192,)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    assert np.all(pos[starts] == 0) and np.all(np.diff(ids) >= 0)
+
+
+def test_decode_cache_lengths_seed0():
+    lens = w.decode_cache_lengths(32, 4096, 32768, seed=0)
+    assert lens.dtype == np.int32 and lens.shape == (32,)
+    assert int(lens.sum()) == 614602
+    assert lens.min() >= 4096 and lens.max() <= 32768
+
+
+def test_qkv_draw_order_and_cast():
+    q, k, v = w.randn_qkv(1, 2, 1, 3, 5, 4, 6, seed=0, dtype=torch.float32)
+    g = torch.Generator("cpu").manual_seed(0)
+    q2 = torch.randn((1, 2, 3, 4), generator=g)
+    k2 = torch.randn((1, 1, 5, 4), generator=g)
+    v2 = torch.randn((1, 1, 5, 6), generator=g)
+    assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
+    qb, _, _ = w.randn_qkv(1, 2, 1, 3, 5, 4, 6, seed=0, dtype=torch.bfloat16)
+    assert torch.equal(qb, q2.to(torch.bfloat16))
+
+
+def test_cache_tail_sentinels():
+    k = torch.zeros(2, 1, 8, 2)
+    v = torch.zeros(2, 1, 8, 2)
+    w.fill_cache_tail(k, v, np.array([8, 5]))
+    assert torch.all(k[0] == 0) and torch.all(k[1, :, 5:] == 1e4) and torch.all(v[1, :, 5:] == -1e4)
+    assert torch.all(k[1, :, :5] == 0)
+
+
+def test_configs_are_complete():
+    for name, c in w.CONFIGS.items():
+        for key in ("B", "Hq", "Hkv", "L", "S", "E", "Ev", "dtype", "seed", "scale", "BM", "BN", "mask", "score"):
+            assert key in c, (name, key)
+        assert c["Hq"] % c["Hkv"] == 0
