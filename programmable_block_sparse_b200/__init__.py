@@ -1,0 +1,232 @@
+"""B200 (sm_100a) FlexAttention forward: Python binding of ``libflexattn_b200.so``.
+
+The functions here carry the C entry points' names and only marshal
+arguments: torch tensors become device pointers, sizes and strides; mask and
+score specifications (plain dicts) become the C structs.  Every step of the
+computation runs in the CUDA library; there is no CPU fallback -- importing
+works without the library, but any call raises if it is not built.
+
+Specification dicts (the menu of include/flexattn.h):
+
+* mask_mod: ``{"kind": "none" | "causal" | "sliding_window" | "document" |
+  "prefix_lm" | "chunked", "window": W, "n_sink": n, "prefix": P,
+  "chunk": C, "doc_id": int32 tensor (B or 1, S), "kv_len": int32 tensor (B,)}``
+* score_mod: ``{"kind": "none" | "softcap" | "alibi" | "cap_then_bias",
+  "cap": c, "slope_heads": H, "pos": int32 tensor (B or 1, S) or None}``
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+from dataclasses import dataclass
+
+from . import _abi
+
+__all__ = [
+    "BlockMask", "FlexAttnError", "library_path", "load_library",
+    "flexattn_version", "flexattn_last_error", "flexattn_block_mask_dims", "flexattn_build_block_mask",
+    "flexattn_forward_workspace_size", "flexattn_forward", "flexattn_poll_device_status",
+]
+
+_LIB = None
+_PKG = os.path.dirname(os.path.abspath(__file__))
+
+
+class FlexAttnError(RuntimeError):
+    """A non-zero status from the library; ``.status`` holds the code."""
+
+    def __init__(self, status, message):
+        self.status = status
+        super().__init__(f"{_abi.STATUS_NAMES.get(status, status)}: {message}")
+
+
+def library_path():
+    return os.path.join(_PKG, "libflexattn_b200.so")
+
+
+def load_library():
+    """Load the CUDA library (built in-tree by ``build.py``); raise if it is missing."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is not built: run `python -m programmable_block_sparse_b200.build` "
+                "(the CUDA library is required; there is no fallback)")
+        _LIB = _abi.bind(C.CDLL(path))
+    return _LIB
+
+
+def _check(status):
+    if status != _abi.FA_OK:
+        raise FlexAttnError(status, load_library().flexattn_last_error().decode())
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return C.c_void_p(stream)
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _tensor_struct(t):
+    import torch
+    if t.dim() != 4:
+        raise FlexAttnError(2, f"expected a 4-D tensor (B, H, N, D), got shape {tuple(t.shape)}")
+    if t.dtype == torch.bfloat16:
+        dt = _abi.FA_DTYPE_BF16
+    elif t.dtype == torch.float32:
+        dt = _abi.FA_DTYPE_F32
+    else:
+        raise FlexAttnError(6, f"unsupported dtype {t.dtype}")
+    s = _abi.fa_tensor()
+    s.data = t.data_ptr()
+    s.dtype = dt
+    s.reserved = 0
+    for i in range(4):
+        s.size[i] = t.shape[i]
+        s.stride[i] = t.stride(i)
+    return s
+
+
+def _mask_struct(spec):
+    spec = spec or {"kind": "none"}
+    m = _abi.fa_mask_mod()
+    m.kind = _abi.MASK_KIND[spec["kind"]]
+    m.window = int(spec.get("window", 0))
+    m.n_sink = int(spec.get("n_sink", 0))
+    m.prefix = int(spec.get("prefix", 0))
+    m.chunk = int(spec.get("chunk", 0))
+    doc = spec.get("doc_id")
+    if doc is not None:
+        m.doc_id = doc.data_ptr()
+        m.doc_batch = doc.shape[0] if doc.dim() == 2 else 1
+    kv_len = spec.get("kv_len")
+    if kv_len is not None:
+        m.kv_len = kv_len.data_ptr()
+    return m
+
+
+def _score_struct(spec):
+    spec = spec or {"kind": "none"}
+    s = _abi.fa_score_mod()
+    s.kind = _abi.SCORE_KIND[spec["kind"]]
+    s.cap = float(spec.get("cap", 0.0))
+    s.slope_heads = int(spec.get("slope_heads", 0) or 0)
+    pos = spec.get("pos")
+    if pos is not None and not isinstance(pos, str):
+        s.pos = pos.data_ptr()
+        s.pos_batch = pos.shape[0] if pos.dim() == 2 else 1
+    return s
+
+
+@dataclass
+class BlockMask:
+    """Device-resident BlockMask: the four int32 arrays and their extents."""
+
+    B: int
+    H: int
+    L: int
+    S: int
+    BM: int
+    BN: int
+    Mb: int
+    Nb: int
+    kv_num_blocks: object
+    kv_indices: object
+    full_kv_num_blocks: object
+    full_kv_indices: object
+
+    def as_struct(self):
+        s = _abi.fa_block_mask()
+        s.B, s.H, s.L, s.S, s.BM, s.BN, s.Mb, s.Nb = (self.B, self.H, self.L, self.S, self.BM, self.BN,
+                                                      self.Mb, self.Nb)
+        s.kv_num_blocks = self.kv_num_blocks.data_ptr()
+        s.kv_indices = self.kv_indices.data_ptr()
+        s.full_kv_num_blocks = self.full_kv_num_blocks.data_ptr()
+        s.full_kv_indices = self.full_kv_indices.data_ptr()
+        return s
+
+
+def flexattn_version():
+    return load_library().flexattn_version()
+
+
+def flexattn_last_error():
+    return load_library().flexattn_last_error().decode()
+
+
+def flexattn_block_mask_dims(L, S, BM, BN):
+    mb, nb = C.c_int32(), C.c_int32()
+    _check(load_library().flexattn_block_mask_dims(L, S, BM, BN, C.byref(mb), C.byref(nb)))
+    return mb.value, nb.value
+
+
+def flexattn_build_block_mask(mask_mod, B, H, L, S, BM=128, BN=128, device="cuda", stream=None, out=None):
+    """Allocate the BlockMask arrays on ``device`` and classify every tile on the GPU."""
+    import torch
+    Mb, Nb = flexattn_block_mask_dims(L, S, BM, BN)
+    if out is None:
+        z = dict(dtype=torch.int32, device=device)
+        out = BlockMask(B, H, L, S, BM, BN, Mb, Nb, torch.empty((B, H, Mb), **z), torch.empty((B, H, Mb, Nb), **z),
+                        torch.empty((B, H, Mb), **z), torch.empty((B, H, Mb, Nb), **z))
+    m = _mask_struct(mask_mod)
+    bm = out.as_struct()
+    _check(load_library().flexattn_build_block_mask(C.byref(m), C.byref(bm), _stream_handle(stream)))
+    return out
+
+
+def flexattn_forward_workspace_size(q, k, v, block_mask, split_kv=0):
+    n = C.c_size_t()
+    qs, ks, vs, bm = _tensor_struct(q), _tensor_struct(k), _tensor_struct(v), block_mask.as_struct()
+    _check(load_library().flexattn_forward_workspace_size(C.byref(qs), C.byref(ks), C.byref(vs), C.byref(bm),
+                                                          int(split_kv), C.byref(n)))
+    return n.value
+
+
+def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=None, enable_gqa=False,
+                     out=None, lse=True, split_kv=0, workspace=None, stream=None):
+    """Run the forward pass; returns ``(out, lse)`` (lse None when ``lse=False``).
+
+    ``out`` / ``lse`` may be preallocated tensors; ``workspace`` a uint8 device
+    tensor of at least :func:`flexattn_forward_workspace_size` bytes (allocated
+    here when None and needed).
+    """
+    import torch
+    B, Hq, L, _ = q.shape
+    Ev = v.shape[3]
+    if out is None:
+        out = torch.empty((B, Hq, L, Ev), dtype=q.dtype, device=q.device)
+    if lse is True:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    ws_bytes = flexattn_forward_workspace_size(q, k, v, block_mask, split_kv)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    qs, ks, vs, os_ = _tensor_struct(q), _tensor_struct(k), _tensor_struct(v), _tensor_struct(out)
+    bm = block_mask.as_struct()
+    sm, mm = _score_struct(score_mod), _mask_struct(mask_mod)
+    sc = 0.0 if scale is None else float(scale)
+    if math.isnan(sc):
+        sc = 0.0
+    _check(load_library().flexattn_forward(
+        C.byref(qs), C.byref(ks), C.byref(vs), C.byref(os_), _ptr(lse), C.c_float(sc), int(bool(enable_gqa)),
+        C.byref(sm), C.byref(mm), C.byref(bm), int(split_kv), _ptr(workspace),
+        C.c_size_t(workspace.numel() if workspace is not None else 0), _stream_handle(stream)))
+    return out, lse
+
+
+def flexattn_poll_device_status(stream=None):
+    """Synchronise ``stream`` and return (and clear) the kernels' device status code."""
+    st = C.c_int32()
+    _check(load_library().flexattn_poll_device_status(_stream_handle(stream), C.byref(st)))
+    return st.value

@@ -1,0 +1,368 @@
+// C ABI layer: argument checks, TMA descriptor encoding and kernel choice.
+// Declarations and the contract of every entry point are in include/flexattn.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace fa {
+
+// First error a kernel recorded since the last flexattn_poll_device_status.
+__device__ int g_device_status = 0;
+
+namespace {
+
+// Device address of g_device_status for the current device (looked up once
+// per device; the CUDA runtime loads this module's globals per context).
+int* status_word(int* err) {
+  static int* cache[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  *err = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *err = 1;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+      *err = 1;
+      return nullptr;
+    }
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+thread_local std::string t_last_error;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ----------------------------------------------------------------------------
+// Parameter checks shared by the build and forward calls.
+// ----------------------------------------------------------------------------
+int check_mask_params(const fa_mask_mod* m, int batch) {
+  switch (m->kind) {
+    case FA_MASK_NONE:
+    case FA_MASK_CAUSAL:
+      break;
+    case FA_MASK_SLIDING_WINDOW:
+      if (m->window < 1) return fail(FA_ERR_PARAM, "sliding window needs window >= 1 (got %d)", m->window);
+      if (m->n_sink < 0) return fail(FA_ERR_PARAM, "sliding window needs n_sink >= 0 (got %d)", m->n_sink);
+      break;
+    case FA_MASK_DOCUMENT:
+      if (m->doc_id == nullptr) return fail(FA_ERR_PARAM, "document mask needs doc_id");
+      if (m->doc_batch != 1 && m->doc_batch != batch)
+        return fail(FA_ERR_BATCH, "doc_batch must be 1 or %d (got %d)", batch, m->doc_batch);
+      break;
+    case FA_MASK_PREFIX_LM:
+      if (m->prefix < 0) return fail(FA_ERR_PARAM, "prefix-LM needs prefix >= 0 (got %d)", m->prefix);
+      break;
+    case FA_MASK_CHUNKED:
+      if (m->chunk < 1) return fail(FA_ERR_PARAM, "chunked mask needs chunk >= 1 (got %d)", m->chunk);
+      break;
+    default:
+      return fail(FA_ERR_PARAM, "unknown mask kind %d", m->kind);
+  }
+  return FA_OK;
+}
+
+int check_score_params(const fa_score_mod* s, int batch) {
+  switch (s->kind) {
+    case FA_SCORE_NONE:
+      break;
+    case FA_SCORE_SOFTCAP:
+    case FA_SCORE_CAP_THEN_BIAS:
+      if (!(s->cap > 0.0f) || isinf(s->cap)) return fail(FA_ERR_PARAM, "cap must be finite and > 0 (got %g)", s->cap);
+      // fallthrough
+    case FA_SCORE_ALIBI:
+      if (s->slope_heads < 0) return fail(FA_ERR_PARAM, "slope_heads must be >= 0 (got %d)", s->slope_heads);
+      if (s->kind == FA_SCORE_CAP_THEN_BIAS && s->pos != nullptr && s->pos_batch != 1 && s->pos_batch != batch)
+        return fail(FA_ERR_BATCH, "pos_batch must be 1 or %d (got %d)", batch, s->pos_batch);
+      break;
+    default:
+      return fail(FA_ERR_PARAM, "unknown score kind %d", s->kind);
+  }
+  return FA_OK;
+}
+
+int check_block_mask_dims(const fa_block_mask* bm) {
+  if (bm->L < 1 || bm->S < 1) return fail(FA_ERR_SHAPE, "block mask lengths must be >= 1 (L=%d, S=%d)", bm->L, bm->S);
+  if (bm->BM < 1 || bm->BM > 128 || bm->BN < 1 || bm->BN > 128)
+    return fail(FA_ERR_SHAPE, "block sizes must be in 1..128 (BM=%d, BN=%d)", bm->BM, bm->BN);
+  if (bm->B < 1 || bm->H < 1) return fail(FA_ERR_SHAPE, "block mask B and H must be >= 1");
+  if (bm->Mb != ceil_div(bm->L, bm->BM) || bm->Nb != ceil_div(bm->S, bm->BN))
+    return fail(FA_ERR_MASK_SHAPE, "block mask grid %dx%d does not match ceil(L/BM) x ceil(S/BN) = %dx%d", bm->Mb,
+                bm->Nb, ceil_div(bm->L, bm->BM), ceil_div(bm->S, bm->BN));
+  if (!bm->kv_num_blocks || !bm->kv_indices || !bm->full_kv_num_blocks || !bm->full_kv_indices)
+    return fail(FA_ERR_NULL, "block mask arrays must not be NULL");
+  return FA_OK;
+}
+
+MaskParams to_device(const fa_mask_mod* m) {
+  MaskParams p;
+  p.kind = m->kind;
+  p.window = m->window;
+  p.n_sink = m->n_sink;
+  p.prefix = m->prefix;
+  p.chunk = m->chunk;
+  p.doc_batch = m->doc_batch;
+  p.doc_id = m->doc_id;
+  p.kv_len = m->kv_len;
+  return p;
+}
+
+ScoreParams to_device(const fa_score_mod* s) {
+  ScoreParams p;
+  p.kind = s->kind;
+  p.cap = s->cap;
+  p.slope_heads = s->slope_heads;
+  p.pos_batch = s->pos_batch;
+  p.pos = s->kind == FA_SCORE_CAP_THEN_BIAS ? s->pos : nullptr;
+  return p;
+}
+
+// ----------------------------------------------------------------------------
+// TMA descriptors
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// (B, H, N, D) bf16 tensor -> 4-D map with a 64 x box_rows box, 128 B swizzle.
+int encode_bf16_map(CUtensorMap* map, const fa_tensor* t, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(t->size[3]), static_cast<cuuint64_t>(t->size[2]),
+                        static_cast<cuuint64_t>(t->size[1]), static_cast<cuuint64_t>(t->size[0])};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(t->stride[2]) * 2, static_cast<cuuint64_t>(t->stride[1]) * 2,
+                           static_cast<cuuint64_t>(t->stride[0]) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_ALIGN, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return FA_OK;
+}
+
+// ----------------------------------------------------------------------------
+// Forward argument checks -> FwdArgs
+// ----------------------------------------------------------------------------
+enum class Path { kSimt, kSm100, kDecode };
+
+int check_tensor(const fa_tensor* t, const char* name) {
+  if (t == nullptr || t->data == nullptr) return fail(FA_ERR_NULL, "%s is NULL", name);
+  if (t->dtype != FA_DTYPE_BF16 && t->dtype != FA_DTYPE_F32) return fail(FA_ERR_DTYPE, "%s: unknown dtype %d", name, t->dtype);
+  if (t->reserved != 0) return fail(FA_ERR_PARAM, "%s: reserved field must be 0", name);
+  for (int i = 0; i < 4; ++i)
+    if (t->size[i] < 1 || t->size[i] > INT32_MAX) return fail(FA_ERR_SHAPE, "%s: size[%d] = %lld out of range", name, i, (long long)t->size[i]);
+  if (t->stride[3] != 1) return fail(FA_ERR_ALIGN, "%s: the last dimension must be contiguous (stride %lld)", name, (long long)t->stride[3]);
+  for (int i = 0; i < 3; ++i)
+    if (t->stride[i] < 0) return fail(FA_ERR_ALIGN, "%s: negative stride", name);
+  return FA_OK;
+}
+
+bool aligned16(const fa_tensor* t) {
+  const int es = t->dtype == FA_DTYPE_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(t->data) % 16) return false;
+  for (int i = 0; i < 3; ++i)
+    if ((t->stride[i] * es) % 16) return false;
+  return true;
+}
+
+int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out, float scale,
+            int32_t enable_gqa, const fa_score_mod* score, const fa_mask_mod* mask, const fa_block_mask* bm,
+            int32_t split_kv, FwdArgs* a, Path* path) {
+  int rc;
+  if ((rc = check_tensor(q, "q")) || (rc = check_tensor(k, "k")) || (rc = check_tensor(v, "v"))) return rc;
+  if (out != nullptr && (rc = check_tensor(out, "out"))) return rc;
+  if (!score || !mask || !bm) return fail(FA_ERR_NULL, "score_mod, mask_mod and block_mask must not be NULL");
+  if (k->dtype != q->dtype || v->dtype != q->dtype) return fail(FA_ERR_DTYPE, "q, k and v must share one dtype");
+  if (out && out->dtype != q->dtype) return fail(FA_ERR_DTYPE, "out must have the dtype of q");
+  const int B = (int)q->size[0], Hq = (int)q->size[1], L = (int)q->size[2], E = (int)q->size[3];
+  const int Hkv = (int)k->size[1], S = (int)k->size[2], Ev = (int)v->size[3];
+  if (k->size[0] != B || v->size[0] != B) return fail(FA_ERR_BATCH, "q, k and v must have the same batch size");
+  if (k->size[3] != E) return fail(FA_ERR_SHAPE, "k head dim %lld != q head dim %d", (long long)k->size[3], E);
+  if (v->size[1] != Hkv || v->size[2] != S) return fail(FA_ERR_SHAPE, "v must be (B, Hkv, S, Ev) like k");
+  if (out && (out->size[0] != B || out->size[1] != Hq || out->size[2] != L || out->size[3] != Ev))
+    return fail(FA_ERR_SHAPE, "out must be (B, Hq, L, Ev)");
+  if (Hq != Hkv) {
+    if (!enable_gqa) return fail(FA_ERR_HEADS, "Hq (%d) != Hkv (%d): set enable_gqa", Hq, Hkv);
+    if (Hq % Hkv) return fail(FA_ERR_HEADS, "GQA needs Hq %% Hkv == 0 (Hq=%d, Hkv=%d)", Hq, Hkv);
+  }
+  if (E > 128 || Ev > 128) return fail(FA_ERR_HEADDIM, "head dims above 128 are not supported (E=%d, Ev=%d)", E, Ev);
+  if ((rc = check_block_mask_dims(bm))) return rc;
+  if (bm->L != L || bm->S != S)
+    return fail(FA_ERR_MASK_SHAPE, "block mask is for L=%d, S=%d but the call has L=%d, S=%d (%s)", bm->L, bm->S, L, S,
+                (bm->L < L || bm->S < S) ? "too small" : "too large");
+  if (bm->B != 1 && bm->B != B) return fail(FA_ERR_BATCH, "block mask batch %d is neither 1 nor %d", bm->B, B);
+  if (bm->H != 1 && bm->H != Hq) return fail(FA_ERR_MASK_SHAPE, "block mask heads %d is neither 1 nor %d", bm->H, Hq);
+  if (mask->kv_len && bm->B != B)
+    return fail(FA_ERR_BATCH, "with per-sequence kv_len the block mask needs batch %d (has %d)", B, bm->B);
+  if ((rc = check_mask_params(mask, B)) || (rc = check_score_params(score, B))) return rc;
+
+  *a = FwdArgs{};
+  a->q = q->data;
+  a->k = k->data;
+  a->v = v->data;
+  a->out = out ? out->data : nullptr;
+  for (int i = 0; i < 4; ++i) {
+    a->q_stride[i] = q->stride[i];
+    a->k_stride[i] = k->stride[i];
+    a->v_stride[i] = v->stride[i];
+    a->o_stride[i] = out ? out->stride[i] : 0;
+  }
+  a->B = B;
+  a->Hq = Hq;
+  a->Hkv = Hkv;
+  a->L = L;
+  a->S = S;
+  a->E = E;
+  a->Ev = Ev;
+  a->G = Hq / Hkv;
+  a->dtype = q->dtype;
+  a->scale = (scale > 0.0f && !isinf(scale)) ? scale : 1.0f / sqrtf(static_cast<float>(E));
+  a->mask = to_device(mask);
+  a->score = to_device(score);
+  a->bm = BlockMaskView{bm->B, bm->H, bm->Mb, bm->Nb, bm->BM, bm->BN, bm->kv_num_blocks, bm->kv_indices,
+                        bm->full_kv_num_blocks, bm->full_kv_indices};
+
+  const bool tc_shape = q->dtype == FA_DTYPE_BF16 && E == Ev && (E == 64 || E == 128);
+  const bool tma_ok = aligned16(q) && aligned16(k) && aligned16(v);
+  if (split_kv < 0) return fail(FA_ERR_PARAM, "split_kv must be >= 0");
+  if (split_kv > 1 && !(tc_shape && L <= 16 && bm->Mb == 1))
+    return fail(FA_ERR_UNSUPPORTED, "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16 and one query tile");
+  *path = Path::kSimt;
+  (void)tma_ok;
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int flexattn_version(void) { return 100; }
+
+const char* flexattn_last_error(void) { return t_last_error.c_str(); }
+
+int flexattn_block_mask_dims(int32_t L, int32_t S, int32_t BM, int32_t BN, int32_t* Mb, int32_t* Nb) {
+  if (!Mb || !Nb) return fail(FA_ERR_NULL, "Mb and Nb must not be NULL");
+  if (L < 1 || S < 1) return fail(FA_ERR_SHAPE, "L and S must be >= 1");
+  if (BM < 1 || BM > 128 || BN < 1 || BN > 128) return fail(FA_ERR_SHAPE, "BM and BN must be in 1..128");
+  *Mb = ceil_div(L, BM);
+  *Nb = ceil_div(S, BN);
+  return FA_OK;
+}
+
+int flexattn_build_block_mask(const fa_mask_mod* mask_mod, const fa_block_mask* bm, void* stream) {
+  if (!mask_mod || !bm) return fail(FA_ERR_NULL, "mask_mod and block_mask must not be NULL");
+  int rc;
+  if ((rc = check_block_mask_dims(bm))) return rc;
+  if ((rc = check_mask_params(mask_mod, bm->B))) return rc;
+  ClassifyArgs a;
+  int serr = 0;
+  a.status = status_word(&serr);
+  if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
+  a.mask = to_device(mask_mod);
+  a.B = bm->B;
+  a.H = bm->H;
+  a.L = bm->L;
+  a.S = bm->S;
+  a.BM = bm->BM;
+  a.BN = bm->BN;
+  a.Mb = bm->Mb;
+  a.Nb = bm->Nb;
+  a.kv_num_blocks = bm->kv_num_blocks;
+  a.kv_indices = bm->kv_indices;
+  a.full_kv_num_blocks = bm->full_kv_num_blocks;
+  a.full_kv_indices = bm->full_kv_indices;
+  cudaError_t e = launch_classify(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block-mask classifier launch");
+  return FA_OK;
+}
+
+int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
+                                    const fa_block_mask* block_mask, int32_t split_kv, size_t* bytes) {
+  if (!bytes) return fail(FA_ERR_NULL, "bytes must not be NULL");
+  fa_score_mod none_score{FA_SCORE_NONE, 0.0f, 0, 0, nullptr};
+  fa_mask_mod none_mask{FA_MASK_NONE, 0, 0, 0, 0, 0, nullptr, nullptr};
+  FwdArgs a;
+  Path path;
+  int rc = prepare(q, k, v, nullptr, 0.0f, 1, &none_score, &none_mask, block_mask, split_kv, &a, &path);
+  if (rc) return rc;
+  *bytes = 0;
+  return FA_OK;
+}
+
+int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out, float* lse,
+                     float scale, int32_t enable_gqa, const fa_score_mod* score_mod, const fa_mask_mod* mask_mod,
+                     const fa_block_mask* block_mask, int32_t split_kv, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (!out) return fail(FA_ERR_NULL, "out is NULL");
+  FwdArgs a;
+  Path path;
+  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
+  if (rc) return rc;
+  (void)workspace;
+  (void)workspace_bytes;
+  int serr = 0;
+  a.status = status_word(&serr);
+  if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
+  a.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_fwd_simt(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return FA_OK;
+}
+
+int flexattn_poll_device_status(void* stream, int32_t* status) {
+  if (!status) return fail(FA_ERR_NULL, "status must not be NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e == cudaSuccess && v != 0) e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  *status = v;
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,213 @@
+// BlockMask construction on the GPU: classify every (b, m, n) tile as empty,
+// full or partial and write the ordered index lists.
+//
+// What is computed follows "PyTorch Flex Attention complete guide" (2kiu.com)
+// sections 3.1 (a block counts as sparse only when every element in it is
+// masked), 3.2 (ordered per-row index lists) and 4.1 (dense mask, per-block
+// reduction, full blocks kept apart from partial ones), and the tile classes of
+// "flexattention-score-mod-block-mask" (charlestar.github.io), section
+// "mask_mod defines legal connections, BlockMask defines block work".
+//
+// How: no dense (L, S) temporary.  One CTA per (b, m) row of tiles; each warp
+// classifies whole tiles.  For the interval-shaped rules (none, causal,
+// sliding window with sinks, prefix-LM, chunked) every query row sees a union
+// of at most two key intervals, so a tile is classified from per-row
+// intersection counts (BM work per tile instead of BM x BN).  The document
+// rule is checked cell by cell with a warp-wide early exit once both a
+// visible and a hidden cell are seen, after a sound shortcut: a tile whose row
+// and column document-id ranges are disjoint has no visible cell.
+#include "common.cuh"
+#include "launch.h"
+#include "mods.cuh"
+
+namespace fa {
+
+namespace {
+
+constexpr int kClassifyThreads = 256;
+enum : uint8_t { kEmpty = 0, kPartial = 1, kFull = 2 };
+
+// |[lo, hi] intersect [c0, c1]| for inclusive bounds.
+__device__ __forceinline__ int overlap(int lo, int hi, int c0, int c1) {
+  int a = lo > c0 ? lo : c0;
+  int b = hi < c1 ? hi : c1;
+  return b >= a ? b - a + 1 : 0;
+}
+
+// Number of visible keys in [c0, c1] (inclusive, c1 < S) for logical query q.
+__device__ __forceinline__ int visible_count(const MaskParams& m, int q, int c0, int c1, int S_b) {
+  const int last = S_b - 1;  // keys beyond the valid length are hidden
+  int hi = c1 < last ? c1 : last;
+  if (hi < c0) return 0;
+  switch (m.kind) {
+    case FA_MASK_NONE:
+      return hi - c0 + 1;
+    case FA_MASK_CAUSAL:
+      return q < 0 ? 0 : overlap(0, q, c0, hi);
+    case FA_MASK_SLIDING_WINDOW: {
+      if (q < 0) return 0;
+      int wlo = q - m.window + 1;
+      wlo = wlo < 0 ? 0 : wlo;
+      int win = overlap(wlo, q, c0, hi);
+      int shi = m.n_sink - 1 < q ? m.n_sink - 1 : q;
+      int sink = overlap(0, shi, c0, hi);
+      int both = overlap(wlo, shi, c0, hi);
+      return win + sink - both;
+    }
+    case FA_MASK_PREFIX_LM: {
+      int top = q > m.prefix - 1 ? q : m.prefix - 1;
+      return overlap(0, top, c0, hi);
+    }
+    case FA_MASK_CHUNKED:
+      return q < 0 ? 0 : overlap((q / m.chunk) * m.chunk, q, c0, hi);
+    default:
+      return 0;
+  }
+}
+
+__device__ uint8_t classify_tile_intervals(const MaskParams& m, int r0, int r1, int c0, int c1, int L, int S_b) {
+  const int lane = threadIdx.x & 31;
+  const int width = c1 - c0 + 1;
+  bool all_full = true, any_vis = false;
+  for (int r = r0 + lane; r <= r1; r += 32) {
+    int n = visible_count(m, query_pos(r, L, S_b), c0, c1, S_b);
+    all_full &= (n == width);
+    any_vis |= (n > 0);
+  }
+  all_full = __all_sync(0xffffffffu, all_full);
+  any_vis = __any_sync(0xffffffffu, any_vis);
+  return all_full ? kFull : (any_vis ? kPartial : kEmpty);
+}
+
+__device__ uint8_t classify_tile_cells(const MaskParams& m, int b, int r0, int r1, int c0, int c1, int L, int S,
+                                       int S_b) {
+  const int lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  if (m.kind == FA_MASK_DOCUMENT) {
+    // Disjoint document-id ranges: nothing in the tile can be visible.
+    const int* d = m.doc_id + static_cast<int64_t>(m.doc_batch > 1 ? b : 0) * S;
+    int rmin = INT32_MAX, rmax = INT32_MIN, cmin = INT32_MAX, cmax = INT32_MIN;
+    for (int r = r0 + lane; r <= r1; r += 32) {
+      int q = query_pos(r, L, S_b);
+      if (q >= 0 && q < S) {
+        int v = __ldg(d + q);
+        rmin = min(rmin, v);
+        rmax = max(rmax, v);
+      }
+    }
+    int chi = min(c1, S_b - 1);
+    for (int c = c0 + lane; c <= chi; c += 32) {
+      int v = __ldg(d + c);
+      cmin = min(cmin, v);
+      cmax = max(cmax, v);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      rmin = min(rmin, __shfl_xor_sync(full, rmin, o));
+      rmax = max(rmax, __shfl_xor_sync(full, rmax, o));
+      cmin = min(cmin, __shfl_xor_sync(full, cmin, o));
+      cmax = max(cmax, __shfl_xor_sync(full, cmax, o));
+    }
+    if (rmin > rmax || cmin > cmax || cmax < rmin || cmin > rmax) return kEmpty;
+  }
+  const int nr = r1 - r0 + 1, nc = c1 - c0 + 1;
+  const int64_t cells = static_cast<int64_t>(nr) * nc;
+  bool seen_vis = false, seen_hid = false;
+  for (int64_t base = 0; base < cells; base += 32) {
+    int64_t idx = base + lane;
+    bool vis = false, hid = false;
+    if (idx < cells) {
+      int r = r0 + static_cast<int>(idx / nc);
+      int c = c0 + static_cast<int>(idx % nc);
+      bool v = mask_visible(m, b, query_pos(r, L, S_b), c, S_b, S);
+      vis = v;
+      hid = !v;
+    }
+    seen_vis |= __any_sync(full, vis);
+    seen_hid |= __any_sync(full, hid);
+    if (seen_vis && seen_hid) break;
+  }
+  return seen_vis ? (seen_hid ? kPartial : kFull) : kEmpty;
+}
+
+__global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs a) {
+  extern __shared__ uint8_t cls[];
+  const int mt = blockIdx.x;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int S_b = seq_len_b(a.mask, b, a.S);
+  const int r0 = mt * a.BM;
+  const int r1 = min(a.L, r0 + a.BM) - 1;          // inclusive
+  const int q_hi = query_pos(r1, a.L, S_b);         // largest logical query position
+  const bool causal_family = a.mask.kind == FA_MASK_CAUSAL || a.mask.kind == FA_MASK_SLIDING_WINDOW ||
+                             a.mask.kind == FA_MASK_DOCUMENT || a.mask.kind == FA_MASK_CHUNKED;
+
+  for (int n = warp; n < a.Nb; n += nwarps) {
+    const int c0 = n * a.BN;
+    const int c1 = min(a.S, c0 + a.BN) - 1;        // inclusive
+    uint8_t k;
+    if (c0 >= S_b || (causal_family && c0 > q_hi)) {
+      k = kEmpty;
+    } else if (a.mask.kind == FA_MASK_DOCUMENT) {
+      k = classify_tile_cells(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b);
+    } else {
+      k = classify_tile_intervals(a.mask, r0, r1, c0, c1, a.L, S_b);
+    }
+    if (lane == 0) cls[n] = k;
+  }
+  __syncthreads();
+
+  // Ordered lists: warp 0 scans the classes 32 tiles at a time.
+  __shared__ int s_counts[2];
+  if (warp == 0) {
+    int nfull = 0, npart = 0;
+    for (int base = 0; base < a.Nb; base += 32) {
+      const int n = base + lane;
+      const uint8_t k = n < a.Nb ? cls[n] : kEmpty;
+      const unsigned fb = __ballot_sync(0xffffffffu, k == kFull);
+      const unsigned pb = __ballot_sync(0xffffffffu, k == kPartial);
+      const unsigned below = (1u << lane) - 1u;
+      for (int h = 0; h < a.H; ++h) {
+        const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+        if (k == kFull) a.full_kv_indices[row * a.Nb + nfull + __popc(fb & below)] = n;
+        if (k == kPartial) a.kv_indices[row * a.Nb + npart + __popc(pb & below)] = n;
+      }
+      nfull += __popc(fb);
+      npart += __popc(pb);
+    }
+    if (lane == 0) {
+      s_counts[0] = nfull;
+      s_counts[1] = npart;
+      for (int h = 0; h < a.H; ++h) {
+        const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+        a.full_kv_num_blocks[row] = nfull;
+        a.kv_num_blocks[row] = npart;
+      }
+    }
+  }
+  __syncthreads();
+  const int nfull = s_counts[0], npart = s_counts[1];
+  for (int h = 0; h < a.H; ++h) {
+    const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+    for (int i = threadIdx.x; i < a.Nb; i += blockDim.x) {
+      if (i >= nfull) a.full_kv_indices[row * a.Nb + i] = 0;
+      if (i >= npart) a.kv_indices[row * a.Nb + i] = 0;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream) {
+  dim3 grid(a.Mb, a.B);
+  size_t smem = (static_cast<size_t>(a.Nb) + 15) & ~static_cast<size_t>(15);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  classify_kernel<<<grid, kClassifyThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,69 @@
+// Host-side launch interfaces between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mods.cuh"
+
+namespace fa {
+
+struct ClassifyArgs {
+  int* status;  // device status word
+  MaskParams mask;
+  int B, H, L, S, BM, BN, Mb, Nb;
+  int* kv_num_blocks;
+  int* kv_indices;
+  int* full_kv_num_blocks;
+  int* full_kv_indices;
+};
+cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream);
+
+// Read-only view of a BlockMask; B and H may be 1 (broadcast).
+struct BlockMaskView {
+  int B, H, Mb, Nb, BM, BN;
+  const int* kv_num_blocks;
+  const int* kv_indices;
+  const int* full_kv_num_blocks;
+  const int* full_kv_indices;
+};
+
+struct FwdArgs {
+  int* status;  // device status word
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;                 // [B, Hq, L] or null
+  int64_t q_stride[4], k_stride[4], v_stride[4], o_stride[4];
+  int B, Hq, Hkv, L, S, E, Ev, G;
+  int dtype;                  // FA_DTYPE_*
+  float scale;
+  MaskParams mask;
+  ScoreParams score;
+  BlockMaskView bm;
+};
+
+// General kernel: any dtype, tiles up to 128 x 128, head dims up to 128.
+cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream);
+
+// Tensor-core prefill kernel (bf16, BM = BN = 128, E = Ev in {64, 128}).
+struct Sm100Maps {
+  CUtensorMap q, k, v;
+};
+cudaError_t launch_fwd_sm100(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t stream);
+
+// Split-KV decode for short queries (bf16, E = Ev in {64, 128}) and the
+// log-sum-exp combination of its partial results.
+struct DecodePlan {
+  int rows_per_cta;   // query rows handled by one CTA (heads of a group x L), <= 16
+  int heads_per_cta;  // query heads per CTA
+  int splits;         // KV splits per (b, head group)
+  int tiles_per_split;
+  size_t workspace_bytes;
+};
+int plan_decode(const FwdArgs& a, int split_kv, DecodePlan* plan);
+cudaError_t launch_decode(const FwdArgs& a, const DecodePlan& plan, void* workspace, cudaStream_t stream);
+
+}  // namespace fa
