@@ -267,8 +267,8 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   if (split_kv < 0) return fail(FA_ERR_PARAM, "split_kv must be >= 0");
   if (split_kv > 1 && !(tc_shape && L <= 16 && bm->Mb == 1))
     return fail(FA_ERR_UNSUPPORTED, "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16 and one query tile");
-  *path = Path::kSimt;
-  (void)tma_ok;
+  const bool out_ok = out == nullptr || aligned16(out);
+  *path = (tc_shape && tma_ok && out_ok && bm->BM == 128 && bm->BN == 128) ? Path::kSm100 : Path::kSimt;
   return FA_OK;
 }
 
@@ -348,7 +348,16 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
   if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
   a.lse = lse;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_fwd_simt(a, st);
+  cudaError_t e;
+  if (path == Path::kSm100) {
+    Sm100Maps maps;
+    if ((rc = encode_bf16_map(&maps.q, q, 128)) || (rc = encode_bf16_map(&maps.k, k, 128)) ||
+        (rc = encode_bf16_map(&maps.v, v, 128)))
+      return rc;
+    e = launch_fwd_sm100(a, maps, st);
+  } else {
+    e = launch_fwd_simt(a, st);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
   return FA_OK;
 }

@@ -342,34 +342,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       alive = mbar_wait(&bars.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, a.status);
       tc_fence_after();
     }
-    if (alive && row_ok) {
+    // TMEM loads are warp-collective: every lane takes part, rows past L
+    // included; only the stores depend on the row.
+    if (__all_sync(0xffffffffu, alive)) {
       const bool live = l_sum > 0.0f && ntiles > 0;
       const float inv = live ? 1.0f / l_sum : 0.0f;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] +
-                            static_cast<int64_t>(grow) * a.o_stride[2];
-      if (a.lse) a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.L + grow] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
+                            static_cast<int64_t>(row_ok ? grow : 0) * a.o_stride[2];
+      if (row_ok && a.lse)
+        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.L + grow] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
         uint32_t rr[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rr[i] = 0u;
         if (ntiles > 0) {
           tmem_ld16(tbase + lane_base + kColO + c * 16, rr);
           tmem_wait_ld();
         }
-        uint32_t pk[8];
+        if (row_ok) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-      }
-    } else if (alive && ntiles > 0) {
-      // rows past L still take part in the warp-wide TMEM loads
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t rr[16];
-        tmem_ld16(tbase + lane_base + kColO + c * 16, rr);
-        tmem_wait_ld();
+          for (int i = 0; i < 8; ++i)
+            pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
     }
   }
