@@ -34,35 +34,12 @@ __device__ __forceinline__ int overlap(int lo, int hi, int c0, int c1) {
   return b >= a ? b - a + 1 : 0;
 }
 
-// Number of visible keys in [c0, c1] (inclusive, c1 < S) for logical query q.
+// Number of visible keys in [c0, c1] (inclusive, c1 < S) for logical query q:
+// |A| + |B| - |A and B| over the two visible spans.
 __device__ __forceinline__ int visible_count(const MaskParams& m, int q, int c0, int c1, int S_b) {
-  const int last = S_b - 1;  // keys beyond the valid length are hidden
-  int hi = c1 < last ? c1 : last;
-  if (hi < c0) return 0;
-  switch (m.kind) {
-    case FA_MASK_NONE:
-      return hi - c0 + 1;
-    case FA_MASK_CAUSAL:
-      return q < 0 ? 0 : overlap(0, q, c0, hi);
-    case FA_MASK_SLIDING_WINDOW: {
-      if (q < 0) return 0;
-      int wlo = q - m.window + 1;
-      wlo = wlo < 0 ? 0 : wlo;
-      int win = overlap(wlo, q, c0, hi);
-      int shi = m.n_sink - 1 < q ? m.n_sink - 1 : q;
-      int sink = overlap(0, shi, c0, hi);
-      int both = overlap(wlo, shi, c0, hi);
-      return win + sink - both;
-    }
-    case FA_MASK_PREFIX_LM: {
-      int top = q > m.prefix - 1 ? q : m.prefix - 1;
-      return overlap(0, top, c0, hi);
-    }
-    case FA_MASK_CHUNKED:
-      return q < 0 ? 0 : overlap((q / m.chunk) * m.chunk, q, c0, hi);
-    default:
-      return 0;
-  }
+  const KeySpans sp = visible_spans(m, q, S_b);
+  return overlap(sp.a0, sp.a1, c0, c1) + overlap(sp.b0, sp.b1, c0, c1) -
+         overlap(max(sp.a0, sp.b0), min(sp.a1, sp.b1), c0, c1);
 }
 
 __device__ uint8_t classify_tile_intervals(const MaskParams& m, int r0, int r1, int c0, int c1, int L, int S_b) {

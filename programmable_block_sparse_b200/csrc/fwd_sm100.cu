@@ -75,6 +75,32 @@ __device__ __forceinline__ int tile_at(const FwdArgs& a, int64_t brow, int nfull
                   : __ldg(a.bm.kv_indices + brow * a.bm.Nb + (j - nfull));
 }
 
+// Bits [lo, hi] of a 32-bit word (positions relative to the word's first column).
+__device__ __forceinline__ uint32_t span_bits(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 31);
+  if (hi < lo) return 0u;
+  const uint32_t upto = hi == 31 ? 0xFFFFFFFFu : ((2u << hi) - 1u);
+  return upto & ~((1u << lo) - 1u);
+}
+
+// One TMEM row of 128 fp32 columns into registers: eight loads in flight, one
+// wait.  The empty asm statements after the wait carry the registers as
+// read-write operands so no use of them is scheduled before the wait.
+__device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&t)[128]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(t);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(u + c * 16));
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t* x = u + c * 16;
+    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),
+                 "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]),
+                 "+r"(x[14]), "+r"(x[15]));
+  }
+}
+
 // Score rule in log2 units for one element; `d` = kv - q as a float.
 template <int SCORE>
 __device__ __forceinline__ float score_log2(float s, float c_in, float c_out, float slope2, float dist) {
@@ -97,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
+  __shared__ float s_pos[2][kTile];  // slope * position of the tile's keys (score with positions)
+  __shared__ int s_doc[2][kTile];    // document ids of the tile's keys (partial document tiles)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::kTileBytes;
@@ -238,7 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       c_in = 0.0f;
       c_out = a.scale * kLog2e;
     }
-    const int pq = (SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr) ? pos_at(a.score, b, qpos, a.S) : qpos;
+    const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
+    const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
+    const bool is_doc = a.mask.kind == FA_MASK_DOCUMENT;
+    const int* doc_row = is_doc ? a.mask.doc_id + static_cast<int64_t>(a.mask.doc_batch > 1 ? b : 0) * a.S : nullptr;
+    const int my_doc = (is_doc && row_ok && qpos >= 0) ? __ldg(doc_row + qpos) : -1;
+    const KeySpans spans = visible_spans(a.mask, qpos, S_b);
     float m_ref = -INFINITY, l_sum = 0.0f;
     bool alive = true;
 
@@ -247,43 +280,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = tile_at(a, brow, nfull, j, &full);
       const int kv0 = n * kTile;
       const bool edge = kv0 + kTile > S_b;
+      const bool stage_doc = is_doc && (!full || edge);  // the same for every row of the tile
+      if (has_pos || stage_doc) {
+        // stage this tile's key-side values in smem (double-buffered by j & 1)
+        const int kv = kv0 + r;
+        if (has_pos) s_pos[j & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
+        if (stage_doc) s_doc[j & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
+        named_bar_sync(1, 128);
+      }
       if (!mbar_wait(&bars.s_full[j & 1], (j >> 1) & 1, abort, a.status)) {
         alive = false;
         break;
       }
       tc_fence_after();
       float t[kTile];
-      {
-        uint32_t rr[16];
-#pragma unroll
-        for (int c = 0; c < kTile / 16; ++c) {
-          tmem_ld16(tbase + lane_base + kColS0 + 128 * (j & 1) + c * 16, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) t[c * 16 + i] = __uint_as_float(rr[i]);
-        }
-      }
+      tmem_load_row128(tbase + lane_base + kColS0 + 128 * (j & 1), t);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
 
-      // score rule, then the element mask on partial and edge tiles
-      const bool need_mask = !full || edge || !row_ok;
+      // score rule on every cell (log2 units)
+      if constexpr (SCORE == FA_SCORE_NONE) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) t[c] *= c_out;
+      } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) t[c] = c_out * tanh_fast(t[c] * c_in);
+      } else if constexpr (SCORE == FA_SCORE_ALIBI) {
+        const float bias0 = slope2 * static_cast<float>(kv0 - qpos);
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) t[c] = fmaf(t[c], c_out, fmaf(slope2, static_cast<float>(c), bias0));
+      } else {
+        if (has_pos) {
+          const float* pk = s_pos[j & 1];
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), pk[c] - pq_scaled);
+        } else {
+          const float bias0 = slope2 * static_cast<float>(kv0 - qpos);
+#pragma unroll
+          for (int c = 0; c < kTile; ++c)
+            t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), fmaf(slope2, static_cast<float>(c), bias0));
+        }
+      }
+
+      // element mask on partial tiles, ragged edges and rows past L
+      if (!full || edge || !row_ok) {
+        uint32_t bits[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int base = kv0 + 32 * w;
+          bits[w] = row_ok ? (span_bits(spans.a0 - base, spans.a1 - base) | span_bits(spans.b0 - base, spans.b1 - base))
+                           : 0u;
+        }
+        if (stage_doc) {
+          const int* dk = s_doc[j & 1];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t same = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) same |= (dk[32 * w + i] == my_doc ? 1u : 0u) << i;
+            bits[w] &= same;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!((bits[c >> 5] >> (c & 31)) & 1u)) t[c] = -INFINITY;
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const int kv = kv0 + c;
-        float dist = 0.0f;
-        if constexpr (SCORE == FA_SCORE_ALIBI) {
-          dist = static_cast<float>(kv - qpos);
-        } else if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS) {
-          dist = static_cast<float>((a.score.pos != nullptr ? pos_at(a.score, b, kv, a.S) : kv) - pq);
-        }
-        float v = score_log2<SCORE>(t[c], c_in, c_out, slope2, dist);
-        if (need_mask && !(row_ok && mask_visible(a.mask, b, qpos, kv, S_b, a.S))) v = -INFINITY;
-        t[c] = v;
-        mx = fmaxf(mx, v);
-      }
+      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, t[c]);
 
       // running max: move it (and rescale O) only when it grows past 2^8
       const bool grow_max = mx > m_ref + kRescaleThreshold;

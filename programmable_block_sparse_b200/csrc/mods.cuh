@@ -64,6 +64,49 @@ __device__ __forceinline__ bool mask_visible(const MaskParams& m, int b, int q, 
   }
 }
 
+// The keys visible to the query at logical position q form at most two
+// inclusive spans [a0, a1] and [b0, b1] (empty when the low end exceeds the
+// high end), already clipped to [0, S_b - 1].  For DOCUMENT this is only the
+// causal bound [0, q]: the same-document test is applied per key on top.
+struct KeySpans {
+  int a0, a1, b0, b1;
+};
+
+__device__ __forceinline__ KeySpans visible_spans(const MaskParams& m, int q, int S_b) {
+  const int last = S_b - 1;
+  KeySpans r{1, 0, 1, 0};
+  switch (m.kind) {
+    case FA_MASK_NONE:
+      r.a0 = 0;
+      r.a1 = last;
+      break;
+    case FA_MASK_CAUSAL:
+    case FA_MASK_DOCUMENT:
+      r.a0 = 0;
+      r.a1 = min(q, last);
+      break;
+    case FA_MASK_SLIDING_WINDOW:
+      r.a0 = max(q - m.window + 1, 0);
+      r.a1 = min(q, last);
+      r.b0 = 0;
+      r.b1 = min(min(m.n_sink - 1, q), last);
+      break;
+    case FA_MASK_PREFIX_LM:
+      r.a0 = 0;
+      r.a1 = min(max(q, m.prefix - 1), last);
+      break;
+    case FA_MASK_CHUNKED:
+      if (q >= 0) {
+        r.a0 = (q / m.chunk) * m.chunk;
+        r.a1 = min(q, last);
+      }
+      break;
+    default:
+      break;
+  }
+  return r;
+}
+
 // slope_h = 2^(-8 (h + 1) / H).
 __device__ __forceinline__ float distance_slope(int h, int H) {
   return exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(H));

@@ -1,0 +1,38 @@
+"""bench.py's exact work counts agree with the oracle's visibility on small shapes."""
+import numpy as np
+
+import bench
+import oracle.flex_oracle as o
+import workloads as wl
+
+
+def _oracle_pairs(c, kv_len=None, doc_ids=None):
+    mask = dict(c["mask"])
+    if doc_ids is not None:
+        mask["doc_id"] = doc_ids
+    tot = 0
+    for b in range(c["B"]):
+        S_b = c["S"] if kv_len is None else int(kv_len[b])
+        vis = o.visible(mask, b, 0, o.query_positions(c["L"], S_b), np.arange(c["S"]), S_b)
+        tot += int(vis.sum())
+    return tot
+
+
+def test_visible_pair_counts():
+    c = wl.config("causal_softcap_alibi", B=2, L=300, S=300)
+    assert bench.visible_pairs_per_head(c) == _oracle_pairs(c)
+    c = wl.config("gqa_sliding_window", B=1, L=700, S=700, mask=dict(kind="sliding_window", window=100, n_sink=4))
+    assert bench.visible_pairs_per_head(c) == _oracle_pairs(c)
+    lens = wl.doc_lengths(500, 20, 90, 3)
+    c = wl.config("packed_docs", L=500, S=500)
+    assert bench.visible_pairs_per_head(c, doc_lengths=lens) == _oracle_pairs(c, doc_ids=wl.doc_ids_from_lengths(lens))
+    c = wl.config("decode_kv_cache", B=5, S=900)
+    kv = np.array([900, 13, 400, 4, 77])
+    assert bench.visible_pairs_per_head(c, kv_len=kv) == _oracle_pairs(c, kv_len=kv)
+
+
+def test_full_size_counts_match_closed_forms():
+    c = wl.config("causal_softcap_alibi")
+    assert bench.visible_pairs_per_head(c) == 4 * 2048 * 2049 // 2
+    c = wl.config("gqa_sliding_window")
+    assert bench.visible_pairs_per_head(c) == 2 * 16314874

@@ -23,15 +23,21 @@ def test_decode_cache_lengths_seed0():
     assert lens.min() >= 4096 and lens.max() <= 32768
 
 
-def test_qkv_draw_order_and_cast():
-    q, k, v = w.randn_qkv(1, 2, 1, 3, 5, 4, 6, seed=0, dtype=torch.float32)
-    g = torch.Generator("cpu").manual_seed(0)
-    q2 = torch.randn((1, 2, 3, 4), generator=g)
-    k2 = torch.randn((1, 1, 5, 4), generator=g)
-    v2 = torch.randn((1, 1, 5, 6), generator=g)
-    assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(v, v2)
-    qb, _, _ = w.randn_qkv(1, 2, 1, 3, 5, 4, 6, seed=0, dtype=torch.bfloat16)
-    assert torch.equal(qb, q2.to(torch.bfloat16))
+def test_qkv_slices_regenerate_alone():
+    q, k, v = w.randn_qkv(2, 3, 1, 5, 7, 4, 6, seed=0, dtype=torch.float32)
+    for which, t in ((0, q), (1, k), (2, v)):
+        B, H, N, D = t.shape
+        for b in range(B):
+            for h in range(H):
+                g = torch.Generator("cpu").manual_seed(w.slice_seed(0, which, b, h))
+                assert torch.equal(t[b, h], torch.randn((N, D), generator=g))
+    qb, _, _ = w.randn_qkv(2, 3, 1, 5, 7, 4, 6, seed=0, dtype=torch.bfloat16)
+    assert torch.equal(qb, q.to(torch.bfloat16))
+    assert not torch.equal(q[0, 0], q[0, 1]) and not torch.equal(q[0, 0], q[1, 0])
+    q1, _, _ = w.randn_qkv(2, 3, 1, 5, 7, 4, 6, seed=1, dtype=torch.float32)
+    assert not torch.equal(q, q1)
+    seeds = {w.slice_seed(s, t, b, h) for s in range(3) for t in range(3) for b in range(32) for h in range(64)}
+    assert len(seeds) == 3 * 3 * 32 * 64 and max(seeds) < 2 ** 32
 
 
 def test_cache_tail_sentinels():

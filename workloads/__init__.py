@@ -8,9 +8,10 @@ the oracle and the C-ABI binding each interpret them with their own code.
 
 Recipes (stated so that every number below can be regenerated):
 
-* Q/K/V: ``torch.Generator('cpu').manual_seed(seed)``, then ``torch.randn`` in
-  fp32 in the order q, k, v, each of its full (B, H, N, D) shape, then a cast to
-  the workload dtype.  iid N(0, 1).
+* Q/K/V: every (b, h) slice of q (which = 0), k (1) and v (2) is drawn with
+  ``torch.randn`` in fp32 from its own ``torch.Generator('cpu')`` seeded with
+  ``slice_seed(seed, which, b, h)`` (a 32-bit mix of the four indices), then
+  cast to the workload dtype.  iid N(0, 1); any slice can be regenerated alone.
 * Packed documents: lengths drawn one at a time from
   ``numpy.random.default_rng(seed).integers(lo, hi + 1)`` until their sum
   reaches the total, the last one trimmed so the sum is exact.
@@ -22,11 +23,15 @@ Recipes (stated so that every number below can be regenerated):
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
 
 __all__ = [
+    "slice_seed",
+    "randn_slice",
     "randn_qkv",
     "doc_lengths",
     "doc_ids_from_lengths",
@@ -38,13 +43,55 @@ __all__ = [
 ]
 
 
+def slice_seed(seed, which, b, h):
+    """32-bit seed of the (b, h) slice of tensor ``which`` (0 = q, 1 = k, 2 = v).
+
+    torch's CPU generator keeps 32 bits of a seed, so the four indices are
+    folded into 32 bits: a weighted sum, then an integer bit mixer.
+    """
+    m = 0xFFFFFFFF
+    x = (int(seed) * 0x9E3779B1 + int(which) * 0x85EBCA77 + int(b) * 0xC2B2AE3D + int(h) * 0x27D4EB2F) & m
+    x ^= x >> 16
+    x = (x * 0x7FEB352D) & m
+    x ^= x >> 15
+    x = (x * 0x846CA68B) & m
+    x ^= x >> 16
+    return x
+
+
+def randn_slice(seed, which, b, h, N, D, dtype=torch.bfloat16):
+    """One (N, D) slice: torch.randn in fp32 from its own generator, then cast."""
+    g = torch.Generator("cpu").manual_seed(slice_seed(seed, which, b, h))
+    return torch.randn((N, D), generator=g, dtype=torch.float32).to(dtype)
+
+
+def _fill(t, seed, which):
+    B, H, N, D = t.shape
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+
+    def one(bh):
+        b, h = bh
+        t[b, h].copy_(randn_slice(seed, which, b, h, N, D, t.dtype))
+
+    if len(jobs) * N * D >= (1 << 22):
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+            list(ex.map(one, jobs))
+    else:
+        for bh in jobs:
+            one(bh)
+    return t
+
+
 def randn_qkv(B, Hq, Hkv, L, S, E, Ev, seed=0, dtype=torch.bfloat16):
-    """iid N(0,1) q (B,Hq,L,E), k (B,Hkv,S,E), v (B,Hkv,S,Ev) on the CPU."""
-    g = torch.Generator("cpu").manual_seed(int(seed))
-    q = torch.randn((B, Hq, L, E), generator=g, dtype=torch.float32)
-    k = torch.randn((B, Hkv, S, E), generator=g, dtype=torch.float32)
-    v = torch.randn((B, Hkv, S, Ev), generator=g, dtype=torch.float32)
-    return q.to(dtype), k.to(dtype), v.to(dtype)
+    """iid N(0,1) q (B,Hq,L,E), k (B,Hkv,S,E), v (B,Hkv,S,Ev) on the CPU.
+
+    Every (b, h) slice of every tensor has its own generator (see
+    :func:`randn_slice`), so any slice can be regenerated on its own.
+    """
+    q = _fill(torch.empty((B, Hq, L, E), dtype=dtype), seed, 0)
+    k = _fill(torch.empty((B, Hkv, S, E), dtype=dtype), seed, 1)
+    v = _fill(torch.empty((B, Hkv, S, Ev), dtype=dtype), seed, 2)
+    return q, k, v
 
 
 def doc_lengths(total, lo, hi, seed=0):
