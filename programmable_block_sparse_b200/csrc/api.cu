@@ -185,6 +185,18 @@ int encode_bf16_map(CUtensorMap* map, const fa_tensor* t, int box_rows) {
 // ----------------------------------------------------------------------------
 enum class Path { kSimt, kSm100, kDecode };
 
+int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 int check_tensor(const fa_tensor* t, const char* name) {
   if (t == nullptr || t->data == nullptr) return fail(FA_ERR_NULL, "%s is NULL", name);
   if (t->dtype != FA_DTYPE_BF16 && t->dtype != FA_DTYPE_F32) return fail(FA_ERR_DTYPE, "%s: unknown dtype %d", name, t->dtype);
@@ -265,10 +277,19 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   const bool tc_shape = q->dtype == FA_DTYPE_BF16 && E == Ev && (E == 64 || E == 128);
   const bool tma_ok = aligned16(q) && aligned16(k) && aligned16(v);
   if (split_kv < 0) return fail(FA_ERR_PARAM, "split_kv must be >= 0");
-  if (split_kv > 1 && !(tc_shape && L <= 16 && bm->Mb == 1))
-    return fail(FA_ERR_UNSUPPORTED, "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16 and one query tile");
+  if (split_kv > 1 && !(tc_shape && L <= kDecodeMaxRows && bm->Mb == 1 && bm->BN % 64 == 0))
+    return fail(FA_ERR_UNSUPPORTED,
+                "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16, one query tile and BN in {64, 128}");
+  if (split_kv > 1 && !tma_ok) return fail(FA_ERR_ALIGN, "split_kv > 1 needs 16-byte aligned q, k, v and strides");
   const bool out_ok = out == nullptr || aligned16(out);
-  *path = (tc_shape && tma_ok && out_ok && bm->BM == 128 && bm->BN == 128) ? Path::kSm100 : Path::kSimt;
+  const bool decode_ok = tc_shape && tma_ok && L <= kDecodeMaxRows && bm->Mb == 1 && bm->BN % 64 == 0;
+  if (split_kv != 1 && decode_ok) {
+    *path = Path::kDecode;
+  } else if (tc_shape && tma_ok && out_ok && bm->BM == 128 && bm->BN == 128) {
+    *path = Path::kSm100;
+  } else {
+    *path = Path::kSimt;
+  }
   return FA_OK;
 }
 
@@ -329,6 +350,11 @@ int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, cons
   int rc = prepare(q, k, v, nullptr, 0.0f, 1, &none_score, &none_mask, block_mask, split_kv, &a, &path);
   if (rc) return rc;
   *bytes = 0;
+  if (path == Path::kDecode) {
+    DecodePlan plan;
+    plan_decode(a, split_kv, sm_count(), &plan);
+    *bytes = plan.workspace_bytes;
+  }
   return FA_OK;
 }
 
@@ -341,8 +367,6 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
   Path path;
   int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
   if (rc) return rc;
-  (void)workspace;
-  (void)workspace_bytes;
   int serr = 0;
   a.status = status_word(&serr);
   if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
@@ -355,6 +379,17 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
         (rc = encode_bf16_map(&maps.v, v, 128)))
       return rc;
     e = launch_fwd_sm100(a, maps, st);
+  } else if (path == Path::kDecode) {
+    DecodePlan plan;
+    plan_decode(a, split_kv, sm_count(), &plan);
+    if (plan.workspace_bytes > 0 && (workspace == nullptr || workspace_bytes < plan.workspace_bytes))
+      return fail(FA_ERR_WORKSPACE, "split-KV decode needs %zu bytes of workspace (got %zu)", plan.workspace_bytes,
+                  workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (plan.workspace_bytes > 0 && reinterpret_cast<uintptr_t>(workspace) % 16)
+      return fail(FA_ERR_ALIGN, "workspace must be 16-byte aligned");
+    Sm100Maps maps;
+    if ((rc = encode_bf16_map(&maps.k, k, 64)) || (rc = encode_bf16_map(&maps.v, v, 64))) return rc;
+    e = launch_decode(a, plan, maps, workspace, st);
   } else {
     e = launch_fwd_simt(a, st);
   }

@@ -1,0 +1,431 @@
+// Split-KV decode for short queries against long KV caches, and the
+// log-sum-exp combination of its partial results.
+//
+// The computation is the forward definition of "flexattention-score-mod-
+// block-mask" (charlestar.github.io), "What one connection goes through", with
+// logical query positions q = i + (S_b - L) ("At decode, q_idx = 0 is not
+// position 0"; bottom-right alignment, "Causal Mask" (quant67.com) section 4).
+// Only the tiles the BlockMask lists are read.  A decode step streams the whole
+// valid cache once, so the kernel is built around HBM bandwidth:
+//
+//   grid      (split, KV head x head chunk, batch); one CTA takes the query rows
+//             of up to 16 (query head, position) pairs that share one KV head
+//             (GQA: the group's heads reuse every K/V byte it loads) and a
+//             contiguous run of the row's listed tiles.
+//   warp 0    TMA producer: 64-key K and V sub-tiles (128-byte swizzle) into a
+//             3-stage ring.
+//   warps 1-4 consumers: each takes 16 of every 64 keys; S = Q K^T and O += P V
+//             with mma.sync m16n8k16 (bf16 in, fp32 accumulate; at most 16 rows
+//             make the 128-row tcgen05 tile a poor fit and the step is bound by
+//             HBM, not the tensor pipe); score rule, element mask and online
+//             softmax in registers.  The four warps' (max, sum, O) are merged
+//             through shared memory at the end.
+//   output    one split: out and lse directly.  Several splits: normalised O
+//             and lse per split into the workspace, then combine_kernel merges
+//             them: lse = ln sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "mods.cuh"
+
+namespace fa {
+
+namespace {
+
+constexpr int kDecThreads = 160;
+constexpr int kSub = 64;        // keys per pipeline stage
+constexpr int kStagesDec = 3;
+constexpr int kRows = 16;       // query rows per CTA (one m16 fragment)
+constexpr float kLog2eD = 1.4426950408889634f;
+constexpr float kLn2D = 0.6931471805599453f;
+
+template <int D>
+struct DecCfg {
+  static constexpr int kBoxBytes = kSub * 128;            // 64 keys x 64 columns of bf16
+  static constexpr int kTileBytes = kSub * D * 2;         // one K or V sub-tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kSmemBytes = kStagesDec * kStageBytes + 1024;
+};
+
+struct DecBars {
+  uint64_t full[kStagesDec], empty[kStagesDec];
+  int abort;
+};
+
+__device__ __forceinline__ float ex2f_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of (row, 8-element chunk) inside a 128-byte-swizzled box of
+// 64 rows x 64 bf16, as written by TMA.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ int list_tile(const FwdArgs& a, int64_t brow, int nfull, int j) {
+  return j < nfull ? __ldg(a.bm.full_kv_indices + brow * a.bm.Nb + j)
+                   : __ldg(a.bm.kv_indices + brow * a.bm.Nb + (j - nfull));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    decode_kernel(const FwdArgs a, const DecodePlan p, const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v, float* ws_o, float* ws_lse) {
+  using C = DecCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ DecBars bars;
+  __shared__ float s_m[4][kRows], s_l[4][kRows];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int head_chunks = (a.G + p.heads_per_cta - 1) / p.heads_per_cta;
+  const int hk = blockIdx.y / head_chunks, hc = blockIdx.y % head_chunks;
+  const int b = blockIdx.z;
+  const int S_b = seq_len_b(a.mask, b, a.S);
+  const int bmb = a.bm.B > 1 ? b : 0;
+  const int64_t brow = static_cast<int64_t>(bmb) * a.bm.H * a.bm.Mb;  // head row 0, tile row 0
+  const int nfull = __ldg(a.bm.full_kv_num_blocks + brow);
+  const int ntiles = nfull + __ldg(a.bm.kv_num_blocks + brow);
+  const int t0 = split * p.tiles_per_split;
+  const int t1 = min(ntiles, t0 + p.tiles_per_split);
+  const int subs_per_tile = a.bm.BN / kSub;
+  const int nsub = t1 > t0 ? (t1 - t0) * subs_per_tile : 0;
+  volatile int* abort = &bars.abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesDec; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 4);
+    }
+    bars.abort = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  // rows of this CTA: row rho -> (query head, position)
+  auto row_head = [&](int rho) { return hk * a.G + hc * p.heads_per_cta + rho / a.L; };
+  auto row_valid = [&](int rho) {
+    const int g = hc * p.heads_per_cta + rho / a.L;
+    return rho < p.rows_per_cta && rho / a.L < p.heads_per_cta && g < a.G;
+  };
+
+  if (warp == 0) {
+    if (lane == 0 && nsub > 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      int issued = 0;
+      for (int u = 0; u < nsub && !*abort; ++u) {
+        const int s = u % kStagesDec;
+        if (u >= kStagesDec && !mbar_wait(&bars.empty[s], ((u / kStagesDec) - 1) & 1, abort, a.status)) break;
+        const int n = list_tile(a, brow, nfull, t0 + u / subs_per_tile);
+        const int kv0 = n * a.bm.BN + (u % subs_per_tile) * kSub;
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_expect_tx(&bars.full[s], C::kStageBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(st + c * C::kBoxBytes, &map_k, &bars.full[s], c * 64, kv0, hk, b);
+          tma_load_4d(st + C::kTileBytes + c * C::kBoxBytes, &map_v, &bars.full[s], c * 64, kv0, hk, b);
+        }
+        issued = u + 1;
+      }
+      if (*abort) {
+        volatile int never = 0;
+        for (int u = (issued > kStagesDec ? issued - kStagesDec : 0); u < issued; ++u)
+          mbar_wait(&bars.full[u % kStagesDec], (u / kStagesDec) & 1, &never, nullptr);
+      }
+    }
+  } else {
+    const int cw = warp - 1;            // consumer warp: keys [16 cw, 16 cw + 16) of each stage
+    const int r_lo = lane >> 2;          // fragment rows r_lo and r_lo + 8
+    const int quad = lane & 3;
+    // Q as A fragments, straight from global memory
+    uint32_t qa[D / 16][4];
+    {
+      const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int rho = r_lo + 8 * half;
+        const bool ok = row_valid(rho);
+        const __nv_bfloat16* qrow =
+            ok ? qb + b * a.q_stride[0] + row_head(rho) * a.q_stride[1] + (rho % a.L) * a.q_stride[2] : qb;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int e = 16 * ks + 2 * quad;
+          qa[ks][half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + e) : 0u;
+          qa[ks][half + 2] = ok ? *reinterpret_cast<const uint32_t*>(qrow + e + 8) : 0u;
+        }
+      }
+    }
+    // per-row constants for the two fragment rows
+    int qpos[2], hq[2];
+    bool rok[2];
+    float slope2[2];
+    const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int rho = r_lo + 8 * half;
+      rok[half] = row_valid(rho);
+      hq[half] = rok[half] ? row_head(rho) : 0;
+      qpos[half] = query_pos(rho % a.L, a.L, S_b);
+      slope2[half] = distance_slope(hq[half], Hs);
+    }
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+
+    for (int u = 0; u < nsub; ++u) {
+      const int s = u % kStagesDec;
+      if (!mbar_wait(&bars.full[s], (u / kStagesDec) & 1, abort, a.status)) break;
+      const int j = t0 + u / subs_per_tile;
+      const bool full = j < nfull;
+      const int n = list_tile(a, brow, nfull, j);
+      const int kv0 = n * a.bm.BN + (u % subs_per_tile) * kSub;
+      const uint32_t sk = smem_u32(smem + s * C::kStageBytes);
+      const uint32_t sv = sk + C::kTileBytes;
+      // S = Q K^T for keys kv0 + 16 cw + [0, 16)
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int key = 16 * cw + 8 * (mi >> 1) + rr;
+        const int e = 16 * ks + 8 * (mi & 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(sk + (e >> 6) * C::kBoxBytes + swz(key, (e & 63) >> 3), b0, b1, b2, b3);
+        mma_bf16_16816(sc[0], qa[ks], b0, b1);
+        mma_bf16_16816(sc[1], qa[ks], b2, b3);
+      }
+      // score rule, element mask, online softmax (log2 units)
+      const bool need_mask = !full || (kv0 + kSub > S_b);
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int half = e >> 1;
+          const int kv = kv0 + 16 * cw + 8 * nt + 2 * quad + (e & 1);
+          float g = score_apply<false>(a.score, sc[nt][e] * a.scale, b, qpos[half], kv, a.S, slope2[half]) * kLog2eD;
+          const bool vis = rok[half] && (!need_mask || mask_visible(a.mask, b, qpos[half], kv, S_b, a.S));
+          g = vis ? g : -INFINITY;
+          sc[nt][e] = g;
+          mx[half] = fmaxf(mx[half], g);
+        }
+      }
+      float alpha[2], mu[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 1));
+        mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 2));
+        const float m_new = fmaxf(m_run[half], mx[half]);
+        alpha[half] = (m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - m_new);
+        m_run[half] = m_new;
+        mu[half] = (m_new == -INFINITY) ? 0.0f : m_new;
+      }
+      float ps[2] = {0.0f, 0.0f};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          sc[nt][e] = ex2f_approx(sc[nt][e] - mu[e >> 1]);
+          ps[e >> 1] += sc[nt][e];
+        }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) l_run[half] = l_run[half] * alpha[half] + ps[half];
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        o[i][0] *= alpha[0];
+        o[i][1] *= alpha[0];
+        o[i][2] *= alpha[1];
+        o[i][3] *= alpha[1];
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
+      pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
+      pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
+      pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
+      // O += P V over the same 16 keys
+#pragma unroll
+      for (int et = 0; et < D / 16; ++et) {
+        const int key = 16 * cw + 8 * (mi & 1) + rr;
+        const int ev = 16 * et + 8 * (mi >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(sv + (ev >> 6) * C::kBoxBytes + swz(key, (ev & 63) >> 3), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * et], pa, b0, b1);
+        mma_bf16_16816(o[2 * et + 1], pa, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.empty[s]);
+    }
+    // row sums across the quad
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      l_run[half] += __shfl_xor_sync(0xffffffffu, l_run[half], 1);
+      l_run[half] += __shfl_xor_sync(0xffffffffu, l_run[half], 2);
+    }
+    if (quad == 0) {
+      s_m[cw][r_lo] = m_run[0];
+      s_m[cw][r_lo + 8] = m_run[1];
+      s_l[cw][r_lo] = l_run[0];
+      s_l[cw][r_lo + 8] = l_run[1];
+    }
+    named_bar_sync(1, 128);
+    // merge the four warps: scale each warp's O by 2^(m_w - m) and add in smem
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int rho = r_lo + 8 * half;
+      float m = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) m = fmaxf(m, s_m[w][rho]);
+      const float f = (m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - m);
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        o[i][2 * half] *= f;
+        o[i][2 * half + 1] *= f;
+      }
+    }
+    // the stage buffers are idle now (every stage was consumed): reuse them
+    float* s_o = reinterpret_cast<float*>(smem);  // [kRows][D]
+    for (int i = threadIdx.x - 32; i < kRows * D; i += 128) s_o[i] = 0.0f;
+    named_bar_sync(1, 128);
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      const int col = 8 * i + 2 * quad;
+      atomicAdd(&s_o[r_lo * D + col], o[i][0]);
+      atomicAdd(&s_o[r_lo * D + col + 1], o[i][1]);
+      atomicAdd(&s_o[(r_lo + 8) * D + col], o[i][2]);
+      atomicAdd(&s_o[(r_lo + 8) * D + col + 1], o[i][3]);
+    }
+    named_bar_sync(1, 128);
+    // write: warp cw handles rows 4 cw .. 4 cw + 3, lanes across columns
+    for (int rho = 4 * cw; rho < 4 * cw + 4; ++rho) {
+      if (!row_valid(rho)) continue;
+      const int hqr = row_head(rho), i = rho % a.L;
+      float m = -INFINITY, l = 0.0f;
+      for (int w = 0; w < 4; ++w) m = fmaxf(m, s_m[w][rho]);
+      for (int w = 0; w < 4; ++w) l += (s_m[w][rho] == -INFINITY) ? 0.0f : s_l[w][rho] * ex2f_approx(s_m[w][rho] - m);
+      const bool live = l > 0.0f;
+      const float inv = live ? 1.0f / l : 0.0f;
+      const float lse = live ? (m + log2f(l)) * kLn2D : -INFINITY;
+      const int64_t row_id = (static_cast<int64_t>(b) * a.Hq + hqr) * a.L + i;
+      if (p.splits == 1) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + hqr * a.o_stride[1] +
+                              i * a.o_stride[2];
+        for (int c = lane; c < D; c += 32) orow[c] = __float2bfloat16_rn(s_o[rho * D + c] * inv);
+        if (lane == 0 && a.lse) a.lse[row_id] = lse;
+      } else {
+        float* wrow = ws_o + (row_id * p.splits + split) * D;
+        for (int c = lane; c < D; c += 32) wrow[c] = s_o[rho * D + c] * inv;
+        if (lane == 0) ws_lse[row_id * p.splits + split] = lse;
+      }
+    }
+  }
+}
+
+// One warp per (b, h, i) row: merge the per-split (o_s, lse_s).
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(const FwdArgs a, const DecodePlan p, const float* ws_o,
+                                                      const float* ws_lse) {
+  const int64_t row_id = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
+  if (row_id >= rows) return;
+  const int i = static_cast<int>(row_id % a.L);
+  const int h = static_cast<int>((row_id / a.L) % a.Hq);
+  const int b = static_cast<int>(row_id / (static_cast<int64_t>(a.L) * a.Hq));
+  const float* lrow = ws_lse + row_id * p.splits;
+  float m = -INFINITY;
+  for (int s = lane; s < p.splits; s += 32) m = fmaxf(m, lrow[s]);
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float acc[D / 32];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) acc[c] = 0.0f;
+  float tot = 0.0f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < p.splits; ++s) {
+      const float ls = lrow[s];
+      if (ls == -INFINITY) continue;
+      const float w = expf(ls - m);
+      tot += w;
+      const float* orow = ws_o + (row_id * p.splits + s) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, orow[lane + 32 * c], acc[c]);
+    }
+  }
+  const bool live = tot > 0.0f;
+  const float inv = live ? 1.0f / tot : 0.0f;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] + i * a.o_stride[2];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) out[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
+  if (lane == 0 && a.lse) a.lse[row_id] = live ? m + logf(tot) : -INFINITY;
+}
+
+template <int D>
+cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Maps& maps, void* workspace,
+                            cudaStream_t stream) {
+  const int head_chunks = (a.G + p.heads_per_cta - 1) / p.heads_per_cta;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_lse = ws_o ? ws_o + static_cast<int64_t>(a.B) * a.Hq * a.L * p.splits * D : nullptr;
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecCfg<D>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.splits, a.Hkv * head_chunks, a.B);
+  decode_kernel<D><<<grid, kDecThreads, DecCfg<D>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
+  combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(a, p, ws_o, ws_lse);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int plan_decode(const FwdArgs& a, int split_kv, int num_sms, DecodePlan* p) {
+  p->heads_per_cta = a.G < kRows / a.L ? a.G : kRows / a.L;
+  p->rows_per_cta = p->heads_per_cta * a.L;
+  const int head_chunks = (a.G + p->heads_per_cta - 1) / p->heads_per_cta;
+  const int units = a.B * a.Hkv * head_chunks;
+  const int Nb = a.bm.Nb;
+  int splits;
+  if (split_kv > 1) {
+    splits = split_kv < Nb ? split_kv : Nb;
+  } else {
+    // about eight CTAs' worth of work per SM over the longest row of tiles
+    const int target = 8 * num_sms;
+    splits = (target + units - 1) / units;
+    splits = splits < 1 ? 1 : (splits > Nb ? Nb : splits);
+  }
+  p->tiles_per_split = (Nb + splits - 1) / splits;
+  p->splits = (Nb + p->tiles_per_split - 1) / p->tiles_per_split;
+  p->workspace_bytes = p->splits > 1 ? static_cast<size_t>(a.B) * a.Hq * a.L * p->splits * (a.Ev + 1) * sizeof(float)
+                                     : 0;
+  return 0;
+}
+
+cudaError_t launch_decode(const FwdArgs& a, const DecodePlan& p, const Sm100Maps& maps, void* workspace,
+                          cudaStream_t stream) {
+  return a.E == 64 ? launch_decode_d<64>(a, p, maps, workspace, stream)
+                   : launch_decode_d<128>(a, p, maps, workspace, stream);
+}
+
+}  // namespace fa

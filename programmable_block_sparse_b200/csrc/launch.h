@@ -54,16 +54,18 @@ struct Sm100Maps {
 };
 cudaError_t launch_fwd_sm100(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t stream);
 
-// Split-KV decode for short queries (bf16, E = Ev in {64, 128}) and the
-// log-sum-exp combination of its partial results.
+// Split-KV decode for short queries (bf16, E = Ev in {64, 128}, L <= 16) and
+// the log-sum-exp combination of its partial results.
 struct DecodePlan {
-  int rows_per_cta;   // query rows handled by one CTA (heads of a group x L), <= 16
-  int heads_per_cta;  // query heads per CTA
-  int splits;         // KV splits per (b, head group)
-  int tiles_per_split;
+  int rows_per_cta;     // query rows one CTA handles (heads of a group x L), <= 16
+  int heads_per_cta;    // query heads per CTA
+  int splits;           // KV splits per (b, head group)
+  int tiles_per_split;  // listed tiles per split
   size_t workspace_bytes;
 };
-int plan_decode(const FwdArgs& a, int split_kv, DecodePlan* plan);
-cudaError_t launch_decode(const FwdArgs& a, const DecodePlan& plan, void* workspace, cudaStream_t stream);
+constexpr int kDecodeMaxRows = 16;
+int plan_decode(const FwdArgs& a, int split_kv, int num_sms, DecodePlan* plan);
+cudaError_t launch_decode(const FwdArgs& a, const DecodePlan& plan, const Sm100Maps& maps, void* workspace,
+                          cudaStream_t stream);
 
 }  // namespace fa

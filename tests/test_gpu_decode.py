@@ -1,0 +1,103 @@
+"""Split-KV decode (short queries, long KV caches) vs the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_cases import Case, assert_close, bf16_tolerance
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from programmable_block_sparse_b200 import build
+    build.build()
+
+
+def _status_ok():
+    import programmable_block_sparse_b200 as fa
+    assert fa.flexattn_poll_device_status() == 0
+
+
+@pytest.mark.parametrize("split_kv", [0, 3, 1])
+@pytest.mark.parametrize("L,Hq,Hkv", [(1, 8, 2), (4, 8, 2), (16, 4, 4), (2, 32, 4), (3, 6, 2)])
+@pytest.mark.parametrize("E", [64, 128])
+def test_decode_against_oracle(L, Hq, Hkv, E, split_kv):
+    kv_len = [1500, 700, 129, 64]
+    case = Case(4, Hq, Hkv, L, 1500, E, E, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=L + E,
+                kv_len=kv_len, sentinel_tail=True)
+    out, lse = case.run(128, 128, split_kv=split_kv)
+    assert_close(case, out, lse, *case.oracle())
+    assert out.abs().max().item() < 10.0  # the +-1e4 cache tail never leaks
+    _status_ok()
+
+
+@pytest.mark.parametrize("mask", [{"kind": "none"}, {"kind": "sliding_window", "window": 200, "n_sink": 4},
+                                  {"kind": "chunked", "chunk": 300}, {"kind": "prefix_lm", "prefix": 100}],
+                         ids=lambda m: m["kind"])
+@pytest.mark.parametrize("score", [{"kind": "none"}, {"kind": "alibi"},
+                                   {"kind": "cap_then_bias", "cap": 30.0, "pos": "global"}], ids=lambda s: s["kind"])
+def test_decode_mask_and_score_kinds(mask, score):
+    case = Case(3, 8, 2, 4, 1000, 128, 128, "bf16", mask, score, seed=4, kv_len=[1000, 555, 77], sentinel_tail=True)
+    out, lse = case.run(128, 128, split_kv=4)
+    assert_close(case, out, lse, *case.oracle())
+    _status_ok()
+
+
+def test_decode_tiles_of_64_keys():
+    case = Case(2, 4, 1, 1, 640, 128, 128, "bf16", {"kind": "causal"}, {"kind": "none"}, seed=8, kv_len=[640, 100],
+                sentinel_tail=True)
+    out, lse = case.run(64, 64, split_kv=0)
+    assert_close(case, out, lse, *case.oracle())
+    _status_ok()
+
+
+def test_decode_rows_without_keys():
+    """kv_len smaller than L: the first rows see no key and give (0, -inf)."""
+    case = Case(2, 4, 2, 8, 256, 64, 64, "bf16", {"kind": "causal"}, {"kind": "none"}, seed=6, kv_len=[256, 5],
+                sentinel_tail=True)
+    out, lse = case.run(128, 128, split_kv=2)
+    assert torch.all(lse[1, :, :3] == -np.inf) and torch.all(out[1, :, :3] == 0)
+    assert_close(case, out, lse, *case.oracle())
+    _status_ok()
+
+
+def test_split_counts_agree():
+    import programmable_block_sparse_b200 as fa
+    case = Case(2, 8, 2, 4, 4096, 128, 128, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=1,
+                kv_len=[4096, 3000], sentinel_tail=True)
+    ref = None
+    for split in (1, 0, 2, 7, 32):
+        out, lse = case.run(128, 128, split_kv=split)
+        if ref is None:
+            ref = (out.float(), lse)
+            continue
+        assert (out.float() - ref[0]).abs().max().item() < 2e-2
+        assert (lse - ref[1]).abs().max().item() < 1e-4
+    bm = case.block_mask(128, 128)
+    need = fa.flexattn_forward_workspace_size(case.q, case.k, case.v, bm, split_kv=7)
+    assert need > 0
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fa.FlexAttnError) as e:
+        fa.flexattn_forward(case.q, case.k, case.v, bm, score_mod=case.dev_score, mask_mod=case.dev_mask,
+                            enable_gqa=True, split_kv=7, workspace=small)
+    assert e.value.status == 10
+    _status_ok()
+
+
+@pytest.mark.parametrize("L", [4, 1])
+def test_decode_workload_full_size(L):
+    case = Case.from_config("decode_kv_cache", L=L)
+    out, lse = case.run(case.BM, case.BN)
+    assert torch.isfinite(lse).all() and not torch.isnan(out).any()
+    assert out.abs().max().item() < 10.0
+    rng = np.random.default_rng(0)
+    samples = sorted({(int(rng.integers(case.B)), int(rng.integers(case.Hq)), int(rng.integers(L))) for _ in range(40)}
+                     | {(0, 0, 0), (case.B - 1, case.Hq - 1, L - 1)})
+    ref_o, ref_l = case.oracle_rows(samples)
+    got_o = np.stack([out[b, h, i].float().cpu().numpy() for b, h, i in samples]).astype(np.float64)
+    got_l = np.array([lse[b, h, i].item() for b, h, i in samples])
+    assert np.all(np.abs(got_o - ref_o) <= bf16_tolerance(ref_o)), np.abs(got_o - ref_o).max()
+    assert np.all(np.abs(got_l - ref_l) <= 1e-3), np.abs(got_l - ref_l).max()
+    _status_ok()
