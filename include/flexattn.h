@@ -14,7 +14,9 @@
  * Conventions shared by every entry point:
  *   - Every pointer to tensor data is DEVICE memory owned by the caller.  The
  *     library keeps no pointer after a call returns and allocates no device
- *     memory of its own (scratch comes from the caller's workspace).
+ *     memory during a call: scratch comes from the caller's workspace, except
+ *     in flexattn_forward_decode_noalloc, which uses a fixed array the library
+ *     holds for that purpose.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).  Host-side argument checks happen
  *     before anything is enqueued; on an error nothing is enqueued.
@@ -217,6 +219,36 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
                      float* lse, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
                      const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, int32_t split_kv,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* The split-KV decode of flexattn_forward, for callers that must not allocate
+ * device memory.  The pages have no counterpart of this entry point: it exists
+ * for code that runs where cudaMalloc is off limits -- inside a serving loop
+ * whose memory is fixed at start-up, between the steps of a captured CUDA
+ * graph, or in a host runtime with no allocator of its own -- and so cannot
+ * provide the workspace flexattn_forward asks for.
+ *
+ * Arguments and results are those of flexattn_forward, without the workspace:
+ * the partial results of the KV splits go to a scratch array inside the
+ * library, 16 MiB, which every GPU that loads the library holds until the
+ * process exits.  This call allocates nothing and calls no allocating
+ * routine.  The first call on a device looks up that array's device address
+ * (with that device current) and caches it; make that first call before any
+ * stream capture.
+ *
+ * All calls share the one array and it keeps whatever the last call wrote;
+ * nothing in it has to start at zero, because every split writes its slot
+ * before the combine step reads it.  Calls whose kernels overlap on the GPU
+ * (other streams, other threads) race on the array: serialise them.
+ *
+ * Only the decode path runs here (bf16, E == Ev in {64, 128}, L <= 16, one
+ * query tile, BN in {64, 128}, split_kv != 1); anything else returns
+ * FA_ERR_UNSUPPORTED.  A call needing more than 16 MiB of scratch
+ * (B * Hq * L * splits * (Ev + 1) * 4 bytes) returns FA_ERR_WORKSPACE.
+ * Other errors: those of flexattn_forward. */
+int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
+                                    float* lse, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
+                                    const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, int32_t split_kv,
+                                    void* stream);
 
 /* Wait for `stream`, then read and clear the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or an index check

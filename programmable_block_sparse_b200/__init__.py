@@ -27,7 +27,8 @@ from . import _abi
 __all__ = [
     "BlockMask", "FlexAttnError", "library_path", "load_library",
     "flexattn_version", "flexattn_last_error", "flexattn_block_mask_dims", "flexattn_build_block_mask",
-    "flexattn_forward_workspace_size", "flexattn_forward", "flexattn_poll_device_status",
+    "flexattn_forward_workspace_size", "flexattn_forward", "flexattn_forward_decode_noalloc",
+    "flexattn_poll_device_status",
 ]
 
 _LIB = None
@@ -222,6 +223,31 @@ def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=N
         C.byref(qs), C.byref(ks), C.byref(vs), C.byref(os_), _ptr(lse), C.c_float(sc), int(bool(enable_gqa)),
         C.byref(sm), C.byref(mm), C.byref(bm), int(split_kv), _ptr(workspace),
         C.c_size_t(workspace.numel() if workspace is not None else 0), _stream_handle(stream)))
+    return out, lse
+
+
+def flexattn_forward_decode_noalloc(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=None,
+                                    enable_gqa=False, out=None, lse=True, split_kv=0, stream=None):
+    """Split-KV decode without a workspace: for callers that cannot allocate
+    device memory at call time.  The library's built-in 16 MiB scratch holds
+    the per-split partial results; calls that overlap on the GPU share it and
+    must be serialised.  Returns ``(out, lse)``; ``out``/``lse`` may be
+    preallocated so that the call allocates nothing at all."""
+    import torch
+    B, Hq, L, _ = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, L, v.shape[3]), dtype=q.dtype, device=q.device)
+    if lse is True:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    elif lse is False:
+        lse = None
+    qs, ks, vs, os_ = _tensor_struct(q), _tensor_struct(k), _tensor_struct(v), _tensor_struct(out)
+    bm = block_mask.as_struct()
+    sm, mm = _score_struct(score_mod), _mask_struct(mask_mod)
+    sc = 0.0 if scale is None or math.isnan(float(scale)) else float(scale)
+    _check(load_library().flexattn_forward_decode_noalloc(
+        C.byref(qs), C.byref(ks), C.byref(vs), C.byref(os_), _ptr(lse), C.c_float(sc), int(bool(enable_gqa)),
+        C.byref(sm), C.byref(mm), C.byref(bm), int(split_kv), _stream_handle(stream)))
     return out, lse
 
 

@@ -63,6 +63,10 @@ PROTOTYPES = [
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
       C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),
       C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
+    ("flexattn_forward_decode_noalloc", C.c_int,
+     [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
+      C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),
+      C.c_int32, C.c_void_p]),
     ("flexattn_poll_device_status", C.c_int, [C.c_void_p, C.POINTER(C.c_int32)]),
 ]
 

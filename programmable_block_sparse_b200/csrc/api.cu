@@ -40,6 +40,37 @@ int* status_word(int* err) {
   return cache[dev];
 }
 
+// Scratch of flexattn_forward_decode_noalloc: a fixed device array that the
+// library owns, so that entry point never allocates.  It occupies this many
+// bytes on every GPU that loads the library, until the process exits.
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device.  Host code may
+// not use the array's name as a device pointer (it is a host-side stand-in),
+// so the address is asked of the runtime once per device, with that device
+// current, and cached.
+void* noalloc_scratch(int* err) {
+  static void* cache[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  *err = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *err = 1;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *err = 1;
+      return nullptr;
+    }
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+
 thread_local std::string t_last_error;
 
 int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
@@ -394,6 +425,39 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
     e = launch_fwd_simt(a, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return FA_OK;
+}
+
+int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
+                                    float* lse, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
+                                    const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, int32_t split_kv,
+                                    void* stream) {
+  if (!out) return fail(FA_ERR_NULL, "out is NULL");
+  FwdArgs a;
+  Path path;
+  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
+  if (rc) return rc;
+  if (path != Path::kDecode)
+    return fail(FA_ERR_UNSUPPORTED,
+                "the no-allocation entry point runs only the split-KV decode path (bf16, E == Ev in {64, 128}, "
+                "L <= 16, one query tile, BN in {64, 128}, split_kv != 1)");
+  DecodePlan plan;
+  plan_decode(a, split_kv, sm_count(), &plan);
+  if (plan.workspace_bytes > kNoAllocScratchBytes)
+    return fail(FA_ERR_WORKSPACE,
+                "this call needs %zu bytes of scratch but the built-in scratch holds %zu: pass fewer splits, or "
+                "use flexattn_forward with a caller-owned workspace",
+                plan.workspace_bytes, kNoAllocScratchBytes);
+  int err = 0;
+  void* scratch = noalloc_scratch(&err);
+  if (err) return fail(FA_ERR_CUDA, "cannot locate the built-in decode scratch on the current device");
+  a.status = status_word(&err);
+  if (err) return fail(FA_ERR_CUDA, "cannot locate the device status word");
+  a.lse = lse;
+  Sm100Maps maps;
+  if ((rc = encode_bf16_map(&maps.k, k, 64)) || (rc = encode_bf16_map(&maps.v, v, 64))) return rc;
+  cudaError_t e = launch_decode(a, plan, maps, scratch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return FA_OK;
 }
 
