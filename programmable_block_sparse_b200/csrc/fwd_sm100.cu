@@ -10,20 +10,28 @@
 // first); section "The compiler plugs local rules into the attention template"
 // (online softmax and tiling without materialising the score matrix).
 //
-// One CTA computes one 128-row query tile of one (batch, query head):
-//   warp 0      TMA producer: Q once, then K_j and V_j for every listed tile j
-//               into NS-stage rings (128 x 64 bf16 boxes, 128-byte swizzle).
-//   warp 1      TMEM allocator and MMA issuer (one elected thread):
-//               S[j%2] = Q K_j^T (SS form, both K-major), then
-//               O += P[j%2] V_j (TS form: P from TMEM, V MN-major in smem).
-//   warps 2-5   softmax warpgroup, one query row per thread (TMEM lane):
-//               load S_j, apply the score rule and (partial / edge tiles) the
-//               element mask, update the running max, write P_j = 2^(t - m) as
-//               bf16 into TMEM, keep the running sum; finally O / l and lse.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
-// The running max is only moved (and O rescaled) when it grows by more than
-// 2^8, so most tiles skip the O rescale; P then stays below 2^8, exact in the
-// final O / l ratio.
+// One CTA computes two adjacent 128-row query tiles (A = 2p, B = 2p + 1) of one
+// (batch, query head).  The two tiles' BlockMask lists are merged in key order
+// and every K/V tile of the union is loaded once for both:
+//   warp 0       TMA producer: Q_A, Q_B, then K_u, V_u of every union tile u
+//                into NS-stage rings (128 x 64 bf16 boxes, 128-byte swizzle).
+//   warp 1       TMEM allocator and MMA issuer (one elected thread):
+//                S_X = Q_X K_u^T (SS form, both K-major), O_X += P_X V_u (TS
+//                form: P from TMEM, V MN-major), for X in {A, B} and u in the
+//                tile's own list.
+//   warps 2-5    softmax group of tile A, warps 6-9 of tile B (warp % 4 picks
+//                the TMEM lane quadrant); one query
+//                row per thread (TMEM lane): S row -> score rule -> element mask
+//                (partial / edge tiles) -> running max -> P = 2^(t - m) as bf16
+//                into TMEM over the S columns it has read -> running sum;
+//                finally O / l and lse.  The two groups alternate on the tensor
+//                core: while one computes its softmax the other's MMAs run.
+// TMEM columns: tile X in {0, 1}: S/P at 256 X, O at 256 X + 128.
+// Ordering: the MMA thread issues PV_X(u) before QK_X(next), and the commit
+// that signals S_X(next) also covers PV_X(u), so a softmax group that sees its
+// S ready may read and rescale O_X and overwrite P_X without further waits.
+// The running max only moves (and O rescales) when it grows by more than 2^8;
+// P then stays below 2^8 and the final O / l ratio is exact.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records FA_ERR_TIMEOUT
 // in the status word, stops issuing work, drains its own copies and MMAs
@@ -38,27 +46,30 @@ namespace fa {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTile = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384;
 
 template <int D>
 struct Cfg {
-  static constexpr int kBoxes = D / 64;                  // 64-column boxes per tile row
-  static constexpr int kTileBytes = kTile * D * 2;       // one Q/K/V tile
+  static constexpr int kBoxes = D / 64;             // 64-column boxes per tile row
+  static constexpr int kTileBytes = kTile * D * 2;  // one Q/K/V tile
   static constexpr int kStages = D == 64 ? 4 : 2;
-  static constexpr int kSmemBytes = kTileBytes * (1 + 2 * kStages) + 1024;
+  static constexpr int kSmemBytes = kTileBytes * (2 + 2 * kStages) + 1024;
 };
+
+enum : uint32_t { kInA = 1, kFullA = 2, kInB = 4, kFullB = 8 };
+constexpr int kInfoFull = 1 << 30;  // class bit in the published tile info
 
 struct Barriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
-  uint64_t drain;
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_final;
+  int info[2][2];  // per group, ring of 2: tile index | kFullA-style class bit
   uint32_t tmem_base;
   int abort;
 };
@@ -69,11 +80,50 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ int tile_at(const FwdArgs& a, int64_t brow, int nfull, int j, bool* is_full) {
-  *is_full = j < nfull;
-  return *is_full ? __ldg(a.bm.full_kv_indices + brow * a.bm.Nb + j)
-                  : __ldg(a.bm.kv_indices + brow * a.bm.Nb + (j - nfull));
-}
+// Walks the union of the two query tiles' full and partial lists in
+// descending key order (for causal-like rules the nearest, highest-scoring
+// keys come first, so the running max rarely has to move afterwards).
+struct UnionIter {
+  const int* f[2];
+  const int* p[2];
+  int jf[2], jp[2];  // next index to take, counting down
+
+  __device__ void init(const FwdArgs& a, int64_t row_a, bool has_b) {
+    for (int t = 0; t < 2; ++t) {
+      const int64_t row = row_a + t;
+      const bool on = t == 0 || has_b;
+      f[t] = a.bm.full_kv_indices + row * a.bm.Nb;
+      p[t] = a.bm.kv_indices + row * a.bm.Nb;
+      jf[t] = (on ? __ldg(a.bm.full_kv_num_blocks + row) : 0) - 1;
+      jp[t] = (on ? __ldg(a.bm.kv_num_blocks + row) : 0) - 1;
+    }
+  }
+  __device__ bool next(int& n, uint32_t& flags) {
+    int c[4];
+    c[0] = jf[0] >= 0 ? __ldg(f[0] + jf[0]) : -1;
+    c[1] = jp[0] >= 0 ? __ldg(p[0] + jp[0]) : -1;
+    c[2] = jf[1] >= 0 ? __ldg(f[1] + jf[1]) : -1;
+    c[3] = jp[1] >= 0 ? __ldg(p[1] + jp[1]) : -1;
+    n = max(max(c[0], c[1]), max(c[2], c[3]));
+    if (n < 0) return false;
+    flags = 0;
+    if (c[0] == n) {
+      flags |= kInA | kFullA;
+      --jf[0];
+    } else if (c[1] == n) {
+      flags |= kInA;
+      --jp[0];
+    }
+    if (c[2] == n) {
+      flags |= kInB | kFullB;
+      --jf[1];
+    } else if (c[3] == n) {
+      flags |= kInB;
+      --jp[1];
+    }
+    return true;
+  }
+};
 
 // Bits [lo, hi] of a 32-bit word (positions relative to the word's first column).
 __device__ __forceinline__ uint32_t span_bits(int lo, int hi) {
@@ -84,34 +134,229 @@ __device__ __forceinline__ uint32_t span_bits(int lo, int hi) {
   return upto & ~((1u << lo) - 1u);
 }
 
-// One TMEM row of 128 fp32 columns into registers: eight loads in flight, one
-// wait.  The empty asm statements after the wait carry the registers as
-// read-write operands so no use of them is scheduled before the wait.
-__device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&t)[128]) {
+// 64 consecutive fp32 TMEM columns of this thread's row into registers: four
+// loads in flight, one wait.  The empty asm statements after the wait carry
+// the registers as read-write operands so no use is scheduled before it.
+__device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&t)[64]) {
   uint32_t* u = reinterpret_cast<uint32_t*>(t);
 #pragma unroll
-  for (int c = 0; c < 8; ++c) tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(u + c * 16));
+  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(u + c * 16));
   tmem_wait_ld();
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < 4; ++c) {
     uint32_t* x = u + c * 16;
     asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),
                  "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]),
                  "+r"(x[14]), "+r"(x[15]));
   }
 }
+__device__ __forceinline__ void tmem_store64(uint32_t taddr, const float (&t)[64]) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(t);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_st16(taddr + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(u + c * 16));
+}
 
-// Score rule in log2 units for one element; `d` = kv - q as a float.
-template <int SCORE>
-__device__ __forceinline__ float score_log2(float s, float c_in, float c_out, float slope2, float dist) {
-  if constexpr (SCORE == FA_SCORE_NONE) {
-    return s * c_out;
-  } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
-    return c_out * tanh_fast(s * c_in);
-  } else if constexpr (SCORE == FA_SCORE_ALIBI) {
-    return fmaf(s, c_out, slope2 * dist);
+// Softmax and epilogue of one 128-row query tile; runs on one warpgroup.
+template <int D, int SCORE>
+__device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, float (*s_pos)[kTile],
+                                              int (*s_doc)[kTile], int X, int mt, int h, int b, int S_b,
+                                              int64_t row_a, bool has_b, uint32_t tbase) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const int grow = mt * kTile + r;
+  const bool row_ok = grow < a.L;
+  const int qpos = query_pos(grow, a.L, S_b);
+  const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+  const uint32_t col_s = 256u * X, col_o = 256u * X + 128u;
+  volatile int* abort = &bars.abort;
+  const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
+  const float slope2 = distance_slope(h, Hs) * kLog2e;
+  float c_in, c_out;
+  if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) {
+    c_in = a.scale / a.score.cap;
+    c_out = a.score.cap * kLog2e;
   } else {
-    return fmaf(c_out, tanh_fast(s * c_in), slope2 * dist);
+    c_in = 0.0f;
+    c_out = a.scale * kLog2e;
+  }
+  const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
+  const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
+  const bool is_doc = a.mask.kind == FA_MASK_DOCUMENT;
+  const int* doc_row = is_doc ? a.mask.doc_id + static_cast<int64_t>(a.mask.doc_batch > 1 ? b : 0) * a.S : nullptr;
+  const int my_doc = (is_doc && row_ok && qpos >= 0) ? __ldg(doc_row + qpos) : -1;
+  const KeySpans spans = visible_spans(a.mask, qpos, S_b);
+  float m_ref = -INFINITY, l_sum = 0.0f;
+  bool alive = true;
+  int cnt = 0;
+
+  const int64_t row_x = row_a + X;
+  const bool x_on = X == 0 || has_b;
+  const int total = x_on ? __ldg(a.bm.full_kv_num_blocks + row_x) + __ldg(a.bm.kv_num_blocks + row_x) : 0;
+  for (; cnt < total; ++cnt) {
+    if (!mbar_wait(&bars.s_full[X], cnt & 1, abort, a.status)) {
+      alive = false;
+      break;
+    }
+    const int info = bars.info[X][cnt & 1];
+    const int n = info & (kInfoFull - 1);
+    const bool full = (info & kInfoFull) != 0;
+    const int kv0 = n * kTile;
+    const bool edge = kv0 + kTile > S_b;
+    const bool stage_doc = is_doc && (!full || edge);  // the same for every row of the tile
+    if (has_pos || stage_doc) {
+      // this tile's key-side values into smem (double-buffered by cnt & 1)
+      const int kv = kv0 + r;
+      if (has_pos) s_pos[cnt & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
+      if (stage_doc) s_doc[cnt & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
+      named_bar_sync(1 + X, 128);
+    }
+    tc_fence_after();
+
+    // pass 1, per 64-column half: score rule on every cell, element mask on
+    // partial tiles / ragged edges / rows past L, row max; the transformed
+    // scores go back to TMEM for pass 2
+    const bool need_mask = !full || edge || !row_ok;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float t[64];
+      const int c0 = 64 * half;
+      tmem_load64(tbase + lane_base + col_s + c0, t);
+      if constexpr (SCORE == FA_SCORE_NONE) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) t[c] *= c_out;
+      } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) t[c] = c_out * tanh_fast(t[c] * c_in);
+      } else if constexpr (SCORE == FA_SCORE_ALIBI) {
+        const float bias0 = slope2 * static_cast<float>(kv0 + c0 - qpos);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) t[c] = fmaf(t[c], c_out, fmaf(slope2, static_cast<float>(c), bias0));
+      } else {
+        if (has_pos) {
+          const float* pk = s_pos[cnt & 1] + c0;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), pk[c] - pq_scaled);
+        } else {
+          const float bias0 = slope2 * static_cast<float>(kv0 + c0 - qpos);
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), fmaf(slope2, static_cast<float>(c), bias0));
+        }
+      }
+      if (need_mask) {
+        uint32_t bits[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int base = kv0 + c0 + 32 * w;
+          bits[w] = row_ok ? (span_bits(spans.a0 - base, spans.a1 - base) |
+                              span_bits(spans.b0 - base, spans.b1 - base))
+                           : 0u;
+        }
+        if (stage_doc) {
+          const int* dk = s_doc[cnt & 1] + c0;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            uint32_t same = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) same |= (dk[32 * w + i] == my_doc ? 1u : 0u) << i;
+            bits[w] &= same;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (!((bits[c >> 5] >> (c & 31)) & 1u)) t[c] = -INFINITY;
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, t[c]);
+      tmem_store64(tbase + lane_base + col_s + c0, t);
+    }
+    tmem_wait_st();
+
+    // running max: move it (and rescale O) only when it grows past 2^8.  O_X
+    // holds the sum through this group's previous tile: the commit behind
+    // s_full covered that PV, and no MMA writes O_X until P_X is signalled.
+    const bool grow_max = mx > m_ref + kRescaleThreshold;
+    const float m_new = grow_max ? mx : m_ref;
+    const bool rescale = grow_max && m_ref != -INFINITY;
+    if (__any_sync(0xffffffffu, rescale)) {
+      const float f = rescale ? ex2_approx(m_ref - m_new) : 1.0f;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t rr[16];
+        tmem_ld16(tbase + lane_base + col_o + c * 16, rr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+        tmem_st16(tbase + lane_base + col_o + c * 16, rr);
+      }
+      l_sum *= f;
+    }
+    m_ref = m_new;
+    const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+
+    // pass 2, per half: P = 2^(t - m) as bf16 pairs over the first 64 columns
+    // (half h writes columns [32 h, 32 h + 32), all of which pass 2 has read)
+    float psum = 0.0f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float t[64];
+      tmem_load64(tbase + lane_base + col_s + 64 * half, t);
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        t[c] = ex2_approx(t[c] - m_use);
+        psum += t[c];
+      }
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[32 * g + 2 * i], t[32 * g + 2 * i + 1]);
+        tmem_st16(tbase + lane_base + col_s + 32 * half + 16 * g, pk);
+      }
+    }
+    l_sum += psum;
+
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.p_full[X]);
+  }
+
+  // ------------------------------------------------------------- epilogue
+  if (alive && cnt > 0) {
+    alive = mbar_wait(&bars.o_final, 0, abort, a.status);
+    tc_fence_after();
+  }
+  // TMEM loads are warp-collective: every lane takes part, rows past L
+  // included; only the stores depend on the row.
+  if (__all_sync(0xffffffffu, alive)) {
+    const bool live = l_sum > 0.0f && cnt > 0;
+    const float inv = live ? 1.0f / l_sum : 0.0f;
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] +
+                          static_cast<int64_t>(row_ok ? grow : 0) * a.o_stride[2];
+    if (row_ok && a.lse)
+      a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.L + grow] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t rr[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) rr[i] = 0u;
+      if (cnt > 0) {
+        tmem_ld16(tbase + lane_base + col_o + c * 16, rr);
+        tmem_wait_ld();
+      }
+      if (row_ok) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
   }
 }
 
@@ -123,22 +368,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Barriers bars;
-  __shared__ float s_pos[2][kTile];  // slope * position of the tile's keys (score with positions)
-  __shared__ int s_doc[2][kTile];    // document ids of the tile's keys (partial document tiles)
+  __shared__ float s_pos[2][2][kTile];  // per group: slope * position of the tile's keys
+  __shared__ int s_doc[2][2][kTile];    // per group: document ids of the tile's keys
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::kTileBytes;
+  uint8_t* sQ = smem;  // Q_A, Q_B
+  uint8_t* sK = sQ + 2 * C::kTileBytes;
   uint8_t* sV = sK + NS * C::kTileBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = gridDim.x - 1 - blockIdx.x;  // longest rows of tiles first
+  const int pair = gridDim.x - 1 - blockIdx.x;  // longest rows of tiles first
   const int h = blockIdx.y, b = blockIdx.z;
+  const int mtA = 2 * pair, mtB = 2 * pair + 1;
+  const bool has_b = mtB < a.bm.Mb;
   const int hk = h / a.G;
   const int S_b = seq_len_b(a.mask, b, a.S);
   const int bmb = a.bm.B > 1 ? b : 0, bmh = a.bm.H > 1 ? h : 0;
-  const int64_t brow = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb + mt;
-  const int nfull = __ldg(a.bm.full_kv_num_blocks + brow);
-  const int ntiles = nfull + __ldg(a.bm.kv_num_blocks + brow);
+  const int64_t row_a = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb + mtA;
   volatile int* abort = &bars.abort;
 
   if (threadIdx.x == 0) {
@@ -150,12 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_free[i], 4);
+      mbar_init(&bars.s_full[i], 2);  // the QK commit + the MMA thread's tile-info arrive
       mbar_init(&bars.p_full[i], 4);
-      mbar_init(&bars.pv_done[i], 1);
     }
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
   }
@@ -167,275 +410,141 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
-    if (lane == 0 && ntiles > 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-      mbar_expect_tx(&bars.q_full, C::kTileBytes);
-      for (int c = 0; c < C::kBoxes; ++c)
-        tma_load_4d(sQ + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mt * kTile, h, b);
-      int issued = 0;
-      for (int j = 0; j < ntiles && !*abort; ++j) {
-        bool full;
-        const int n = tile_at(a, brow, nfull, j, &full);
-        const int s = j % NS;
-        const uint32_t round = j / NS;
-        if (j >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status)) break;
-        mbar_expect_tx(&bars.k_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kBoxes; ++c)
-          tma_load_4d(sK + s * C::kTileBytes + c * (kTile * 128), &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
-        if (j >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status)) {
-          issued = j + 1;  // K_j is in flight
-          break;
+    if (lane == 0) {
+      UnionIter it;
+      it.init(a, row_a, has_b);
+      int n;
+      uint32_t flags;
+      bool any = it.next(n, flags);
+      if (any) {
+        tma_prefetch_desc(&map_k);
+        tma_prefetch_desc(&map_v);
+        mbar_expect_tx(&bars.q_full, (has_b ? 2 : 1) * C::kTileBytes);
+        for (int c = 0; c < C::kBoxes; ++c) {
+          tma_load_4d(sQ + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mtA * kTile, h, b);
+          if (has_b)
+            tma_load_4d(sQ + C::kTileBytes + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mtB * kTile, h, b);
         }
-        mbar_expect_tx(&bars.v_full[s], C::kTileBytes);
-        for (int c = 0; c < C::kBoxes; ++c)
-          tma_load_4d(sV + s * C::kTileBytes + c * (kTile * 128), &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
-        issued = j + 1;
-      }
-      if (*abort) {
-        // Drain: let every copy this thread issued land before the CTA exits.
-        volatile int never = 0;
-        mbar_wait(&bars.q_full, 0, &never, nullptr);
-        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) {
-          mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
-          mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
+        int u = 0, issued = 0;
+        for (; any && !*abort; ++u, any = it.next(n, flags)) {
+          const int s = u % NS;
+          const uint32_t round = u / NS;
+          if (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status)) break;
+          mbar_expect_tx(&bars.k_full[s], C::kTileBytes);
+          for (int c = 0; c < C::kBoxes; ++c)
+            tma_load_4d(sK + s * C::kTileBytes + c * (kTile * 128), &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
+          issued = u + 1;
+          if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status)) break;
+          mbar_expect_tx(&bars.v_full[s], C::kTileBytes);
+          for (int c = 0; c < C::kBoxes; ++c)
+            tma_load_4d(sV + s * C::kTileBytes + c * (kTile * 128), &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
+        }
+        if (*abort) {
+          // drain: let every copy this thread issued land before the CTA exits
+          volatile int never = 0;
+          mbar_wait(&bars.q_full, 0, &never, nullptr);
+          for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) {
+            mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
+            mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(&bars.q_full, 0, abort, a.status);
-      auto issue_pv = [&](int t) -> bool {
-        const int s = t % NS;
-        if (!mbar_wait(&bars.v_full[s], (t / NS) & 1, abort, a.status)) return false;
-        if (!mbar_wait(&bars.p_full[t & 1], (t >> 1) & 1, abort, a.status)) return false;
+      UnionIter it;
+      it.init(a, row_a, has_b);
+      int n_cur, n_nxt = 0;
+      uint32_t f_cur, f_nxt = 0;
+      bool have_cur = it.next(n_cur, f_cur);
+      int pcnt[2] = {0, 0};  // P tiles consumed per group
+      bool acc[2] = {false, false};
+      int qcnt[2] = {0, 0};  // QK tiles issued per group
+      auto issue_qk = [&](int X, int s, int n, uint32_t flags) {
+        // publish the tile index and class for the softmax group (released by
+        // this thread's arrive; the phase completes with the MMA commit below)
+        bars.info[X][qcnt[X] & 1] = n | ((flags & (X == 0 ? kFullA : kFullB)) ? kInfoFull : 0);
+        ++qcnt[X];
+        mbar_arrive(&bars.s_full[X]);
+        const uint32_t qx = q_addr + X * C::kTileBytes, ks = k_addr + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
+          umma_ss(tbase + 256u * X, umma_desc_sw128(qx + off, 16, 1024), umma_desc_sw128(ks + off, 16, 1024),
+                  idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars.s_full[X]);
+      };
+      auto issue_pv = [&](int X, int s) -> bool {
+        if (!mbar_wait(&bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
         tc_fence_after();
-        const uint32_t p_tmem = tbase + kColP0 + 64 * (t & 1);
         const uint32_t vs = v_addr + s * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
           const uint64_t bdesc = umma_desc_sw128(vs + kk * 16 * 128, kTile * 128, 1024);
-          umma_ts(tbase + kColO, p_tmem + kk * 8, bdesc, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tbase + 256u * X + 128u, tbase + 256u * X + kk * 8, bdesc, idesc_pv, (acc[X] || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars.pv_done[t & 1]);
-        umma_commit(&bars.v_empty[s]);
+        acc[X] = true;
+        ++pcnt[X];
         return true;
       };
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(&bars.k_full[s], (j / NS) & 1, abort, a.status)) break;
-        if (j >= 2 && !mbar_wait(&bars.s_free[j & 1], ((j - 2) >> 1) & 1, abort, a.status)) break;
+      bool ok = have_cur && mbar_wait(&bars.q_full, 0, abort, a.status);
+      if (ok) {
+        ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
         tc_fence_after();
-        const uint32_t ks = k_addr + s * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
-          umma_ss(tbase + kColS0 + 128 * (j & 1), umma_desc_sw128(q_addr + off, 16, 1024),
-                  umma_desc_sw128(ks + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        if (ok) {
+          if (f_cur & kInA) issue_qk(0, 0, n_cur, f_cur);
+          if (f_cur & kInB) issue_qk(1, 0, n_cur, f_cur);
+          umma_commit(&bars.k_empty[0]);
         }
-        umma_commit(&bars.s_full[j & 1]);
-        umma_commit(&bars.k_empty[s]);
-        if (j >= 1 && !issue_pv(j - 1)) break;
       }
-      if (!*abort) issue_pv(ntiles - 1);
-      // All MMAs this thread issued complete before TMEM is released.
-      umma_commit(&bars.drain);
+      for (int u = 0; ok && have_cur; ++u) {
+        const int s = u % NS, s1 = (u + 1) % NS;
+        const bool have_nxt = it.next(n_nxt, f_nxt);
+        bool k_nxt_ready = false;
+        if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status)) break;
+        for (int X = 0; X < 2 && ok; ++X) {
+          const uint32_t in_x = X == 0 ? kInA : kInB;
+          if (f_cur & in_x) ok = issue_pv(X, s);
+          if (ok && have_nxt && (f_nxt & in_x)) {
+            if (!k_nxt_ready) {
+              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+              tc_fence_after();
+              k_nxt_ready = true;
+            }
+            if (ok) issue_qk(X, s1, n_nxt, f_nxt);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&bars.v_empty[s]);
+        if (have_nxt) {
+          if (!k_nxt_ready) {
+            // K_{u+1} is listed for neither group's next QK only if a group
+            // skips it; it still has to be consumed before its slot is reused
+            ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+            if (!ok) break;
+          }
+          umma_commit(&bars.k_empty[s1]);
+        }
+        have_cur = have_nxt;
+        n_cur = n_nxt;
+        f_cur = f_nxt;
+      }
+      (void)n_cur;
+      // every MMA issued above completes before the epilogue or TMEM release
+      umma_commit(&bars.o_final);
       volatile int never = 0;
-      mbar_wait(&bars.drain, 0, &never, nullptr);
+      mbar_wait(&bars.o_final, 0, &never, nullptr);
     }
   } else {
     // -------------------------------------------------------------- softmax
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int grow = mt * kTile + r;
-    const bool row_ok = grow < a.L;
-    const int qpos = query_pos(grow, a.L, S_b);
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
-    const float slope2 = distance_slope(h, Hs) * kLog2e;
-    float c_in, c_out;
-    if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) {
-      c_in = a.scale / a.score.cap;
-      c_out = a.score.cap * kLog2e;
-    } else {
-      c_in = 0.0f;
-      c_out = a.scale * kLog2e;
-    }
-    const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
-    const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
-    const bool is_doc = a.mask.kind == FA_MASK_DOCUMENT;
-    const int* doc_row = is_doc ? a.mask.doc_id + static_cast<int64_t>(a.mask.doc_batch > 1 ? b : 0) * a.S : nullptr;
-    const int my_doc = (is_doc && row_ok && qpos >= 0) ? __ldg(doc_row + qpos) : -1;
-    const KeySpans spans = visible_spans(a.mask, qpos, S_b);
-    float m_ref = -INFINITY, l_sum = 0.0f;
-    bool alive = true;
-
-    for (int j = 0; j < ntiles; ++j) {
-      bool full;
-      const int n = tile_at(a, brow, nfull, j, &full);
-      const int kv0 = n * kTile;
-      const bool edge = kv0 + kTile > S_b;
-      const bool stage_doc = is_doc && (!full || edge);  // the same for every row of the tile
-      if (has_pos || stage_doc) {
-        // stage this tile's key-side values in smem (double-buffered by j & 1)
-        const int kv = kv0 + r;
-        if (has_pos) s_pos[j & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
-        if (stage_doc) s_doc[j & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
-        named_bar_sync(1, 128);
-      }
-      if (!mbar_wait(&bars.s_full[j & 1], (j >> 1) & 1, abort, a.status)) {
-        alive = false;
-        break;
-      }
-      tc_fence_after();
-      float t[kTile];
-      tmem_load_row128(tbase + lane_base + kColS0 + 128 * (j & 1), t);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[j & 1]);
-
-      // score rule on every cell (log2 units)
-      if constexpr (SCORE == FA_SCORE_NONE) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) t[c] *= c_out;
-      } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) t[c] = c_out * tanh_fast(t[c] * c_in);
-      } else if constexpr (SCORE == FA_SCORE_ALIBI) {
-        const float bias0 = slope2 * static_cast<float>(kv0 - qpos);
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) t[c] = fmaf(t[c], c_out, fmaf(slope2, static_cast<float>(c), bias0));
-      } else {
-        if (has_pos) {
-          const float* pk = s_pos[j & 1];
-#pragma unroll
-          for (int c = 0; c < kTile; ++c) t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), pk[c] - pq_scaled);
-        } else {
-          const float bias0 = slope2 * static_cast<float>(kv0 - qpos);
-#pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), fmaf(slope2, static_cast<float>(c), bias0));
-        }
-      }
-
-      // element mask on partial tiles, ragged edges and rows past L
-      if (!full || edge || !row_ok) {
-        uint32_t bits[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int base = kv0 + 32 * w;
-          bits[w] = row_ok ? (span_bits(spans.a0 - base, spans.a1 - base) | span_bits(spans.b0 - base, spans.b1 - base))
-                           : 0u;
-        }
-        if (stage_doc) {
-          const int* dk = s_doc[j & 1];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t same = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) same |= (dk[32 * w + i] == my_doc ? 1u : 0u) << i;
-            bits[w] &= same;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (!((bits[c >> 5] >> (c & 31)) & 1u)) t[c] = -INFINITY;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, t[c]);
-
-      // running max: move it (and rescale O) only when it grows past 2^8
-      const bool grow_max = mx > m_ref + kRescaleThreshold;
-      const float m_new = grow_max ? mx : m_ref;
-      const bool rescale = grow_max && m_ref != -INFINITY;
-      if (__any_sync(0xffffffffu, rescale) && j > 0) {
-        // O holds the sum through tile j-1: wait for that PV, then scale in place
-        if (!mbar_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, a.status)) {
-          alive = false;
-          break;
-        }
-        tc_fence_after();
-        const float f = rescale ? ex2_approx(m_ref - m_new) : 1.0f;
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t rr[16];
-          tmem_ld16(tbase + lane_base + kColO + c * 16, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
-          tmem_st16(tbase + lane_base + kColO + c * 16, rr);
-        }
-        tmem_wait_st();
-        l_sum *= f;
-      }
-      m_ref = m_new;
-      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float psum = 0.0f;
-#pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        t[c] = ex2_approx(t[c] - m_use);
-        psum += t[c];
-      }
-      l_sum += psum;
-
-      // P_j goes to TMEM buffer j%2 once PV_{j-2} has consumed it
-      if (j >= 2 && !mbar_wait(&bars.pv_done[j & 1], ((j - 2) >> 1) & 1, abort, a.status)) {
-        alive = false;
-        break;
-      }
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[c * 32 + 2 * i], t[c * 32 + 2 * i + 1]);
-        tmem_st16(tbase + lane_base + kColP0 + 64 * (j & 1) + c * 16, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full[j & 1]);
-    }
-
-    // ------------------------------------------------------------ epilogue
-    if (alive && ntiles > 0) {
-      alive = mbar_wait(&bars.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, a.status);
-      tc_fence_after();
-    }
-    // TMEM loads are warp-collective: every lane takes part, rows past L
-    // included; only the stores depend on the row.
-    if (__all_sync(0xffffffffu, alive)) {
-      const bool live = l_sum > 0.0f && ntiles > 0;
-      const float inv = live ? 1.0f / l_sum : 0.0f;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] +
-                            static_cast<int64_t>(row_ok ? grow : 0) * a.o_stride[2];
-      if (row_ok && a.lse)
-        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.L + grow] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t rr[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) rr[i] = 0u;
-        if (ntiles > 0) {
-          tmem_ld16(tbase + lane_base + kColO + c * 16, rr);
-          tmem_wait_ld();
-        }
-        if (row_ok) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
-    }
+    // warps 2-5: tile A, warps 6-9: tile B; warp % 4 is the TMEM lane quadrant
+    const int X = (warp - 2) >> 2;
+    softmax_group<D, SCORE>(a, bars, s_pos[X], s_doc[X], X, X == 0 ? mtA : mtB, h, b, S_b, row_a, has_b, tbase);
   }
 
   tc_fence_before();
@@ -449,7 +558,7 @@ cudaError_t launch_one(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t str
   auto kern = fwd_sm100_kernel<D, SCORE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.bm.Mb, a.Hq, a.B);
+  dim3 grid((a.bm.Mb + 1) / 2, a.Hq, a.B);
   kern<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(a, maps.q, maps.k, maps.v);
   return cudaGetLastError();
 }
