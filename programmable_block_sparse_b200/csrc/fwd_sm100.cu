@@ -455,7 +455,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // Base smem descriptors, built once; per-MMA descriptors only add the
+      // (address >> 4) offset of the K step or stage to the start-address
+      // field, which keeps the issue path short.
+      const uint64_t dq0 = umma_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv0 = umma_desc_sw128(smem_u32(sV), kTile * 128, 1024);
+      constexpr uint32_t kTileStep = C::kTileBytes >> 4;
       UnionIter it;
       it.init(a, row_a, has_b);
       int n_cur, n_nxt = 0;
@@ -470,24 +476,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars.info[X][qcnt[X] & 1] = n | ((flags & (X == 0 ? kFullA : kFullB)) ? kInfoFull : 0);
         ++qcnt[X];
         mbar_arrive(&bars.s_full[X]);
-        const uint32_t qx = q_addr + X * C::kTileBytes, ks = k_addr + s * C::kTileBytes;
+        const uint64_t dq = dq0 + X * kTileStep, dk = dk0 + s * kTileStep;
+        const uint32_t d_tmem = tbase + 256u * X;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTile * 128) + (kk & 3) * 32;
-          umma_ss(tbase + 256u * X, umma_desc_sw128(qx + off, 16, 1024), umma_desc_sw128(ks + off, 16, 1024),
-                  idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * (kTile * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(d_tmem, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars.s_full[X]);
       };
       auto issue_pv = [&](int X, int s) -> bool {
         if (!mbar_wait(&bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
         tc_fence_after();
-        const uint32_t vs = v_addr + s * C::kTileBytes;
+        const uint64_t dv = dv0 + s * kTileStep;
+        const uint32_t o_tmem = tbase + 256u * X + 128u, p_tmem = tbase + 256u * X;
+        const uint32_t acc0 = acc[X] ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t bdesc = umma_desc_sw128(vs + kk * 16 * 128, kTile * 128, 1024);
-          umma_ts(tbase + 256u * X + 128u, tbase + 256u * X + kk * 8, bdesc, idesc_pv, (acc[X] || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
         acc[X] = true;
         ++pcnt[X];
         return true;
