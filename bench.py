@@ -38,15 +38,28 @@ METRIC_PREFILL = "visible-score TFLOP/s & % BF16 tensor peak (prefill); KV GB/s 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the forward kernel,
-# from the ncu capture summarised under profiles/, keyed by workload; valid only
-# while the kernel source hashes to the recorded value.
-NCU_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
+# kernel, from the ncu captures summarised under profiles/, keyed by workload;
+# valid only while that kernel's sources hash to the recorded value.
+#  - causal_softcap_alibi: fwd_sm100_kernel, full workload, one launch
+#    (50.417408 MB read + 1.241088 MB written).
+#  - decode_kv_cache: decode_kernel captured at batch 8 (454.419456 MB read +
+#    9.769472 MB written over 110440 cached tokens), scaled to the full batch
+#    of 32 by cached tokens (614602): traffic grows with the tokens streamed.
+NCU_TRAFFIC = {
+    "causal_softcap_alibi": {"bytes": 51658496, "source_hash": "cf294bd830293192"},
+    "decode_kv_cache": {"bytes": 2583225675, "source_hash": "1d71549d51afb208"},
+}
+
+KERNEL_SOURCES = {
+    "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh"),
+    "decode": ("decode.cu", "mods.cuh", "common.cuh"),
+}
 
 
-def kernel_source_hash():
+def kernel_source_hash(kind="prefill"):
     h = hashlib.sha256()
-    for name in ("fwd_sm100.cu", "mods.cuh", "common.cuh"):
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, "programmable_block_sparse_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -177,9 +190,11 @@ def describe(name, c):
     return f"{name}", d
 
 
-def make_inputs(name, device, seed_offset=0):
+def make_inputs(name, device, seed_offset=0, batch=None):
     import torch
     c = wl.config(name)
+    if batch:
+        c["B"] = int(batch)
     kv_len = doc_lengths = None
     if name == "decode_kv_cache":
         kv_len = wl.decode_cache_lengths(c["B"], c["kv_lo"], c["kv_hi"], c["seed"])
@@ -259,7 +274,12 @@ def oracle_sample_rate(name, target_s=12.0, max_heads=None):
         if el >= target_s or (max_heads and heads >= max_heads):
             break
     cores = len(os.sched_getaffinity(0))
-    sample = f"{heads} of {c['B'] * c['Hq']} (batch, query head) units, every query row in full"
+    units = c["B"] * c["Hq"]
+    if heads <= units:
+        sample = f"{heads} of the {units} (batch, query head) units, every query row in full"
+    else:
+        sample = (f"{heads} (batch, query head) unit evaluations, cycling over all {units} units "
+                  f"({heads / units:.2f} passes), every query row in full")
     if decode:
         return work / el / 1e9, el, cores, sample, heads, "GB/s"
     return work / el / 1e12, el, cores, sample, heads, "TFLOP/s"
@@ -315,7 +335,7 @@ def run_gpu(args):
     fa.load_library()
 
     name = args.workload
-    c, (q_h, k_h, v_h), mask, score, kv_len, doc_lengths = make_inputs(name, dev, seed_offset=rank)
+    c, (q_h, k_h, v_h), mask, score, kv_len, doc_lengths = make_inputs(name, dev, seed_offset=rank, batch=args.batch)
     B, Hq, L, E, Ev = c["B"], c["Hq"], c["L"], c["E"], c["Ev"]
     BM, BN = c["BM"], c["BN"]
     B_mask = B if kv_len is not None else 1
@@ -329,6 +349,8 @@ def run_gpu(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     decode = name == "decode_kv_cache"
+    # classifier + forward kernel, + the log-sum-exp combine when decode splits the keys
+    launches_per_step = 2 + (1 if decode and ws_bytes > 0 else 0)
     flop_pair = 2 * E + 2 * Ev
     vis_pairs = visible_pairs_per_head(c, kv_len, doc_lengths) * Hq
     vis_flops = vis_pairs * flop_pair
@@ -434,14 +456,15 @@ def run_gpu(args):
                     "frac": achieved / peaks["bf16_tflops"], "peak_source": f"bf16_tflops (burst) of {peak_src}",
                     "flops_counted_over": "visited-tile cells, (2E + 2Ev) per cell"}
         e2e_val = world * vis_flops / (e2e_ms * 1e-3) / 1e12
+    src_hash = kernel_source_hash("decode" if decode else "prefill")
     tr = NCU_TRAFFIC.get(name)
-    roofline["traffic"] = tr["bytes"] if tr and tr["source_hash"] == kernel_source_hash() else None
+    roofline["traffic"] = tr["bytes"] if tr and tr["source_hash"] == src_hash and not args.batch else None
 
     line = {
         "metric": METRIC_PREFILL, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if c["dtype"] == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": describe(name, c)[0], **describe(name, c)[1],
+        "config": {"workload": name, **describe(name, c)[1],
                    "l2": "flushed: 256 MiB written between timed steps, outside the events",
                    "step": "block-mask build + forward",
                    "parallelism": f"weak scaling over {world} GPU(s): each rank runs the full per-GPU workload"},
@@ -450,10 +473,10 @@ def run_gpu(args):
                    "visible_pairs": vis_pairs, "visited_cells": cells,
                    "visible_tflops_forward_only": vis_flops / (fwd_mean * 1e-3) / 1e12,
                    "visited_tflops_forward_only": visited_flops / (fwd_mean * 1e-3) / 1e12,
-                   "kernel_source": kernel_source_hash()},
+                   "kernel_source": src_hash},
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
@@ -473,6 +496,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller captures for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

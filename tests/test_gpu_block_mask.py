@@ -79,6 +79,24 @@ def test_document_mask_bit_exact(shape, sorted_ids):
     _compare({"kind": "document", "doc_id": ids}, 1, 1, L, S, BM, BN)
 
 
+@pytest.mark.parametrize("pattern", ["random3", "alternating", "single", "blocks_of_5"])
+@pytest.mark.parametrize("shape", [(200, 200, 16, 32), (300, 300, 128, 128), (129, 257, 64, 128), (97, 97, 128, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_document_mask_interleaved_ids(shape, pattern):
+    """Ids that repeat out of order: up to BN runs per tile, one id in many runs."""
+    L, S, BM, BN = shape
+    rng = np.random.default_rng(S + BN)
+    if pattern == "random3":
+        ids = rng.integers(0, 3, S)
+    elif pattern == "alternating":
+        ids = np.arange(S) % 2
+    elif pattern == "single":
+        ids = np.zeros(S)
+    else:
+        ids = (np.arange(S) // 5) % 3
+    _compare({"kind": "document", "doc_id": ids.astype(np.int32)}, 1, 1, L, S, BM, BN)
+
+
 @pytest.mark.parametrize("mask", MASKS[:6] + [{"kind": "document"}], ids=lambda m: m["kind"])
 def test_per_sequence_kv_len_and_head_broadcast(mask):
     B, H, L, S = 3, 2, 7, 333
