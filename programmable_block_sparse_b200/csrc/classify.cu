@@ -13,9 +13,8 @@
 // sliding window with sinks, prefix-LM, chunked) every query row sees a union
 // of at most two key intervals, so a tile is classified from per-row
 // intersection counts (BM work per tile instead of BM x BN).  The document
-// rule is checked cell by cell with a warp-wide early exit once both a
-// visible and a hidden cell are seen, after a sound shortcut: a tile whose row
-// and column document-id ranges are disjoint has no visible cell.
+// rule counts the same way over runs of equal document id (see
+// classify_tile_document).
 #include "common.cuh"
 #include "launch.h"
 #include "mods.cuh"
@@ -56,58 +55,66 @@ __device__ uint8_t classify_tile_intervals(const MaskParams& m, int r0, int r1, 
   return all_full ? kFull : (any_vis ? kPartial : kEmpty);
 }
 
-__device__ uint8_t classify_tile_cells(const MaskParams& m, int b, int r0, int r1, int c0, int c1, int L, int S,
-                                       int S_b) {
+// Document rule: key kv is visible to query q when kv <= q, kv < S_b and
+// doc[kv] == doc[q].  The tile's columns [c0, chi] (chi = last in-range key)
+// are cut into runs of equal document id (at most BN <= 128 of them, found
+// with ballots and written to this warp's slice of shared memory); a row's
+// visible count is the summed overlap of [c0, min(q, chi)] with the runs whose
+// id equals doc[q].  Exact for any id layout; a packed batch of documents has
+// one or two runs per tile, so a tile costs about BM / 32 steps per lane.
+__device__ uint8_t classify_tile_document(const MaskParams& m, int b, int r0, int r1, int c0, int c1, int L, int S,
+                                          int S_b, int* run_a, int* run_id) {
   const int lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
-  if (m.kind == FA_MASK_DOCUMENT) {
-    // Disjoint document-id ranges: nothing in the tile can be visible.
-    const int* d = m.doc_id + static_cast<int64_t>(m.doc_batch > 1 ? b : 0) * S;
-    int rmin = INT32_MAX, rmax = INT32_MIN, cmin = INT32_MAX, cmax = INT32_MIN;
-    for (int r = r0 + lane; r <= r1; r += 32) {
-      int q = query_pos(r, L, S_b);
-      if (q >= 0 && q < S) {
-        int v = __ldg(d + q);
-        rmin = min(rmin, v);
-        rmax = max(rmax, v);
+  const int* d = m.doc_id + static_cast<int64_t>(m.doc_batch > 1 ? b : 0) * S;
+  const int chi = min(c1, S_b - 1);
+  int nr = 0;
+  int prev_last = 0;
+  for (int base = c0; base <= chi; base += 32) {
+    const int c = base + lane;
+    const bool valid = c <= chi;
+    const int v = valid ? __ldg(d + c) : 0;
+    int prev = __shfl_up_sync(full, v, 1);
+    if (lane == 0) prev = prev_last;
+    const bool start = valid && (c == c0 || v != prev);
+    const unsigned bal = __ballot_sync(full, start);
+    if (start) {
+      const int idx = nr + __popc(bal & ((1u << lane) - 1u));
+      run_a[idx] = c;
+      run_id[idx] = v;
+    }
+    nr += __popc(bal);
+    prev_last = __shfl_sync(full, v, 31);
+  }
+  if (lane == 0) run_a[nr] = chi + 1;
+  __syncwarp();
+  const int width = c1 - c0 + 1;
+  bool all_full = true, any_vis = false;
+  for (int r = r0 + lane; r <= r1; r += 32) {
+    const int q = query_pos(r, L, S_b);
+    const int hi = min(q, chi);
+    int cnt = 0;
+    if (hi >= c0) {
+      const int dq = __ldg(d + q);
+      for (int k = 0; k < nr; ++k) {
+        const int a = run_a[k];
+        if (a > hi) break;
+        if (run_id[k] == dq) cnt += min(run_a[k + 1] - 1, hi) - a + 1;
       }
     }
-    int chi = min(c1, S_b - 1);
-    for (int c = c0 + lane; c <= chi; c += 32) {
-      int v = __ldg(d + c);
-      cmin = min(cmin, v);
-      cmax = max(cmax, v);
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      rmin = min(rmin, __shfl_xor_sync(full, rmin, o));
-      rmax = max(rmax, __shfl_xor_sync(full, rmax, o));
-      cmin = min(cmin, __shfl_xor_sync(full, cmin, o));
-      cmax = max(cmax, __shfl_xor_sync(full, cmax, o));
-    }
-    if (rmin > rmax || cmin > cmax || cmax < rmin || cmin > rmax) return kEmpty;
+    all_full &= (cnt == width);
+    any_vis |= (cnt > 0);
   }
-  const int nr = r1 - r0 + 1, nc = c1 - c0 + 1;
-  const int64_t cells = static_cast<int64_t>(nr) * nc;
-  bool seen_vis = false, seen_hid = false;
-  for (int64_t base = 0; base < cells; base += 32) {
-    int64_t idx = base + lane;
-    bool vis = false, hid = false;
-    if (idx < cells) {
-      int r = r0 + static_cast<int>(idx / nc);
-      int c = c0 + static_cast<int>(idx % nc);
-      bool v = mask_visible(m, b, query_pos(r, L, S_b), c, S_b, S);
-      vis = v;
-      hid = !v;
-    }
-    seen_vis |= __any_sync(full, vis);
-    seen_hid |= __any_sync(full, hid);
-    if (seen_vis && seen_hid) break;
-  }
-  return seen_vis ? (seen_hid ? kPartial : kFull) : kEmpty;
+  all_full = __all_sync(full, all_full);
+  any_vis = __any_sync(full, any_vis);
+  __syncwarp();  // run_a / run_id are rewritten for the warp's next tile
+  return all_full ? kFull : (any_vis ? kPartial : kEmpty);
 }
 
 __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs a) {
   extern __shared__ uint8_t cls[];
+  __shared__ int s_run_a[kClassifyThreads / 32][129];
+  __shared__ int s_run_id[kClassifyThreads / 32][128];
   const int mt = blockIdx.x;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,7 +133,7 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs
     if (c0 >= S_b || (causal_family && c0 > q_hi)) {
       k = kEmpty;
     } else if (a.mask.kind == FA_MASK_DOCUMENT) {
-      k = classify_tile_cells(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b);
+      k = classify_tile_document(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b, s_run_a[warp], s_run_id[warp]);
     } else {
       k = classify_tile_intervals(a.mask, r0, r1, c0, c1, a.L, S_b);
     }
