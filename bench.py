@@ -314,6 +314,33 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank plumbing (one process per GPU; no collective on the data path)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, device, world):
+    """The largest of every rank's ``value`` (a device time in ms): the job's time."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_rank, world, ms_per_step, scale):
+    """Weak scaling: every rank does ``work_per_rank`` per step; the job's rate
+    is all ranks' work over the slowest rank's step time, in units of ``scale``."""
+    return world * work_per_rank / (ms_per_step * 1e-3) / scale
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 
@@ -322,9 +349,7 @@ def run_gpu(args):
     import torch.distributed as dist
     import programmable_block_sparse_b200 as fa
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     if world > 1:
         torch.cuda.set_device(local)
         from datetime import timedelta
@@ -396,11 +421,7 @@ def run_gpu(args):
     mask_ms = [a.elapsed_time(b) for a, b, _ in ev]
     fwd_ms = [b.elapsed_time(c_) for _, b, c_ in ev]
     step_ms = [a.elapsed_time(c_) for a, _, c_ in ev]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev, world)
     if fa.flexattn_poll_device_status() != 0:
         raise RuntimeError("device status word set during the timed region")
 
@@ -425,11 +446,7 @@ def run_gpu(args):
         ee[i][1].record(stream)
         flush.zero_()
     torch.cuda.synchronize()
-    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in ee)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ee), dev, world)
     h2d = (q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size())
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
@@ -442,20 +459,20 @@ def run_gpu(args):
     ms_per_step = total_ms / args.steps
     fwd_mean = statistics.mean(fwd_ms)
     if decode:
-        value = world * kv_bytes / (ms_per_step * 1e-3) / 1e9
+        value = whole_job_rate(kv_bytes, world, ms_per_step, 1e9)
         unit = "GB/s"
         achieved = kv_bytes / (fwd_mean * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}"}
-        e2e_val = world * kv_bytes / (e2e_ms * 1e-3) / 1e9
+        e2e_val = whole_job_rate(kv_bytes, world, e2e_ms, 1e9)
     else:
-        value = world * vis_flops / (ms_per_step * 1e-3) / 1e12
+        value = whole_job_rate(vis_flops, world, ms_per_step, 1e12)
         unit = "TFLOP/s"
         achieved = visited_flops / (fwd_mean * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": achieved / peaks["bf16_tflops"], "peak_source": f"bf16_tflops (burst) of {peak_src}",
                     "flops_counted_over": "visited-tile cells, (2E + 2Ev) per cell"}
-        e2e_val = world * vis_flops / (e2e_ms * 1e-3) / 1e12
+        e2e_val = whole_job_rate(vis_flops, world, e2e_ms, 1e12)
     src_hash = kernel_source_hash("decode" if decode else "prefill")
     tr = NCU_TRAFFIC.get(name)
     roofline["traffic"] = tr["bytes"] if tr and tr["source_hash"] == src_hash and not args.batch else None
