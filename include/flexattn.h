@@ -41,7 +41,7 @@ extern "C" {
 enum {
   FA_OK = 0,
   FA_ERR_NULL = 1,         /* a required pointer is NULL                                   */
-  FA_ERR_SHAPE = 2,        /* a size is non-positive or q/k/v/out sizes disagree           */
+  FA_ERR_SHAPE = 2,        /* a size is non-positive, above 65535 for batch or heads, or sizes disagree */
   FA_ERR_HEADS = 3,        /* Hq != Hkv without enable_gqa, or Hq % Hkv != 0 ([guide] 1.3, 6.1) */
   FA_ERR_BATCH = 4,        /* batch sizes disagree, or a broadcast extent is neither 1 nor B    */
   FA_ERR_MASK_SHAPE = 5,   /* block mask built for other lengths/blocks: "too small / too large" ([guide] 1.3) */

@@ -260,6 +260,8 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   const int B = (int)q->size[0], Hq = (int)q->size[1], L = (int)q->size[2], E = (int)q->size[3];
   const int Hkv = (int)k->size[1], S = (int)k->size[2], Ev = (int)v->size[3];
   if (k->size[0] != B || v->size[0] != B) return fail(FA_ERR_BATCH, "q, k and v must have the same batch size");
+  // launch grids carry the batch and the head count in their y / z extents
+  if (B > 65535 || Hq > 65535) return fail(FA_ERR_SHAPE, "batch and head counts above 65535 are not supported");
   if (k->size[3] != E) return fail(FA_ERR_SHAPE, "k head dim %lld != q head dim %d", (long long)k->size[3], E);
   if (v->size[1] != Hkv || v->size[2] != S) return fail(FA_ERR_SHAPE, "v must be (B, Hkv, S, Ev) like k");
   if (out && (out->size[0] != B || out->size[1] != Hq || out->size[2] != L || out->size[3] != Ev))
@@ -316,7 +318,7 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   const bool decode_ok = tc_shape && tma_ok && L <= kDecodeMaxRows && bm->Mb == 1 && bm->BN % 64 == 0;
   if (split_kv != 1 && decode_ok) {
     *path = Path::kDecode;
-  } else if (tc_shape && tma_ok && out_ok && bm->BM == 128 && bm->BN == 128) {
+  } else if (tc_shape && tma_ok && out_ok && bm->BM == 128 && bm->BN == 128 && (bm->Mb + 1) / 2 <= 65535) {
     *path = Path::kSm100;
   } else {
     *path = Path::kSimt;
@@ -443,6 +445,12 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
                 "L <= 16, one query tile, BN in {64, 128}, split_kv != 1)");
   DecodePlan plan;
   plan_decode(a, split_kv, sm_count(), &plan);
+  if (split_kv == 0 && plan.workspace_bytes > kNoAllocScratchBytes) {
+    // automatic split count: take the most splits the built-in scratch holds
+    const size_t per_split = static_cast<size_t>(a.B) * a.Hq * a.L * (a.Ev + 1) * sizeof(float);
+    const size_t fit = kNoAllocScratchBytes / per_split;
+    if (fit >= 2) plan_decode(a, static_cast<int32_t>(fit < 65536 ? fit : 65536), sm_count(), &plan);
+  }
   if (plan.workspace_bytes > kNoAllocScratchBytes)
     return fail(FA_ERR_WORKSPACE,
                 "this call needs %zu bytes of scratch but the built-in scratch holds %zu: pass fewer splits, or "

@@ -26,10 +26,15 @@
 //                into TMEM over the S columns it has read -> running sum;
 //                finally O / l and lse.  The two groups alternate on the tensor
 //                core: while one computes its softmax the other's MMAs run.
-// TMEM columns: tile X in {0, 1}: S/P at 256 X, O at 256 X + 128.
-// Ordering: the MMA thread issues PV_X(u) before QK_X(next), and the commit
-// that signals S_X(next) also covers PV_X(u), so a softmax group that sees its
-// S ready may read and rescale O_X and overwrite P_X without further waits.
+// TMEM columns of tile X in {0, 1}: at head dim 128, S/P at 256 X (P as bf16
+// pairs over the first 64 S columns, once read) and O at 256 X + 128; the
+// MMA thread issues PV_X(u) before QK_X(next), and the commit that signals
+// S_X(next) also covers PV_X(u), so a softmax group that sees its S ready may
+// read and rescale O_X and overwrite P_X without further waits.  At head dim
+// 64, S at 256 X, P at 256 X + 128 and O at 256 X + 192 have columns of their
+// own: QK_X(next) is issued as soon as the group has read S (s_free), ahead
+// of PV_X(u), and the group waits for that PV (o_done) only before it writes
+// P or rescales O.
 // The running max only moves (and O rescales) when it grows by more than 2^8;
 // P then stays below 2^8 and the final O / l ratio is exact.
 //
@@ -68,6 +73,7 @@ struct Barriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
+  uint64_t s_free[2], o_done[2];  // head dim 64 only: S read out / PV finished
   uint64_t o_final;
   int info[2][2];  // per group, ring of 2: tile index | kFullA-style class bit
   uint32_t tmem_base;
@@ -84,42 +90,47 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // descending key order (for causal-like rules the nearest, highest-scoring
 // keys come first, so the running max rarely has to move afterwards).
 struct UnionIter {
-  const int* f[2];
-  const int* p[2];
-  int jf[2], jp[2];  // next index to take, counting down
+  // lists 0 / 1: full / partial of tile A; 2 / 3: full / partial of tile B
+  const int* lst[4];
+  int j[4];  // index of each list's head, counting down
+  int c[4];  // head values (-1 once a list is exhausted), loaded a step ahead
+             // so that next() does not wait on global-memory latency
 
   __device__ void init(const FwdArgs& a, int64_t row_a, bool has_b) {
+#pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int64_t row = row_a + t;
       const bool on = t == 0 || has_b;
-      f[t] = a.bm.full_kv_indices + row * a.bm.Nb;
-      p[t] = a.bm.kv_indices + row * a.bm.Nb;
-      jf[t] = (on ? __ldg(a.bm.full_kv_num_blocks + row) : 0) - 1;
-      jp[t] = (on ? __ldg(a.bm.kv_num_blocks + row) : 0) - 1;
+      lst[2 * t] = a.bm.full_kv_indices + row * a.bm.Nb;
+      lst[2 * t + 1] = a.bm.kv_indices + row * a.bm.Nb;
+      j[2 * t] = (on ? __ldg(a.bm.full_kv_num_blocks + row) : 0) - 1;
+      j[2 * t + 1] = (on ? __ldg(a.bm.kv_num_blocks + row) : 0) - 1;
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = j[i] >= 0 ? __ldg(lst[i] + j[i]) : -1;
+  }
+  template <int I>
+  __device__ __forceinline__ void advance() {
+    --j[I];
+    c[I] = j[I] >= 0 ? __ldg(lst[I] + j[I]) : -1;
   }
   __device__ bool next(int& n, uint32_t& flags) {
-    int c[4];
-    c[0] = jf[0] >= 0 ? __ldg(f[0] + jf[0]) : -1;
-    c[1] = jp[0] >= 0 ? __ldg(p[0] + jp[0]) : -1;
-    c[2] = jf[1] >= 0 ? __ldg(f[1] + jf[1]) : -1;
-    c[3] = jp[1] >= 0 ? __ldg(p[1] + jp[1]) : -1;
     n = max(max(c[0], c[1]), max(c[2], c[3]));
     if (n < 0) return false;
     flags = 0;
     if (c[0] == n) {
       flags |= kInA | kFullA;
-      --jf[0];
+      advance<0>();
     } else if (c[1] == n) {
       flags |= kInA;
-      --jp[0];
+      advance<1>();
     }
     if (c[2] == n) {
       flags |= kInB | kFullB;
-      --jf[1];
+      advance<2>();
     } else if (c[3] == n) {
       flags |= kInB;
-      --jp[1];
+      advance<3>();
     }
     return true;
   }
@@ -168,7 +179,13 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   const bool row_ok = grow < a.L;
   const int qpos = query_pos(grow, a.L, S_b);
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-  const uint32_t col_s = 256u * X, col_o = 256u * X + 128u;
+  // head dim 64: S, P and O each have their own columns (S at 256 X, P at
+  // 256 X + 128, O at 256 X + 192), so the next tile's S can be computed
+  // while this tile's P is still being written.  Head dim 128: P overwrites
+  // the S columns it has read and O sits at 256 X + 128.
+  constexpr bool kSepP = D == 64;
+  const uint32_t col_s = 256u * X, col_o = 256u * X + (kSepP ? 192u : 128u);
+  const uint32_t col_p = kSepP ? 256u * X + 128u : col_s;
   volatile int* abort = &bars.abort;
   const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
   const float slope2 = distance_slope(h, Hs) * kLog2e;
@@ -218,7 +235,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     // scores go back to TMEM for pass 2
     const bool need_mask = !full || edge || !row_ok;
     float mx = -INFINITY;
-#pragma unroll
+#pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       float t[64];
       const int c0 = 64 * half;
@@ -275,12 +292,24 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     tmem_wait_st();
 
     // running max: move it (and rescale O) only when it grows past 2^8.  O_X
-    // holds the sum through this group's previous tile: the commit behind
-    // s_full covered that PV, and no MMA writes O_X until P_X is signalled.
+    // holds the sum through this group's previous tile once that PV is done:
+    // at head dim 128 the commit behind s_full covered it; at head dim 64 the
+    // o_done barrier says so.  No MMA writes O_X until P_X is signalled.
     const bool grow_max = mx > m_ref + kRescaleThreshold;
     const float m_new = grow_max ? mx : m_ref;
     const bool rescale = grow_max && m_ref != -INFINITY;
+    bool pv_done = !kSepP || cnt == 0;
+    auto wait_pv = [&]() {
+      // the previous tile's PV reads P and writes O; with separate S columns
+      // the S of this tile may have landed before that PV finished
+      if (!pv_done) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[X], (cnt - 1) & 1, abort, a.status))) alive = false;
+        tc_fence_after();
+        pv_done = true;
+      }
+    };
     if (__any_sync(0xffffffffu, rescale)) {
+      wait_pv();
       const float f = rescale ? ex2_approx(m_ref - m_new) : 1.0f;
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
@@ -296,25 +325,38 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     m_ref = m_new;
     const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
 
-    // pass 2, per half: P = 2^(t - m) as bf16 pairs over the first 64 columns
-    // (half h writes columns [32 h, 32 h + 32), all of which pass 2 has read)
+    // pass 2, per half: P = 2^(t - m) as bf16 pairs, 64 columns in all
+    // (head dim 128: over the first 64 S columns; half h writes columns
+    // [32 h, 32 h + 32), all of which pass 2 has read)
     float psum = 0.0f;
-#pragma unroll
+#pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       float t[64];
       tmem_load64(tbase + lane_base + col_s + 64 * half, t);
+      if (kSepP && half == 1) {
+        // all of S is in registers now: the next tile's QK may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free[X]);
+      }
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         t[c] = ex2_approx(t[c] - m_use);
         psum += t[c];
       }
+      if (half == 0) wait_pv();
+      if (!alive) break;
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[32 * g + 2 * i], t[32 * g + 2 * i + 1]);
-        tmem_st16(tbase + lane_base + col_s + 32 * half + 16 * g, pk);
+        tmem_st16(tbase + lane_base + col_p + 32 * half + 16 * g, pk);
       }
+    }
+    if (!alive) {
+      tmem_wait_st();
+      break;
     }
     l_sum += psum;
 
@@ -376,8 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = sK + NS * C::kTileBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = gridDim.x - 1 - blockIdx.x;  // longest rows of tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // Blocks start in linear order (x fastest, z slowest): with the query-tile
+  // pair in z, counted down, every (batch, head)'s last pairs -- the longest
+  // rows of tiles under causal-like rules -- start first and the short ones
+  // fill in at the end, instead of long CTAs starting in the last wave.
+  const int pair = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int mtA = 2 * pair, mtB = 2 * pair + 1;
   const bool has_b = mtB < a.bm.Mb;
   const int hk = h / a.G;
@@ -397,6 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 2);  // the QK commit + the MMA thread's tile-info arrive
       mbar_init(&bars.p_full[i], 4);
+      mbar_init(&bars.s_free[i], 4);
+      mbar_init(&bars.o_done[i], 1);
     }
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
@@ -499,46 +547,117 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       bool ok = have_cur && mbar_wait(&bars.q_full, 0, abort, a.status);
-      if (ok) {
-        ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
-        tc_fence_after();
+      if constexpr (D == 64) {
+        // S, P and O in separate columns: the next tile's QK of a group goes
+        // in as soon as its softmax has read S (s_free), ahead of this
+        // tile's PV (p_full), so the next S is ready when the softmax needs it.
+        int freed[2] = {0, 0};  // S tiles of each group read out so far
+        auto issue_pv_sep = [&](int X, int s) -> bool {
+          if (!mbar_wait(&bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
+          tc_fence_after();
+          const uint64_t dv = dv0 + s * kTileStep;
+          const uint32_t o_tmem = tbase + 256u * X + 192u, p_tmem = tbase + 256u * X + 128u;
+          const uint32_t acc0 = acc[X] ? 1u : 0u;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          umma_commit(&bars.o_done[X]);
+          acc[X] = true;
+          ++pcnt[X];
+          return true;
+        };
+        auto qk_after_free = [&](int X, int s, int n, uint32_t flags) -> bool {
+          if (qcnt[X] > 0) {  // the group's previous S must be read out first
+            if (!mbar_wait(&bars.s_free[X], freed[X] & 1, abort, a.status)) return false;
+            ++freed[X];
+            tc_fence_after();
+          }
+          issue_qk(X, s, n, flags);
+          return true;
+        };
         if (ok) {
-          if (f_cur & kInA) issue_qk(0, 0, n_cur, f_cur);
-          if (f_cur & kInB) issue_qk(1, 0, n_cur, f_cur);
-          umma_commit(&bars.k_empty[0]);
+          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
+          tc_fence_after();
+          if (ok && (f_cur & kInA)) ok = qk_after_free(0, 0, n_cur, f_cur);
+          if (ok && (f_cur & kInB)) ok = qk_after_free(1, 0, n_cur, f_cur);
+          if (ok) umma_commit(&bars.k_empty[0]);
         }
-      }
-      for (int u = 0; ok && have_cur; ++u) {
-        const int s = u % NS, s1 = (u + 1) % NS;
-        const bool have_nxt = it.next(n_nxt, f_nxt);
-        bool k_nxt_ready = false;
-        if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status)) break;
-        for (int X = 0; X < 2 && ok; ++X) {
-          const uint32_t in_x = X == 0 ? kInA : kInB;
-          if (f_cur & in_x) ok = issue_pv(X, s);
-          if (ok && have_nxt && (f_nxt & in_x)) {
-            if (!k_nxt_ready) {
-              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
-              tc_fence_after();
-              k_nxt_ready = true;
+        for (int u = 0; ok && have_cur; ++u) {
+          const int s = u % NS, s1 = (u + 1) % NS;
+          const bool have_nxt = it.next(n_nxt, f_nxt);
+          bool k_ready = false, v_ready = false;
+          for (int X = 0; X < 2 && ok; ++X) {
+            const uint32_t in_x = X == 0 ? kInA : kInB;
+            if (have_nxt && (f_nxt & in_x)) {
+              if (!k_ready) {
+                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+                tc_fence_after();
+                k_ready = true;
+              }
+              if (ok) ok = qk_after_free(X, s1, n_nxt, f_nxt);
             }
-            if (ok) issue_qk(X, s1, n_nxt, f_nxt);
+            if (ok && (f_cur & in_x)) {
+              if (!v_ready) {
+                ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status);
+                tc_fence_after();
+                v_ready = true;
+              }
+              if (ok) ok = issue_pv_sep(X, s);
+            }
+          }
+          if (!ok) break;
+          // every union tile is some group's tile, and so is the next one
+          umma_commit(&bars.v_empty[s]);
+          if (have_nxt) {
+            if (!k_ready && !mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status)) break;
+            umma_commit(&bars.k_empty[s1]);
+          }
+          have_cur = have_nxt;
+          n_cur = n_nxt;
+          f_cur = f_nxt;
+        }
+      } else {
+        if (ok) {
+          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
+          tc_fence_after();
+          if (ok) {
+            if (f_cur & kInA) issue_qk(0, 0, n_cur, f_cur);
+            if (f_cur & kInB) issue_qk(1, 0, n_cur, f_cur);
+            umma_commit(&bars.k_empty[0]);
           }
         }
-        if (!ok) break;
-        umma_commit(&bars.v_empty[s]);
-        if (have_nxt) {
-          if (!k_nxt_ready) {
-            // K_{u+1} is listed for neither group's next QK only if a group
-            // skips it; it still has to be consumed before its slot is reused
-            ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
-            if (!ok) break;
+        for (int u = 0; ok && have_cur; ++u) {
+          const int s = u % NS, s1 = (u + 1) % NS;
+          const bool have_nxt = it.next(n_nxt, f_nxt);
+          bool k_nxt_ready = false;
+          if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status)) break;
+          for (int X = 0; X < 2 && ok; ++X) {
+            const uint32_t in_x = X == 0 ? kInA : kInB;
+            if (f_cur & in_x) ok = issue_pv(X, s);
+            if (ok && have_nxt && (f_nxt & in_x)) {
+              if (!k_nxt_ready) {
+                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+                tc_fence_after();
+                k_nxt_ready = true;
+              }
+              if (ok) issue_qk(X, s1, n_nxt, f_nxt);
+            }
           }
-          umma_commit(&bars.k_empty[s1]);
+          if (!ok) break;
+          umma_commit(&bars.v_empty[s]);
+          if (have_nxt) {
+            if (!k_nxt_ready) {
+              // K_{u+1} is listed for neither group's next QK only if a group
+              // skips it; it still has to be consumed before its slot is reused
+              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+              if (!ok) break;
+            }
+            umma_commit(&bars.k_empty[s1]);
+          }
+          have_cur = have_nxt;
+          n_cur = n_nxt;
+          f_cur = f_nxt;
         }
-        have_cur = have_nxt;
-        n_cur = n_nxt;
-        f_cur = f_nxt;
       }
       (void)n_cur;
       // every MMA issued above completes before the epilogue or TMEM release
@@ -564,7 +683,7 @@ cudaError_t launch_one(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t str
   auto kern = fwd_sm100_kernel<D, SCORE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.bm.Mb + 1) / 2, a.Hq, a.B);
+  dim3 grid(a.Hq, a.B, (a.bm.Mb + 1) / 2);
   kern<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(a, maps.q, maps.k, maps.v);
   return cudaGetLastError();
 }

@@ -68,3 +68,15 @@ def test_noalloc_refuses_oversized_scratch():
     with pytest.raises(fa.FlexAttnError) as e:
         fa.flexattn_forward_decode_noalloc(case.q, case.k, case.v, bm, mask_mod=case.dev_mask, split_kv=32)
     assert e.value.status == 10 and "scratch" in str(e.value)
+
+
+def test_noalloc_automatic_split_count():
+    """With split_kv = 0 the entry point picks its own split count (capped by
+    what the built-in scratch holds) and matches the workspace entry point on
+    a decode-sized cache: 8 sequences of 4096-32768 keys, 64 query heads over
+    8 KV heads, 16 query rows."""
+    rng = np.random.default_rng(5)
+    kv_len = rng.integers(4096, 32769, 8).tolist()
+    case = Case(8, 64, 8, 16, 32768, 64, 64, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=9,
+                kv_len=kv_len, sentinel_tail=True)
+    _compare(case, split_kv=0)
