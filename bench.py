@@ -42,12 +42,16 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel, from the ncu captures summarised under profiles/, keyed by workload;
 # valid only while that kernel's sources hash to the recorded value.
 #  - causal_softcap_alibi: fwd_sm100_kernel, full workload, one launch
-#    (50.417408 MB read + 1.241088 MB written).
+#    (50.407680 MB read + 1.167872 MB written).
+#  - gqa_sliding_window: fwd_sm100_kernel captured at batch 1 (201.633536 MB
+#    read + 100.084992 MB written), doubled for the batch of 2: both
+#    sequences carry the same work.
 #  - decode_kv_cache: decode_kernel captured at batch 8 (454.419456 MB read +
 #    9.769472 MB written over 110440 cached tokens), scaled to the full batch
 #    of 32 by cached tokens (614602): traffic grows with the tokens streamed.
 NCU_TRAFFIC = {
-    "causal_softcap_alibi": {"bytes": 51658496, "source_hash": "cf294bd830293192"},
+    "causal_softcap_alibi": {"bytes": 51575552, "source_hash": "50727d24277efc09"},
+    "gqa_sliding_window": {"bytes": 603437056, "source_hash": "50727d24277efc09"},
     "decode_kv_cache": {"bytes": 2583225675, "source_hash": "1d71549d51afb208"},
 }
 
