@@ -39,6 +39,7 @@ constexpr int kStagesDec = 3;
 constexpr int kRows = 16;       // query rows per CTA (one m16 fragment)
 constexpr float kLog2eD = 1.4426950408889634f;
 constexpr float kLn2D = 0.6931471805599453f;
+constexpr float kRescaleThresholdD = 8.0f;  // log2 units
 
 template <int D>
 struct DecCfg {
@@ -89,7 +90,7 @@ __device__ __forceinline__ int list_tile(const FwdArgs& a, int64_t brow, int nfu
                    : __ldg(a.bm.kv_indices + brow * a.bm.Nb + (j - nfull));
 }
 
-template <int D>
+template <int D, int SCORE>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_kernel(const FwdArgs a, const DecodePlan p, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, float* ws_o, float* ws_lse) {
@@ -190,6 +191,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       qpos[half] = query_pos(rho % a.L, a.L, S_b);
       slope2[half] = distance_slope(hq[half], Hs);
     }
+    // score rule constants in log2 units (SCORE is fixed at compile time)
+    const float c_in = (SCORE == FA_SCORE_SOFTCAP) ? a.scale / a.score.cap : 0.0f;
+    const float c_out = (SCORE == FA_SCORE_SOFTCAP) ? a.score.cap * kLog2eD : a.scale * kLog2eD;
     float o[D / 8][4];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
@@ -225,23 +229,52 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         for (int e = 0; e < 4; ++e) {
           const int half = e >> 1;
           const int kv = kv0 + 16 * cw + 8 * nt + 2 * quad + (e & 1);
-          float g = score_apply<false>(a.score, sc[nt][e] * a.scale, b, qpos[half], kv, a.S, slope2[half]) * kLog2eD;
+          float g;
+          if constexpr (SCORE == FA_SCORE_NONE) {
+            g = sc[nt][e] * c_out;
+          } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
+            g = c_out * tanh_fast(sc[nt][e] * c_in);
+          } else if constexpr (SCORE == FA_SCORE_ALIBI) {
+            g = fmaf(sc[nt][e], c_out, -slope2[half] * kLog2eD * static_cast<float>(qpos[half] - kv));
+          } else {
+            g = score_apply<false>(a.score, sc[nt][e] * a.scale, b, qpos[half], kv, a.S, slope2[half]) * kLog2eD;
+          }
           const bool vis = rok[half] && (!need_mask || mask_visible(a.mask, b, qpos[half], kv, S_b, a.S));
           g = vis ? g : -INFINITY;
           sc[nt][e] = g;
           mx[half] = fmaxf(mx[half], g);
         }
       }
-      float alpha[2], mu[2];
+      // The running max moves (and O, l rescale) only when a row's max grows
+      // by more than 2^8 or on its first visible key; P then stays below 2^8
+      // and O / l is unchanged.  The four lanes of a row share its max, so
+      // they decide alike.
+      bool grow[2];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 1));
         mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 2));
-        const float m_new = fmaxf(m_run[half], mx[half]);
-        alpha[half] = (m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - m_new);
-        m_run[half] = m_new;
-        mu[half] = (m_new == -INFINITY) ? 0.0f : m_new;
+        grow[half] = mx[half] > m_run[half] + kRescaleThresholdD;
       }
+      if (__any_sync(0xffffffffu, grow[0] || grow[1])) {
+        float alpha[2];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          alpha[half] = grow[half] ? ((m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - mx[half])) : 1.0f;
+          if (grow[half]) m_run[half] = mx[half];
+          l_run[half] *= alpha[half];
+        }
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          o[i][0] *= alpha[0];
+          o[i][1] *= alpha[0];
+          o[i][2] *= alpha[1];
+          o[i][3] *= alpha[1];
+        }
+      }
+      float mu[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) mu[half] = (m_run[half] == -INFINITY) ? 0.0f : m_run[half];
       float ps[2] = {0.0f, 0.0f};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -251,14 +284,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           ps[e >> 1] += sc[nt][e];
         }
 #pragma unroll
-      for (int half = 0; half < 2; ++half) l_run[half] = l_run[half] * alpha[half] + ps[half];
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        o[i][0] *= alpha[0];
-        o[i][1] *= alpha[0];
-        o[i][2] *= alpha[1];
-        o[i][3] *= alpha[1];
-      }
+      for (int half = 0; half < 2; ++half) l_run[half] += ps[half];
       uint32_t pa[4];
       pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
       pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
@@ -386,11 +412,14 @@ cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Ma
   const int head_chunks = (a.G + p.heads_per_cta - 1) / p.heads_per_cta;
   float* ws_o = static_cast<float*>(workspace);
   float* ws_lse = ws_o ? ws_o + static_cast<int64_t>(a.B) * a.Hq * a.L * p.splits * D : nullptr;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       DecCfg<D>::kSmemBytes);
+  auto kern = a.score.kind == FA_SCORE_NONE      ? decode_kernel<D, FA_SCORE_NONE>
+              : a.score.kind == FA_SCORE_SOFTCAP ? decode_kernel<D, FA_SCORE_SOFTCAP>
+              : a.score.kind == FA_SCORE_ALIBI   ? decode_kernel<D, FA_SCORE_ALIBI>
+                                                 : decode_kernel<D, FA_SCORE_CAP_THEN_BIAS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.splits, a.Hkv * head_chunks, a.B);
-  decode_kernel<D><<<grid, kDecThreads, DecCfg<D>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse);
+  kern<<<grid, kDecThreads, DecCfg<D>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
