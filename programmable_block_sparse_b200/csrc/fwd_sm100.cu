@@ -73,6 +73,7 @@ struct Barriers {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
+  uint64_t p_half[2];  // the first 64 keys' P is written: their PV may start
   uint64_t s_free[2], o_done[2];  // head dim 64 only: S read out / PV finished
   uint64_t o_final;
   int info[2][2];  // per group, ring of 2: tile index | kFullA-style class bit
@@ -353,6 +354,14 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[32 * g + 2 * i], t[32 * g + 2 * i + 1]);
         tmem_st16(tbase + lane_base + col_p + 32 * half + 16 * g, pk);
       }
+      if (half == 0) {
+        // P of keys 0-63 is in TMEM: the first half of PV can run while
+        // the second half of P is computed
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_half[X]);
+      }
     }
     if (!alive) {
       tmem_wait_st();
@@ -443,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 2);  // the QK commit + the MMA thread's tile-info arrive
       mbar_init(&bars.p_full[i], 4);
+      mbar_init(&bars.p_half[i], 4);
       mbar_init(&bars.s_free[i], 4);
       mbar_init(&bars.o_done[i], 1);
     }
@@ -534,14 +544,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bars.s_full[X]);
       };
       auto issue_pv = [&](int X, int s) -> bool {
-        if (!mbar_wait(&bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
-        tc_fence_after();
         const uint64_t dv = dv0 + s * kTileStep;
         const uint32_t o_tmem = tbase + 256u * X + 128u, p_tmem = tbase + 256u * X;
         const uint32_t acc0 = acc[X] ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        for (int hf = 0; hf < 2; ++hf) {
+          // keys 64 hf .. 64 hf + 63 once their P is written
+          if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+            umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        }
         acc[X] = true;
         ++pcnt[X];
         return true;
@@ -553,14 +567,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile's PV (p_full), so the next S is ready when the softmax needs it.
         int freed[2] = {0, 0};  // S tiles of each group read out so far
         auto issue_pv_sep = [&](int X, int s) -> bool {
-          if (!mbar_wait(&bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
-          tc_fence_after();
           const uint64_t dv = dv0 + s * kTileStep;
           const uint32_t o_tmem = tbase + 256u * X + 192u, p_tmem = tbase + 256u * X + 128u;
           const uint32_t acc0 = acc[X] ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          for (int hf = 0; hf < 2; ++hf) {
+            if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+              umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          }
           umma_commit(&bars.o_done[X]);
           acc[X] = true;
           ++pcnt[X];
