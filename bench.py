@@ -42,16 +42,16 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel, from the ncu captures summarised under profiles/, keyed by workload;
 # valid only while that kernel's sources hash to the recorded value.
 #  - causal_softcap_alibi: fwd_sm100_kernel, full workload, one launch
-#    (50.407680 MB read + 1.167872 MB written).
-#  - gqa_sliding_window: fwd_sm100_kernel captured at batch 1 (201.633536 MB
-#    read + 100.084992 MB written), doubled for the batch of 2: both
+#    (50.414848 MB read + 0.630272 MB written).
+#  - gqa_sliding_window: fwd_sm100_kernel captured at batch 1 (201.801472 MB
+#    read + 100.076544 MB written), doubled for the batch of 2: both
 #    sequences carry the same work.
 #  - decode_kv_cache: decode_kernel captured at batch 16 (1220.765 MB read +
 #    12.79872 MB written over 296926 cached tokens), scaled to the full batch
 #    of 32 by cached tokens (614602): traffic grows with the tokens streamed.
 NCU_TRAFFIC = {
-    "causal_softcap_alibi": {"bytes": 51575552, "source_hash": "50727d24277efc09"},
-    "gqa_sliding_window": {"bytes": 603437056, "source_hash": "50727d24277efc09"},
+    "causal_softcap_alibi": {"bytes": 51045120, "source_hash": "3679227a0d1e62a5"},
+    "gqa_sliding_window": {"bytes": 603756032, "source_hash": "3679227a0d1e62a5"},
     "decode_kv_cache": {"bytes": 2553332243, "source_hash": "81c7383f35914920"},
 }
 
