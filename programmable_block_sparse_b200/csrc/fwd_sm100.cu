@@ -35,6 +35,9 @@
 // own: QK_X(next) is issued as soon as the group has read S (s_free), ahead
 // of PV_X(u), and the group waits for that PV (o_done) only before it writes
 // P or rescales O.
+// PV runs in two halves: the group signals p_half once P of keys 0-63 is in
+// TMEM and p_full once all of P is, so the first four PV MMAs overlap the
+// second half of the softmax.
 // The running max only moves (and O rescales) when it grows by more than 2^8;
 // P then stays below 2^8 and the final O / l ratio is exact.
 //
