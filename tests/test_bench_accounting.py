@@ -36,3 +36,18 @@ def test_full_size_counts_match_closed_forms():
     assert bench.visible_pairs_per_head(c) == 4 * 2048 * 2049 // 2
     c = wl.config("gqa_sliding_window")
     assert bench.visible_pairs_per_head(c) == 2 * 16314874
+
+
+def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """Recorded ncu counters stay valid across comment edits, not code edits."""
+    import bench
+    csrc = tmp_path / "programmable_block_sparse_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in ("fwd_sm100.cu", "mods.cuh", "common.cuh"):
+        (csrc / name).write_text("int f(int x) {\n  return x + 1;  // add one\n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash("prefill")
+    (csrc / "fwd_sm100.cu").write_text("/* a new\n   block comment */\nint f(int x) {\n\n  return x + 1;\n}\n")
+    assert bench.kernel_source_hash("prefill") == h0
+    (csrc / "fwd_sm100.cu").write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.kernel_source_hash("prefill") != h0
