@@ -23,6 +23,11 @@
  *   - Every call returns an int status: FA_OK (0) or one of FA_ERR_*.  No call
  *     throws or aborts.  flexattn_last_error() gives a message for the last
  *     failing call on the calling thread.
+ *   - flexattn_build_block_mask, flexattn_forward and
+ *     flexattn_forward_decode_noalloc only enqueue kernels, so a stream
+ *     capture of them (CUDA graphs, relaxed capture mode) replays the same
+ *     work; flexattn_poll_device_status synchronises and must stay outside a
+ *     capture.
  *   - Integers on the device are int32; the host-side struct sizes are int32.
  */
 #ifndef FLEXATTN_H_
