@@ -407,12 +407,43 @@ def check_workload_tile_counts(o):
     assert int(bm["full_kv_num_blocks"].sum()) == full and int(bm["kv_num_blocks"].sum()) == part
 
 
+def check_sampled_rows_match_forward(o):
+    """Rows from forward_sampled equal the same rows of forward.
+
+    forward_sampled is the checker of every full-size comparison, so it is held
+    to forward on a case where a slip in its own bookkeeping would show: GQA
+    with three query heads per KV head, a different valid KV length per
+    sequence (so the logical query positions differ per batch), a document
+    mask, the cap-then-in-document-bias score rule (which reads the query
+    head), and sampled rows at every tile edge of a 4-row tiling plus rows
+    that see no key.
+    """
+    B, Hq, Hkv, L, S, E = 3, 6, 2, 12, 16, 4
+    r = np.random.default_rng(77)
+    q = r.standard_normal((B, Hq, L, E))
+    k = r.standard_normal((B, Hkv, S, E))
+    v = r.standard_normal((B, Hkv, S, 3))
+    kv_len = np.array([16, 13, 9])
+    doc = np.array([[0] * 5 + [1] * 4 + [2] * 7, [0] * 3 + [1] * 8 + [2] * 5, [0] * 9 + [1] * 7])
+    mask = {"kind": "document", "doc_id": doc}
+    score = {"kind": "cap_then_bias", "cap": 3.0, "slope_heads": 0, "pos": "in_doc", "doc_id": doc}
+    out, lse = o.forward(q, k, v, 0.45, mask, score, kv_len=kv_len, enable_gqa=True)
+    rows = sorted({0, 1, 3, 4, 7, 8, 11} | set(range(0, L, 5)))
+    samples = [(b, h, i) for b in range(B) for h in range(Hq) for i in rows]
+    so, sl = o.forward_sampled(q, k, v, samples, 0.45, mask, score, kv_len=kv_len, enable_gqa=True)
+    ref_o = np.stack([out[b, h, i] for b, h, i in samples])
+    ref_l = np.array([lse[b, h, i] for b, h, i in samples])
+    assert np.array_equal(np.isfinite(sl), np.isfinite(ref_l)) and (~np.isfinite(ref_l)).any()
+    fin = np.isfinite(ref_l)
+    assert np.allclose(so, ref_o, atol=1e-13, rtol=0) and np.allclose(sl[fin], ref_l[fin], atol=1e-13, rtol=0)
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
     check_causal_block_fraction, check_window_count, check_single_visible_key, check_equal_scores,
     check_alibi_geometric, check_softcap_limits, check_cap_then_bias_order, check_convex_combination,
     check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
-    check_split_combine, check_gqa_is_broadcast,
+    check_split_combine, check_gqa_is_broadcast, check_sampled_rows_match_forward,
 ]
 SLOW_CHECKS = [check_workload_tile_counts]

@@ -42,6 +42,9 @@ MUTATIONS = {
     "partial_as_full": ("if cell.all():", "if cell.any():"),
     "ragged_cells_counted_hidden": ("cell = vis[:, c0:c1]", "cell = np.pad(vis[:, c0:c1], ((0, 0), (0, BN - (c1 - c0))))"),
     "indices_descending": ("full_idx[b, h, mt, nf] = nt", "full_idx[b, h, mt, Nb - 1 - nf] = nt"),
+    "sampled_head_map": ("kk = _as_f64(k[b, h // G])", "kk = _as_f64(k[b, h % Hkv])"),
+    "sampled_positions_ignore_kv_len": ("qp = query_positions(L, S_b)[r:r + 1]", "qp = query_positions(L, S)[r:r + 1]"),
+    "sampled_row_shifted": ("qrow = _as_f64(q[b, h, r:r + 1])", "qrow = _as_f64(q[b, h, max(r - 1, 0):max(r - 1, 0) + 1])"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
                            "out[live] = outs[:, live].mean(axis=0)"),
 }
