@@ -213,13 +213,19 @@ def _as_f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def attention_rows(q_rows, k, v, scale, mask, score, b, h, qp, S_b, Hq):
+def attention_rows(q_rows, k, v, scale, mask, score, b, h, qp, S_b, Hq, with_max=False):
     """Output rows and lse for one (b, h) and a set of query positions.
 
     The definition in "flexattention-score-mod-block-mask", "What one
     connection goes through": s_ij = scale q_i . k_j; s~_ij = g(s_ij, ...) where
     M_ij, -inf elsewhere; o_i = sum_j softmax_j(s~_ij) v_j.  The score rule is
     applied first and the mask second (section "score_mod changes the score").
+
+    With ``with_max`` the row maximum of s~ is returned third: the per-row
+    maximum score that "PyTorch Flex Attention complete guide" section 2
+    (AuxRequest / AuxOutput) offers beside lse, read here as the largest
+    transformed score among the visible keys (natural units, the quantity
+    whose log-sum-exp is lse) and -inf for a row with no visible key.
     """
     S = k.shape[0]
     kv = np.arange(S, dtype=np.int64)
@@ -238,15 +244,19 @@ def attention_rows(q_rows, k, v, scale, mask, score, b, h, qp, S_b, Hq):
         l = p.sum(axis=1)
         out[live] = (p @ v) / l[:, None]
         lse[live] = m[live] + np.log(l)
+    if with_max:
+        return out, lse, st.max(axis=1)
     return out, lse
 
 
-def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, row_group=512):
+def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, row_group=512, aux=False):
     """fp64 FlexAttention forward: returns (out (B,Hq,L,Ev), lse (B,Hq,L)).
 
     q (B,Hq,L,E), k (B,Hkv,S,E), v (B,Hkv,S,Ev); numpy arrays or torch
     tensors (upcast exactly).  ``scale`` defaults to 1/sqrt(E) (guide section
     6.2).  GQA broadcasts KV head h // (Hq // Hkv) (guide section 6.1).
+    With ``aux`` a third array, max_scores (B,Hq,L), is returned (see
+    :func:`attention_rows`).
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     B, Hq, L, E = q.shape
@@ -259,6 +269,7 @@ def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=
     scale = 1.0 / math.sqrt(E) if scale is None else float(scale)
     out = np.zeros((B, Hq, L, v.shape[3]))
     lse = np.full((B, Hq, L), NEG_INF)
+    mxs = np.full((B, Hq, L), NEG_INF)
     for b in range(B):
         S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
         qp_all = query_positions(L, S_b)
@@ -269,18 +280,20 @@ def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=
                 mk = dict(mask)
                 if mask["kind"] == "dense":
                     mk["rows"] = np.arange(r0, r1)
-                o, ls = attention_rows(q[b, h, r0:r1], k[b, hk], v[b, hk], scale, mk, score, b, h,
-                                       qp_all[r0:r1], S_b, Hq)
+                o, ls, mx = attention_rows(q[b, h, r0:r1], k[b, hk], v[b, hk], scale, mk, score, b, h,
+                                           qp_all[r0:r1], S_b, Hq, with_max=True)
                 out[b, h, r0:r1] = o
                 lse[b, h, r0:r1] = ls
-    return out, lse
+                mxs[b, h, r0:r1] = mx
+    return (out, lse, mxs) if aux else (out, lse)
 
 
-def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False):
+def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, aux=False):
     """Output and lse for sampled (b, h, row) triples; returns (out[n,Ev], lse[n]).
 
     Used on workloads too large for :func:`forward`: each sampled row is
-    computed in full by :func:`attention_rows`.
+    computed in full by :func:`attention_rows`.  With ``aux`` the rows'
+    max_scores come third.
     """
     Bq, Hq, L, E = q.shape
     Hkv, S = k.shape[1], k.shape[2]
@@ -288,16 +301,19 @@ def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=
     mask = mask or {"kind": "none"}
     score = score or {"kind": "none"}
     scale = 1.0 / math.sqrt(E) if scale is None else float(scale)
-    outs, lses = [], []
+    outs, lses, mxs = [], [], []
     for (b, h, r) in samples:
         S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
         qp = query_positions(L, S_b)[r:r + 1]
         qrow = _as_f64(q[b, h, r:r + 1])
         kk = _as_f64(k[b, h // G])
         vv = _as_f64(v[b, h // G])
-        o, ls = attention_rows(qrow, kk, vv, scale, mask, score, b, h, qp, S_b, Hq)
+        o, ls, mx = attention_rows(qrow, kk, vv, scale, mask, score, b, h, qp, S_b, Hq, with_max=True)
         outs.append(o[0])
         lses.append(ls[0])
+        mxs.append(mx[0])
+    if aux:
+        return np.stack(outs), np.array(lses), np.array(mxs)
     return np.stack(outs), np.array(lses)
 
 

@@ -67,22 +67,23 @@ def _g(kind, params, s, b, h, q, kv, Hq):
     raise ValueError(kind)
 
 
-def forward_scalar(q, k, v, scale, mask, score, kv_len=None):
+def forward_scalar(q, k, v, scale, mask, score, kv_len=None, with_max=False):
     """q[B][Hq][L][E], k[B][Hkv][S][E], v[B][Hkv][S][Ev] as nested lists of floats.
 
     Returns (out[B][Hq][L][Ev], lse[B][Hq][L]); a row with no visible key gives
-    zeros and -inf.
+    zeros and -inf.  With ``with_max`` a third nested list holds each row's
+    largest visible transformed score (-inf for a row with none).
     """
     B, Hq, L = len(q), len(q[0]), len(q[0][0])
     Hkv, S = len(k[0]), len(k[0][0])
     G = Hq // Hkv
-    out, lse = [], []
+    out, lse, top = [], [], []
     for b in range(B):
         S_b = S if kv_len is None else int(kv_len[b])
-        ob, lb = [], []
+        ob, lb, tb = [], [], []
         for h in range(Hq):
             hk = h // G
-            oh, lh = [], []
+            oh, lh, th = [], [], []
             for i in range(L):
                 qpos = i + (S_b - L)
                 scores = []
@@ -92,7 +93,11 @@ def forward_scalar(q, k, v, scale, mask, score, kv_len=None):
                         dot += q[b][h][i][e] * k[b][hk][j][e]
                     g = _g(score["kind"], score, scale * dot, b, h, qpos, j, Hq)
                     scores.append(g if _visible(mask["kind"], mask, b, qpos, j, S_b) else -math.inf)
-                m = max(scores)
+                m = -math.inf
+                for x in scores:
+                    if x > m:
+                        m = x
+                th.append(m)
                 Ev = len(v[b][hk][0])
                 if m == -math.inf:
                     oh.append([0.0] * Ev)
@@ -104,9 +109,11 @@ def forward_scalar(q, k, v, scale, mask, score, kv_len=None):
                 lh.append(m + math.log(tot))
             ob.append(oh)
             lb.append(lh)
+            tb.append(th)
         out.append(ob)
         lse.append(lb)
-    return out, lse
+        top.append(tb)
+    return (out, lse, top) if with_max else (out, lse)
 
 
 def tile_classes_scalar(mask, L, S, BM, BN, b=0, kv_len=None):

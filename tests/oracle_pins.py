@@ -438,6 +438,64 @@ def check_sampled_rows_match_forward(o):
     assert np.allclose(so, ref_o, atol=1e-13, rtol=0) and np.allclose(sl[fin], ref_l[fin], atol=1e-13, rtol=0)
 
 
+def check_max_scores(o):
+    """max_scores: the largest visible transformed score of each row.
+
+    Pinned by closed forms (a row with one visible key: max = lse = that
+    key's g; q = 0 under ALiBi: max = 0, reached at the query's own key; a
+    row with no visible key: -inf), by the bound max <= lse <= max + ln n
+    with n the row's visible-key count, by a case whose largest raw score
+    sits on a hidden key, and by the pure-Python loops on tiny shapes.
+    """
+    sr = _scalar()
+    B, H, L, E = 1, 3, 9, 5
+    r = np.random.default_rng(31)
+    q = r.standard_normal((B, H, L, E))
+    k = r.standard_normal((B, H, L, E))
+    v = r.standard_normal((B, H, L, E))
+    score = {"kind": "cap_then_bias", "cap": 7.0, "slope_heads": 3, "pos": "global"}
+    out, lse, mx = o.forward(q, k, v, 0.3, {"kind": "causal"}, score, aux=True)
+    for h in range(H):
+        s = 0.3 * float(q[0, h, 0] @ k[0, h, 0])
+        assert abs(mx[0, h, 0] - 7.0 * math.tanh(s / 7.0)) < 1e-12 and mx[0, h, 0] == lse[0, h, 0]
+    # q = 0 under ALiBi: g = -slope (q - kv) <= 0, equal to 0 at kv = q
+    z = np.zeros_like(q)
+    _, _, mz = o.forward(z, k, v, 1.0, {"kind": "causal"}, {"kind": "alibi"}, aux=True)
+    assert np.all(mz == 0.0)
+    # the largest raw score on a hidden key must not leak into the max
+    k2 = k.copy()
+    k2[0, :, L - 1] = 50.0 * q[0, :, 0]            # key L-1 scores highest for query 0
+    _, _, m2 = o.forward(q, k2, v, 1.0, {"kind": "causal"}, None, aux=True)
+    assert np.allclose(m2[0, :, 0], np.einsum("he,he->h", q[0, :, 0], k2[0, :, 0]), atol=1e-12)
+    # no visible key: -inf; otherwise max <= lse <= max + ln n
+    kv_len = np.array([4])
+    o2, l2, m3 = o.forward(q, k, v, 0.5, {"kind": "causal"}, {"kind": "softcap", "cap": 2.0}, kv_len=kv_len,
+                           aux=True)
+    vis = o.visible({"kind": "causal"}, 0, 0, o.query_positions(L, 4), np.arange(L), 4)
+    n = vis.sum(axis=1)
+    assert np.all(m3[0, :, n == 0] == -np.inf) and np.all(l2[0, :, n == 0] == -np.inf)
+    live = n > 0
+    assert np.all(m3[0][:, live] <= l2[0][:, live] + 1e-12)
+    assert np.all(l2[0][:, live] <= m3[0][:, live] + np.log(n[live]) + 1e-12)
+    # brute force on tiny shapes, every mask and score kind
+    seed = 500
+    for mask in TINY_MASKS:
+        for sc in TINY_SCORES:
+            seed += 1
+            q, k, v = _tiny_case(seed, 3, 8, 3, 2)
+            _, _, m = o.forward(q, k, v, 0.7, mask, sc, kv_len=[8, 5], enable_gqa=True, aux=True)
+            _, _, sm = sr.forward_scalar(q.tolist(), k.tolist(), v.tolist(), 0.7, mask, sc, [8, 5], with_max=True)
+            sm = np.array(sm)
+            fin = np.isfinite(sm)
+            assert np.array_equal(fin, np.isfinite(m)) and np.allclose(m[fin], sm[fin], atol=1e-12, rtol=0)
+    # the sampled-row checker returns the same maxima
+    samples = [(0, 1, 0), (1, 0, 2)]
+    _, _, ms = o.forward_sampled(q, k, v, samples, 0.7, TINY_MASKS[1], TINY_SCORES[1], kv_len=[8, 5],
+                                 enable_gqa=True, aux=True)
+    _, _, mf = o.forward(q, k, v, 0.7, TINY_MASKS[1], TINY_SCORES[1], kv_len=[8, 5], enable_gqa=True, aux=True)
+    assert np.array_equal(ms, np.array([mf[b, h, i] for b, h, i in samples]))
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
@@ -445,5 +503,6 @@ ALL_CHECKS = [
     check_alibi_geometric, check_softcap_limits, check_cap_then_bias_order, check_convex_combination,
     check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
     check_split_combine, check_gqa_is_broadcast, check_sampled_rows_match_forward,
+    check_max_scores,
 ]
 SLOW_CHECKS = [check_workload_tile_counts]

@@ -45,6 +45,9 @@ MUTATIONS = {
     "sampled_head_map": ("kk = _as_f64(k[b, h // G])", "kk = _as_f64(k[b, h % Hkv])"),
     "sampled_positions_ignore_kv_len": ("qp = query_positions(L, S_b)[r:r + 1]", "qp = query_positions(L, S)[r:r + 1]"),
     "sampled_row_shifted": ("qrow = _as_f64(q[b, h, r:r + 1])", "qrow = _as_f64(q[b, h, max(r - 1, 0):max(r - 1, 0) + 1])"),
+    "max_scores_unmasked": ("return out, lse, st.max(axis=1)", "return out, lse, g.max(axis=1)"),
+    "max_scores_log2_units": ("return out, lse, st.max(axis=1)", "return out, lse, st.max(axis=1) * 1.4426950408889634"),
+    "max_scores_raw_score": ("return out, lse, st.max(axis=1)", "return out, lse, np.where(vis, s, NEG_INF).max(axis=1)"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
                            "out[live] = outs[:, live].mean(axis=0)"),
 }
