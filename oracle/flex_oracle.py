@@ -272,20 +272,37 @@ def forward(q, k, v, scale=None, mask=None, score=None, kv_len=None, enable_gqa=
     mxs = np.full((B, Hq, L), NEG_INF)
     for b in range(B):
         S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
-        qp_all = query_positions(L, S_b)
         for h in range(Hq):
             hk = h // G
-            for r0 in range(0, L, row_group):
-                r1 = min(L, r0 + row_group)
-                mk = dict(mask)
-                if mask["kind"] == "dense":
-                    mk["rows"] = np.arange(r0, r1)
-                o, ls, mx = attention_rows(q[b, h, r0:r1], k[b, hk], v[b, hk], scale, mk, score, b, h,
-                                           qp_all[r0:r1], S_b, Hq, with_max=True)
-                out[b, h, r0:r1] = o
-                lse[b, h, r0:r1] = ls
-                mxs[b, h, r0:r1] = mx
+            out[b, h], lse[b, h], mxs[b, h] = forward_unit(q[b, h], k[b, hk], v[b, hk], b, h, Hq, S_b, scale,
+                                                           mask, score, row_group)
     return (out, lse, mxs) if aux else (out, lse)
+
+
+def forward_unit(q_bh, k_bh, v_bh, b, h, Hq, S_b, scale, mask, score, row_group=512):
+    """Every query row of one (batch b, query head h) unit: (out (L,Ev), lse (L,), max_scores (L,)).
+
+    q_bh (L,E) are the unit's queries; k_bh (S,E), v_bh (S,Ev) its KV head's
+    keys and values; S_b the valid KV length of sequence b; Hq the number of
+    query heads (the slope of the distance rules reads h and Hq).  This is
+    the body of :func:`forward` for one (b, h), exposed so that large
+    workloads can be checked unit by unit.  Rows are evaluated in groups of
+    ``row_group`` only to bound memory.
+    """
+    q_bh, k_bh, v_bh = _as_f64(q_bh), _as_f64(k_bh), _as_f64(v_bh)
+    L = q_bh.shape[0]
+    qp_all = query_positions(L, S_b)
+    out = np.zeros((L, v_bh.shape[1]))
+    lse = np.full(L, NEG_INF)
+    mxs = np.full(L, NEG_INF)
+    for r0 in range(0, L, row_group):
+        r1 = min(L, r0 + row_group)
+        mk = dict(mask)
+        if mask["kind"] == "dense":
+            mk["rows"] = np.arange(r0, r1)
+        out[r0:r1], lse[r0:r1], mxs[r0:r1] = attention_rows(q_bh[r0:r1], k_bh, v_bh, scale, mk, score, b, h,
+                                                            qp_all[r0:r1], S_b, Hq, with_max=True)
+    return out, lse, mxs
 
 
 def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, aux=False):

@@ -496,6 +496,36 @@ def check_max_scores(o):
     assert np.array_equal(ms, np.array([mf[b, h, i] for b, h, i in samples]))
 
 
+def check_forward_unit_matches_forward(o):
+    """forward_unit on one (b, h) slice gives forward's rows of that unit.
+
+    The full-size checks call forward_unit with slices regenerated per unit,
+    so its arguments (batch b for the document row, query head h and Hq for
+    the slope, the valid length S_b for positions) are held to forward on GQA
+    with per-sequence valid lengths, a per-batch document mask and the
+    in-document cap-then-bias rule.
+    """
+    B, Hq, Hkv, L, S, E = 2, 4, 2, 10, 14, 3
+    r = np.random.default_rng(91)
+    q = r.standard_normal((B, Hq, L, E))
+    k = r.standard_normal((B, Hkv, S, E))
+    v = r.standard_normal((B, Hkv, S, 2))
+    kv_len = np.array([14, 11])
+    doc = np.array([[0] * 6 + [1] * 8, [0] * 2 + [1] * 9 + [2] * 3])
+    mask = {"kind": "document", "doc_id": doc}
+    score = {"kind": "cap_then_bias", "cap": 2.5, "slope_heads": 0, "pos": "in_doc", "doc_id": doc}
+    out, lse, mx = o.forward(q, k, v, 0.6, mask, score, kv_len=kv_len, enable_gqa=True, aux=True)
+    for b in range(B):
+        for h in range(Hq):
+            uo, ul, um = o.forward_unit(q[b, h], k[b, h // 2], v[b, h // 2], b, h, Hq, int(kv_len[b]), 0.6, mask,
+                                        score, row_group=3)
+            assert np.allclose(uo, out[b, h], atol=1e-14, rtol=0)
+            assert np.array_equal(np.isfinite(ul), np.isfinite(lse[b, h]))
+            fin = np.isfinite(ul)
+            assert np.allclose(ul[fin], lse[b, h][fin], atol=1e-14)
+            assert np.array_equal(np.isfinite(um), fin) and np.allclose(um[fin], mx[b, h][fin], atol=1e-14)
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
@@ -503,6 +533,6 @@ ALL_CHECKS = [
     check_alibi_geometric, check_softcap_limits, check_cap_then_bias_order, check_convex_combination,
     check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
     check_split_combine, check_gqa_is_broadcast, check_sampled_rows_match_forward,
-    check_max_scores,
+    check_max_scores, check_forward_unit_matches_forward,
 ]
 SLOW_CHECKS = [check_workload_tile_counts]
