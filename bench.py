@@ -2,16 +2,25 @@
 
 A step is one pass of the whole path over one batch of synthetic input: the
 BlockMask build (tile classifier) and the forward pass over the listed tiles.
-The default workload is the causal + soft-cap(50) + ALiBi prefill
-(B=4, H=16, L=S=2048, E=64, bf16, 128 x 128 tiles).
+By default every workload runs in turn, each with its own warm-up and timed
+steps; the JSON line's headline fields belong to the largest single-GPU
+prefill workload (GQA sliding window: B=2, Hq=32, Hkv=8, L=S=16384, E=128,
+bf16), and every workload's own numbers are under ``detail.per_config``:
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    gqa_sliding_window     headline; tensor roofline
+    causal_softcap_alibi   B=4, H=16, L=S=2048, E=64; tensor roofline
+    packed_docs            H=16, L=S=8192, E=128; tensor roofline
+    decode_kv_cache        B=32, Hq=32, Hkv=8, q_len 4, caches of 4096-32768; HBM roofline
+    decode_kv_cache_q1     the same with q_len 1
+    fp32_causal_small      fp32, L=S=128, 32 x 32 tiles (a correctness workload, no roofline target)
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload LABEL|all] [--impl reference]
 
 With N > 1 it runs under torchrun, one process per GPU; every rank processes
-the same per-GPU workload (weak scaling: the (batch, head) units shard with no
-data-path exchange), times on the device, and rank 0 reports the max over ranks.
-``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
-workload instead (rank 0 only).
+the same per-GPU workloads (weak scaling: the (batch, head) units shard with
+no data-path exchange), times on the device, and rank 0 reports the max over
+ranks.  ``--impl reference`` times the fp64 CPU oracle on bounded samples of
+the headline workload instead (rank 0 only).
 """
 
 from __future__ import annotations
@@ -19,9 +28,9 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import re
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -35,30 +44,33 @@ sys.path.insert(0, ROOT)
 
 import workloads as wl  # noqa: E402
 
-METRIC_PREFILL = "visible-score TFLOP/s & % BF16 tensor peak (prefill); KV GB/s % HBM (decode)"
+METRIC = "visible-score TFLOP/s & % BF16 tensor peak (prefill); KV GB/s % HBM (decode)"
+METRIC_PREFILL = METRIC
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
+# (label, workload, overrides): the bench items, headline first.
+BENCH_ITEMS = [
+    ("gqa_sliding_window", "gqa_sliding_window", {}),
+    ("causal_softcap_alibi", "causal_softcap_alibi", {}),
+    ("packed_docs", "packed_docs", {}),
+    ("decode_kv_cache", "decode_kv_cache", {}),
+    ("decode_kv_cache_q1", "decode_kv_cache", {"L": 1}),
+    ("fp32_causal_small", "fp32_causal_small", {}),
+]
+HEADLINE = BENCH_ITEMS[0][0]
+
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
-# kernel, from the ncu captures summarised under profiles/, keyed by workload;
-# valid only while that kernel's sources hash to the recorded value.
-#  - causal_softcap_alibi: fwd_sm100_kernel, full workload, one launch
-#    (50.414848 MB read + 0.630272 MB written).
-#  - gqa_sliding_window: fwd_sm100_kernel captured at batch 1 (201.801472 MB
-#    read + 100.076544 MB written), doubled for the batch of 2: both
-#    sequences carry the same work.
-#  - decode_kv_cache: decode_kernel captured at batch 16 (1220.765 MB read +
-#    12.79872 MB written over 296926 cached tokens), scaled to the full batch
-#    of 32 by cached tokens (614602): traffic grows with the tokens streamed.
-NCU_TRAFFIC = {
-    "causal_softcap_alibi": {"bytes": 51045120, "source_hash": "3a07580eec5ff9d8"},
-    "gqa_sliding_window": {"bytes": 603756032, "source_hash": "3a07580eec5ff9d8"},
-    "decode_kv_cache": {"bytes": 2553332243, "source_hash": "da0da3a8d76e9df9"},
-}
+# kernel, from the ncu captures summarised under profiles/, keyed by bench
+# label; valid only while that kernel's sources hash to the recorded value
+# (the hash ignores comments).  The scaling of each capture to the full
+# workload is stated in the profile it comes from.
+NCU_TRAFFIC = {}
 
 KERNEL_SOURCES = {
     "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh"),
     "decode": ("decode.cu", "mods.cuh", "common.cuh"),
+    "general": ("fwd_simt.cu", "mods.cuh", "common.cuh"),
 }
 
 
@@ -84,33 +96,42 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def item(label):
+    for it in BENCH_ITEMS:
+        if it[0] == label:
+            return it
+    raise KeyError(label)
+
+
 # ---------------------------------------------------------------------------
 # Work accounting (exact counts from the workload parameters)
 # ---------------------------------------------------------------------------
 
-def visible_pairs_per_head(c, kv_len=None, doc_lengths=None):
-    """Visible (query, key) pairs for one (b, h), summed over the batch."""
+def visible_counts_rows(c, b, kv_len=None, doc_lengths=None):
+    """Visible keys of every query row of batch b (int64 array of length L)."""
     L, S = c["L"], c["S"]
     kind = c["mask"]["kind"]
-    total = 0
-    for b in range(c["B"]):
-        S_b = S if kv_len is None else int(kv_len[b])
-        q = np.arange(L, dtype=np.int64) + (S_b - L)
-        if kind == "causal":
-            n = np.clip(np.minimum(q + 1, S_b), 0, None)
-        elif kind == "sliding_window":
-            W, ns = c["mask"]["window"], c["mask"].get("n_sink", 0)
-            lo = np.maximum(q - W + 1, 0)
-            win = np.clip(np.minimum(q, S_b - 1) - lo + 1, 0, None)
-            sink = np.clip(np.minimum(np.minimum(ns - 1, q), lo - 1) + 1, 0, None)
-            n = win + sink
-        elif kind == "document":
-            starts = np.repeat(np.concatenate([[0], np.cumsum(doc_lengths)[:-1]]), doc_lengths)
-            n = q - starts[q] + 1
-        else:
-            raise ValueError(kind)
-        total += int(n.sum())
-    return total
+    S_b = S if kv_len is None else int(kv_len[b])
+    q = np.arange(L, dtype=np.int64) + (S_b - L)
+    if kind == "causal":
+        n = np.clip(np.minimum(q + 1, S_b), 0, None)
+    elif kind == "sliding_window":
+        W, ns = c["mask"]["window"], c["mask"].get("n_sink", 0)
+        lo = np.maximum(q - W + 1, 0)
+        win = np.clip(np.minimum(q, S_b - 1) - lo + 1, 0, None)
+        sink = np.clip(np.minimum(np.minimum(ns - 1, q), lo - 1) + 1, 0, None)
+        n = win + sink
+    elif kind == "document":
+        starts = np.repeat(np.concatenate([[0], np.cumsum(doc_lengths)[:-1]]), doc_lengths)
+        n = q - starts[q] + 1
+    else:
+        raise ValueError(kind)
+    return n
+
+
+def visible_pairs_per_head(c, kv_len=None, doc_lengths=None):
+    """Visible (query, key) pairs for one (b, h), summed over the batch."""
+    return int(sum(int(visible_counts_rows(c, b, kv_len, doc_lengths).sum()) for b in range(c["B"])))
 
 
 def visited_cells(bm):
@@ -200,9 +221,9 @@ def describe(name, c):
     return f"{name}", d
 
 
-def make_inputs(name, device, seed_offset=0, batch=None):
+def make_inputs(name, device, seed_offset=0, batch=None, **over):
     import torch
-    c = wl.config(name)
+    c = wl.config(name, **over)
     if batch:
         c["B"] = int(batch)
     kv_len = doc_lengths = None
@@ -231,93 +252,121 @@ def make_inputs(name, device, seed_offset=0, batch=None):
 # CPU oracle timing (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_rate(name, target_s=12.0, max_heads=None):
-    """Run the fp64 oracle on whole (b, h) units until ~target_s of oracle time.
+class OracleSampler:
+    """Bounded samples of a workload evaluated by the fp64 oracle.
 
-    Inputs are the workload's own seeded slices (regenerated per unit, outside
-    the timing).  Returns (rate, seconds, cores, sample description, units
-    done, unit): visible-pair FLOP/s (prefill) or KV bytes/s (decode: each
-    query head's share of its KV head's valid cache).
+    A sample is a block of query rows of one (batch, query head) unit -- all
+    L rows for decode, else about 2^21 / S rows -- computed in full by the
+    oracle's row function from slices regenerated for that unit (outside the
+    timing).  Work per block: visible-pair FLOPs (2E + 2Ev per pair) for
+    prefill, or the unit's share of its KV head's valid cache bytes for decode.
     """
-    import torch
 
-    import oracle.flex_oracle as o
-    c = wl.config(name)
-    kv_len = doc_lengths = None
-    if name == "decode_kv_cache":
-        kv_len = wl.decode_cache_lengths(c["B"], c["kv_lo"], c["kv_hi"], c["seed"])
-    if name == "packed_docs":
-        doc_lengths = wl.doc_lengths(c["doc_total"], c["doc_lo"], c["doc_hi"], c["seed"])
-    mask = dict(c["mask"])
-    score = dict(c["score"])
-    if doc_lengths is not None:
-        ids = wl.doc_ids_from_lengths(doc_lengths)
-        mask["doc_id"] = ids
-        score["doc_id"] = ids
-    dt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float32
-    G = c["Hq"] // c["Hkv"]
-    flop_pair = 2 * c["E"] + 2 * c["Ev"]
-    per_head_pairs = visible_pairs_per_head(c, kv_len, doc_lengths) / c["B"]
-    decode = name == "decode_kv_cache"
-    el = 0.0
-    heads = 0
-    work = 0.0
-    b = h = 0
-    while True:
-        qs = wl.randn_slice(c["seed"], 0, b, h, c["L"], c["E"], dt)[None, None]
-        ks = wl.randn_slice(c["seed"], 1, b, h // G, c["S"], c["E"], dt)[None, None]
-        vs = wl.randn_slice(c["seed"], 2, b, h // G, c["S"], c["Ev"], dt)[None, None]
-        sub_kv = None
-        if kv_len is not None:
-            sub_kv = kv_len[b:b + 1]
-            wl.fill_cache_tail(ks, vs, sub_kv)
+    def __init__(self, name, **over):
+        import torch
+        self.name = name
+        self.c = c = wl.config(name, **over)
+        self.kv_len = self.doc_lengths = None
+        if name == "decode_kv_cache":
+            self.kv_len = wl.decode_cache_lengths(c["B"], c["kv_lo"], c["kv_hi"], c["seed"])
+        if name == "packed_docs":
+            self.doc_lengths = wl.doc_lengths(c["doc_total"], c["doc_lo"], c["doc_hi"], c["seed"])
+        self.mask, self.score = dict(c["mask"]), dict(c["score"])
+        if self.doc_lengths is not None:
+            ids = wl.doc_ids_from_lengths(self.doc_lengths)
+            self.mask["doc_id"] = ids
+            self.score["doc_id"] = ids
+        self.dt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float32
+        self.decode = name == "decode_kv_cache"
+        self.rows = c["L"] if self.decode else max(1, min(c["L"], (1 << 21) // c["S"]))
+        self.blocks_per_unit = -(-c["L"] // self.rows)
+        self.units = c["B"] * c["Hq"]
+        self.counts = [visible_counts_rows(c, b, self.kv_len, self.doc_lengths) for b in range(c["B"])]
+        self.unit_desc = ("one (batch, query head) unit, all its query rows" if self.decode else
+                          f"a block of {self.rows} query rows of one (batch, query head) unit, every row in full")
+
+    def block(self, i):
+        """(work, seconds) of the i-th sample; samples are spread over units and rows."""
+        import torch
+
+        import oracle.flex_oracle as o
+        c = self.c
+        total = self.units * self.blocks_per_unit
+        j = (i * 7919) % total
+        unit, blk = divmod(j, self.blocks_per_unit)
+        b, h = divmod(unit, c["Hq"])
+        G = c["Hq"] // c["Hkv"]
+        q = wl.randn_slice(c["seed"], 0, b, h, c["L"], c["E"], self.dt)
+        k = wl.randn_slice(c["seed"], 1, b, h // G, c["S"], c["E"], self.dt)
+        v = wl.randn_slice(c["seed"], 2, b, h // G, c["S"], c["Ev"], self.dt)
+        S_b = c["S"] if self.kv_len is None else int(self.kv_len[b])
+        if self.kv_len is not None:
+            wl.fill_cache_tail(k[None, None], v[None, None], [S_b])
+        r0, r1 = blk * self.rows, min(c["L"], (blk + 1) * self.rows)
+        qn = q[r0:r1].to(torch.float64).numpy()
+        kn = k.to(torch.float64).numpy()
+        vn = v.to(torch.float64).numpy()
+        qp = o.query_positions(c["L"], S_b)[r0:r1]
         t0 = time.perf_counter()
-        o.forward(qs, ks, vs, c["scale"], mask, score, kv_len=sub_kv)
-        el += time.perf_counter() - t0
-        heads += 1
-        if decode:
-            work += int(kv_len[b]) * (c["E"] + c["Ev"]) * 2 / G
+        o.attention_rows(qn, kn, vn, c["scale"], self.mask, self.score, b, h, qp, S_b, c["Hq"])
+        el = time.perf_counter() - t0
+        if self.decode:
+            work = S_b * (c["E"] + c["Ev"]) * 2 / G
         else:
-            work += per_head_pairs * flop_pair
-        h = (h + 1) % c["Hq"]
-        b = (b + (h == 0)) % c["B"]
-        if el >= target_s or (max_heads and heads >= max_heads):
-            break
-    cores = len(os.sched_getaffinity(0))
-    units = c["B"] * c["Hq"]
-    if heads <= units:
-        sample = f"{heads} of the {units} (batch, query head) units, every query row in full"
-    else:
-        sample = (f"{heads} (batch, query head) unit evaluations, cycling over all {units} units "
-                  f"({heads / units:.2f} passes), every query row in full")
-    if decode:
-        return work / el / 1e9, el, cores, sample, heads, "GB/s"
-    return work / el / 1e12, el, cores, sample, heads, "TFLOP/s"
+            work = float(self.counts[b][r0:r1].sum()) * (2 * c["E"] + 2 * c["Ev"])
+        return work, el
+
+    def rate(self, target_s):
+        """(rate, seconds, samples) running samples until ~target_s of oracle time."""
+        work = el = 0.0
+        n = 0
+        while el < target_s or n == 0:
+            w, t = self.block(n)
+            work += w
+            el += t
+            n += 1
+        scale = 1e9 if self.decode else 1e12
+        return work / el / scale, el, n
+
+    @property
+    def unit(self):
+        return "GB/s" if self.decode else "TFLOP/s"
+
+
+def cpu_baseline(label, target_s):
+    _, name, over = item(label)
+    s = OracleSampler(name, **over)
+    rate, el, n = s.rate(target_s)
+    return {"value": rate, "unit": s.unit, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{n} samples of {s.unit_desc}, spread over the workload's units and rows", "seconds": el}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    name = args.workload
-    c = wl.config(name)
-    for _ in range(args.warmup):
-        oracle_sample_rate(name, target_s=0.0, max_heads=1)
-    times, rates = [], []
-    unit, cores = "TFLOP/s", len(os.sched_getaffinity(0))
-    for _ in range(args.steps):
-        rate, el, cores, _, _, unit = oracle_sample_rate(name, target_s=0.0, max_heads=1)
-        times.append(el)
-        rates.append(rate)
-    value = statistics.mean(rates)
-    sample = "one (batch, query head) unit of the workload per step, every query row in full"
+    label = HEADLINE if args.workload == "all" else args.workload
+    _, name, over = item(label)
+    c = wl.config(name, **over)
+    s = OracleSampler(name, **over)
+    for i in range(args.warmup):
+        s.block(i)
+    times, works = [], []
+    for i in range(args.steps):
+        w, t = s.block(args.warmup + i)
+        works.append(w)
+        times.append(t)
+    scale = 1e9 if s.decode else 1e12
+    value = sum(works) / sum(times) / scale
+    cores = len(os.sched_getaffinity(0))
+    sample = f"each step: {s.unit_desc}, spread over the workload's units and rows"
     line = {
-        "impl": "reference", "metric": METRIC_PREFILL, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": s.unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": name, **describe(name, c)[1], "sample": sample},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "data": "synthetic", "config": {"workload": label, **describe(name, c)[1], "sample": sample},
+        "cpu_baseline": {"value": value, "unit": s.unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": s.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
@@ -354,6 +403,212 @@ def whole_job_rate(work_per_rank, world, ms_per_step, scale):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+class Workload:
+    """One bench item on the device: inputs, block mask, outputs, work counts."""
+
+    def __init__(self, label, dev, rank, batch=None):
+        import torch
+        import programmable_block_sparse_b200 as fa
+        self.fa = fa
+        self.label = label
+        _, self.name, over = item(label)
+        (self.c, (self.q_h, self.k_h, self.v_h), self.mask, self.score, self.kv_len,
+         self.doc_lengths) = make_inputs(self.name, dev, seed_offset=rank, batch=batch, **over)
+        c = self.c
+        self.B_mask = c["B"] if self.kv_len is not None else 1
+        self.gqa = c["Hq"] != c["Hkv"]
+        self.q, self.k, self.v = self.q_h.to(dev), self.k_h.to(dev), self.v_h.to(dev)
+        self.out = torch.empty((c["B"], c["Hq"], c["L"], c["Ev"]), dtype=self.q.dtype, device=dev)
+        self.lse = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
+        self.bm = fa.flexattn_build_block_mask(self.mask, self.B_mask, 1, c["L"], c["S"], c["BM"], c["BN"], device=dev)
+        ws = fa.flexattn_forward_workspace_size(self.q, self.k, self.v, self.bm)
+        self.ws_bytes = ws
+        self.ws = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+        self.decode = self.name == "decode_kv_cache"
+        self.general = c["dtype"] != "bf16" or c["BM"] != 128
+        # classifier + forward kernel, + the log-sum-exp combine when decode splits the keys
+        self.launches_per_step = 2 + (1 if self.decode and ws > 0 else 0)
+        fp = 2 * c["E"] + 2 * c["Ev"]
+        self.vis_flops = visible_pairs_per_head(c, self.kv_len, self.doc_lengths) * c["Hq"] * fp
+        cells = visited_cells(self.bm) * (c["Hq"] if self.bm.H == 1 else 1) * (c["B"] if self.bm.B == 1 else 1)
+        self.visited_cells = cells
+        self.visited_flops = cells * fp
+        self.kv_bytes = (int(np.sum(self.kv_len)) * c["Hkv"] * (c["E"] + c["Ev"]) * self.q.element_size()
+                         if self.decode else None)
+
+    def build(self):
+        c = self.c
+        self.fa.flexattn_build_block_mask(self.mask, self.B_mask, 1, c["L"], c["S"], c["BM"], c["BN"], out=self.bm)
+
+    def forward(self):
+        self.fa.flexattn_forward(self.q, self.k, self.v, self.bm, score_mod=self.score, mask_mod=self.mask,
+                                 scale=self.c["scale"], enable_gqa=self.gqa, out=self.out, lse=self.lse,
+                                 workspace=self.ws)
+
+    def step(self):
+        self.build()
+        self.forward()
+
+    def capture_graphs(self):
+        """CUDA graphs of the two calls, used only after a replay into cleared
+        outputs and a sentinel-filled block mask reproduces the eager result
+        (block mask bit for bit, out within 1e-2, lse within 1e-3)."""
+        import torch
+        fa = self.fa
+        try:
+            out_ref, lse_ref = self.out.float().clone(), self.lse.clone()
+            bm_ref = [t.clone() for t in (self.bm.kv_num_blocks, self.bm.kv_indices, self.bm.full_kv_num_blocks,
+                                          self.bm.full_kv_indices)]
+            g_mask, g_fwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_mask, capture_error_mode="relaxed"):
+                self.build()
+            with torch.cuda.graph(g_fwd, capture_error_mode="relaxed"):
+                self.forward()
+            for t in (self.bm.kv_num_blocks, self.bm.kv_indices, self.bm.full_kv_num_blocks,
+                      self.bm.full_kv_indices):
+                t.fill_(-1)
+            self.out.zero_()
+            self.lse.zero_()
+            g_mask.replay()
+            g_fwd.replay()
+            torch.cuda.synchronize()
+            same_mask = all(torch.equal(a, b) for a, b in zip(bm_ref, (self.bm.kv_num_blocks, self.bm.kv_indices,
+                                                                       self.bm.full_kv_num_blocks,
+                                                                       self.bm.full_kv_indices)))
+            fin = torch.isfinite(lse_ref)
+            same = (same_mask and torch.equal(fin, torch.isfinite(self.lse))
+                    and (self.out.float() - out_ref).abs().max().item() <= 1e-2
+                    and (self.lse[fin] - lse_ref[fin]).abs().max().item() <= 1e-3)
+            if same and fa.flexattn_poll_device_status() == 0:
+                return (g_mask, g_fwd), "CUDA graph replay, one graph per call"
+            return None, "eager (graph replay did not reproduce the eager result)"
+        except Exception as exc:  # capture unsupported here: keep the eager launches
+            torch.cuda.synchronize()
+            return None, f"eager (graph capture failed: {type(exc).__name__})"
+
+
+def measure(wk, args, dev, world, flush, peaks, peak_src):
+    """Warm-up, then K device-timed steps; numbers of one workload."""
+    import torch
+    import torch.distributed as dist
+    fa = wk.fa
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        wk.step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    if fa.flexattn_poll_device_status() != 0:
+        raise RuntimeError(f"{wk.label}: device status word set during warm-up")
+    graphs, launch = (None, "eager") if args.eager else wk.capture_graphs()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        time.sleep(0.25)  # let the sampler start
+        for i in range(args.steps):
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            if graphs:
+                graphs[0].replay()
+            else:
+                wk.build()
+            e1.record(stream)
+            if graphs:
+                graphs[1].replay()
+            else:
+                wk.forward()
+            e2.record(stream)
+            flush.zero_()
+        torch.cuda.synchronize()
+        time.sleep(0.15)
+    if world > 1:
+        dist.barrier()
+    mask_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    fwd_ms = [b.elapsed_time(c_) for _, b, c_ in ev]
+    step_ms = [a.elapsed_time(c_) for a, _, c_ in ev]
+    total_ms = max_over_ranks(sum(step_ms), dev, world)
+    if fa.flexattn_poll_device_status() != 0:
+        raise RuntimeError(f"{wk.label}: device status word set during the timed region")
+    del graphs
+
+    ms_per_step = total_ms / args.steps
+    fwd_mean = statistics.mean(fwd_ms)
+    c = wk.c
+    r = {"workload": wk.label, "config": describe(wk.name, c)[1], "launch": launch,
+         "ms_per_step": ms_per_step, "forward_ms": fwd_mean, "forward_ms_median": statistics.median(fwd_ms),
+         "block_mask_ms": statistics.mean(mask_ms), "gpu_launches": wk.launches_per_step * args.steps,
+         "clocks": clocks.summary()}
+    if wk.decode:
+        r["value"] = whole_job_rate(wk.kv_bytes, world, ms_per_step, 1e9)
+        r["unit"] = "GB/s"
+        achieved = wk.kv_bytes / (fwd_mean * 1e-3) / 1e9
+        r["roofline"] = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}",
+                         "frac_of_8000_gbs": achieved / 8000.0,
+                         "bytes_counted": "valid KV cache, sum_b len_b * Hkv * (E + Ev) * 2 B"}
+        r["kv_bytes"] = wk.kv_bytes
+        kind = "decode"
+    else:
+        r["value"] = whole_job_rate(wk.vis_flops, world, ms_per_step, 1e12)
+        r["unit"] = "TFLOP/s"
+        achieved = wk.visited_flops / (fwd_mean * 1e-3) / 1e12
+        if wk.general:
+            r["roofline"] = None
+            kind = "general"
+        else:
+            r["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                             "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                             "flops_counted_over": "visited-tile cells, (2E + 2Ev) per cell"}
+            kind = "prefill"
+        r["visible_pairs_flops"] = wk.vis_flops
+        r["visited_cells"] = wk.visited_cells
+        r["visible_tflops_forward_only"] = wk.vis_flops / (fwd_mean * 1e-3) / 1e12
+        r["visited_tflops_forward_only"] = achieved
+    src_hash = kernel_source_hash(kind)
+    r["kernel_source"] = src_hash
+    if r["roofline"] is not None:
+        tr = NCU_TRAFFIC.get(wk.label)
+        r["roofline"]["traffic"] = tr["bytes"] if tr and tr["source_hash"] == src_hash and not args.batch else None
+    return r
+
+
+def measure_e2e(wk, args, dev, world, flush):
+    """The same metric through the public Python API, with pinned-host inputs
+    copied in and out / lse read back inside the timed region of every step."""
+    import torch
+    stream = torch.cuda.current_stream()
+    q_p, k_p, v_p = wk.q_h.pin_memory(), wk.k_h.pin_memory(), wk.v_h.pin_memory()
+    out_p = torch.empty(wk.out.shape, dtype=wk.out.dtype).pin_memory()
+    lse_p = torch.empty(wk.lse.shape, dtype=wk.lse.dtype).pin_memory()
+    n = max(3, min(args.steps, 20))
+    for _ in range(2):
+        wk.q.copy_(q_p, non_blocking=True)
+        wk.step()
+    torch.cuda.synchronize()
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        ee[i][0].record(stream)
+        wk.q.copy_(q_p, non_blocking=True)
+        wk.k.copy_(k_p, non_blocking=True)
+        wk.v.copy_(v_p, non_blocking=True)
+        wk.step()
+        out_p.copy_(wk.out, non_blocking=True)
+        lse_p.copy_(wk.lse, non_blocking=True)
+        ee[i][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ee), dev, world)
+    h2d = sum(t.numel() * t.element_size() for t in (wk.q, wk.k, wk.v))
+    d2h = wk.out.numel() * wk.out.element_size() + wk.lse.numel() * wk.lse.element_size()
+    work, scale, unit = ((wk.kv_bytes, 1e9, "GB/s") if wk.decode else (wk.vis_flops, 1e12, "TFLOP/s"))
+    return {"value": whole_job_rate(work, world, e2e_ms, scale), "unit": unit, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -368,187 +623,49 @@ def run_gpu(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     fa.load_library()
-
-    name = args.workload
-    c, (q_h, k_h, v_h), mask, score, kv_len, doc_lengths = make_inputs(name, dev, seed_offset=rank, batch=args.batch)
-    B, Hq, L, E, Ev = c["B"], c["Hq"], c["L"], c["E"], c["Ev"]
-    BM, BN = c["BM"], c["BN"]
-    B_mask = B if kv_len is not None else 1
-    gqa = c["Hq"] != c["Hkv"]
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    out = torch.empty((B, Hq, L, Ev), dtype=q.dtype, device=dev)
-    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
-    bm = fa.flexattn_build_block_mask(mask, B_mask, 1, L, c["S"], BM, BN, device=dev)
-    ws_bytes = fa.flexattn_forward_workspace_size(q, k, v, bm)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    decode = name == "decode_kv_cache"
-    # classifier + forward kernel, + the log-sum-exp combine when decode splits the keys
-    launches_per_step = 2 + (1 if decode and ws_bytes > 0 else 0)
-    flop_pair = 2 * E + 2 * Ev
-    vis_pairs = visible_pairs_per_head(c, kv_len, doc_lengths) * Hq
-    vis_flops = vis_pairs * flop_pair
-    cells = visited_cells(bm) * (Hq if bm.H == 1 else 1) * (B if bm.B == 1 else 1)
-    visited_flops = cells * flop_pair
-    kv_bytes = None
-    if decode:
-        kv_bytes = int(np.sum(kv_len)) * c["Hkv"] * (E + Ev) * q.element_size()
-
-    def step():
-        fa.flexattn_build_block_mask(mask, B_mask, 1, L, c["S"], BM, BN, out=bm)
-        fa.flexattn_forward(q, k, v, bm, score_mod=score, mask_mod=mask, scale=c["scale"], enable_gqa=gqa,
-                            out=out, lse=lse, workspace=ws)
-
-    stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        step()
-        flush.zero_()
-    torch.cuda.synchronize()
-    if fa.flexattn_poll_device_status() != 0:
-        raise RuntimeError("device status word set during warm-up")
-
-    # The step's two calls are captured into CUDA graphs (one per call, so
-    # the events can split them) and replayed, as a serving loop would: the
-    # launches then carry no host overhead.  A graph is used only after its
-    # replay reproduces the eager result; otherwise the calls run eagerly.
-    launch = "eager"
-    graphs = None
-    if not args.eager:
-        try:
-            out_ref, lse_ref = out.float().clone(), lse.clone()
-            g_mask, g_fwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_mask, capture_error_mode="relaxed"):
-                fa.flexattn_build_block_mask(mask, B_mask, 1, L, c["S"], BM, BN, out=bm)
-            with torch.cuda.graph(g_fwd, capture_error_mode="relaxed"):
-                fa.flexattn_forward(q, k, v, bm, score_mod=score, mask_mod=mask, scale=c["scale"], enable_gqa=gqa,
-                                    out=out, lse=lse, workspace=ws)
-            out.zero_()
-            lse.zero_()
-            g_mask.replay()
-            g_fwd.replay()
-            torch.cuda.synchronize()
-            fin = torch.isfinite(lse_ref)
-            same = (torch.equal(fin, torch.isfinite(lse)) and (out.float() - out_ref).abs().max().item() <= 1e-2
-                    and (lse[fin] - lse_ref[fin]).abs().max().item() <= 1e-3)
-            if same and fa.flexattn_poll_device_status() == 0:
-                graphs = (g_mask, g_fwd)
-                launch = "CUDA graph replay, one graph per call"
-            else:
-                launch = "eager (graph replay did not reproduce the eager result)"
-        except Exception as exc:  # capture unsupported here: keep the eager launches
-            launch = f"eager (graph capture failed: {type(exc).__name__})"
-            torch.cuda.synchronize()
-
-    # ---- device-timed region: K steps, L2 flushed between steps (outside the events)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
-        time.sleep(0.25)  # let the sampler start
-        for i in range(args.steps):
-            e0, e1, e2 = ev[i]
-            e0.record(stream)
-            if graphs:
-                graphs[0].replay()
-            else:
-                fa.flexattn_build_block_mask(mask, B_mask, 1, L, c["S"], BM, BN, out=bm)
-            e1.record(stream)
-            if graphs:
-                graphs[1].replay()
-            else:
-                fa.flexattn_forward(q, k, v, bm, score_mod=score, mask_mod=mask, scale=c["scale"], enable_gqa=gqa,
-                                    out=out, lse=lse, workspace=ws)
-            e2.record(stream)
-            flush.zero_()
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    mask_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    fwd_ms = [b.elapsed_time(c_) for _, b, c_ in ev]
-    step_ms = [a.elapsed_time(c_) for a, _, c_ in ev]
-    total_ms = max_over_ranks(sum(step_ms), dev, world)
-    if fa.flexattn_poll_device_status() != 0:
-        raise RuntimeError("device status word set during the timed region")
-
-    # ---- end to end through the public API from pinned host buffers
-    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
-    out_p = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        q.copy_(q_p, non_blocking=True)
-        step()
-    torch.cuda.synchronize()
-    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-    for i in range(e2e_steps):
-        ee[i][0].record(stream)
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
-        step()
-        out_p.copy_(out, non_blocking=True)
-        lse_p.copy_(lse, non_blocking=True)
-        ee[i][1].record(stream)
-        flush.zero_()
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ee), dev, world)
-    h2d = (q.numel() * q.element_size() + k.numel() * k.element_size() + v.numel() * v.element_size())
-    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    labels = [it[0] for it in BENCH_ITEMS] if args.workload == "all" else [args.workload]
+    head = labels[0]
+    per, e2e = {}, None
+    for label in labels:
+        wk = Workload(label, dev, rank, batch=args.batch)
+        per[label] = measure(wk, args, dev, world, flush, peaks, peak_src)
+        if label == head:
+            e2e = measure_e2e(wk, args, dev, world, flush)
+        del wk
+        torch.cuda.empty_cache()
 
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    peaks, peak_src = load_peaks()
-    ms_per_step = total_ms / args.steps
-    fwd_mean = statistics.mean(fwd_ms)
-    if decode:
-        value = whole_job_rate(kv_bytes, world, ms_per_step, 1e9)
-        unit = "GB/s"
-        achieved = kv_bytes / (fwd_mean * 1e-3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}"}
-        e2e_val = whole_job_rate(kv_bytes, world, e2e_ms, 1e9)
-    else:
-        value = whole_job_rate(vis_flops, world, ms_per_step, 1e12)
-        unit = "TFLOP/s"
-        achieved = visited_flops / (fwd_mean * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"], "peak_source": f"bf16_tflops (burst) of {peak_src}",
-                    "flops_counted_over": "visited-tile cells, (2E + 2Ev) per cell"}
-        e2e_val = whole_job_rate(vis_flops, world, e2e_ms, 1e12)
-    src_hash = kernel_source_hash("decode" if decode else "prefill")
-    tr = NCU_TRAFFIC.get(name)
-    roofline["traffic"] = tr["bytes"] if tr and tr["source_hash"] == src_hash and not args.batch else None
-
-    line = {
-        "metric": METRIC_PREFILL, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if c["dtype"] == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": name, **describe(name, c)[1],
-                   "l2": "flushed: 256 MiB written between timed steps, outside the events",
-                   "step": "block-mask build + forward",
-                   "launch": launch,
-                   "parallelism": f"weak scaling over {world} GPU(s): each rank runs the full per-GPU workload"},
-        "roofline": roofline,
-        "detail": {"forward_ms": fwd_mean, "block_mask_ms": statistics.mean(mask_ms),
-                   "visible_pairs": vis_pairs, "visited_cells": cells,
-                   "visible_tflops_forward_only": vis_flops / (fwd_mean * 1e-3) / 1e12,
-                   "visited_tflops_forward_only": visited_flops / (fwd_mean * 1e-3) / 1e12,
-                   "kernel_source": src_hash},
-        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
-    }
     if not args.no_cpu_baseline and world == 1:
-        rate, el, cores, sample, _, rate_unit = oracle_sample_rate(name, target_s=args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": rate_unit, "cores": cores, "kind": "oracle",
-                                "sample": sample, "seconds": el}
+        for label in labels:
+            per[label]["cpu_baseline"] = cpu_baseline(label, args.cpu_seconds if label == head else
+                                                      args.cpu_seconds_other)
+    h = per[head]
+    _, hname, hover = item(head)
+    hc = wl.config(hname, **hover)
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": h["unit"], "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if hc["dtype"] == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": head, **describe(hname, hc)[1],
+                   "l2": "flushed: 256 MiB written between timed steps, outside the events",
+                   "step": "block-mask build + forward", "launch": h["launch"],
+                   "parallelism": f"weak scaling over {world} GPU(s): each rank runs the full per-GPU workloads",
+                   "workloads_run": labels},
+        "roofline": h["roofline"],
+        "detail": {"headline": head, "per_config": per},
+        "e2e": e2e,
+        "gpu_launches": h["gpu_launches"],
+        "clocks": h["clocks"],
+    }
+    if "cpu_baseline" in h:
+        line["cpu_baseline"] = h["cpu_baseline"]
     print(json.dumps(line))
     return 0
 
@@ -556,16 +673,19 @@ def run_gpu(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="causal_softcap_alibi", choices=sorted(wl.CONFIGS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="all", choices=["all"] + [it[0] for it in BENCH_ITEMS],
+                    help="one bench item (it becomes the headline), or all of them (default)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle seconds for the headline's cpu_baseline")
+    ap.add_argument("--cpu-seconds-other", type=float, default=3.0,
+                    help="oracle seconds for each other workload's cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed calls directly instead of replaying CUDA graphs of them")
     ap.add_argument("--batch", type=int, default=None,
-                    help="override the workload's batch size (smaller captures for profiling)")
+                    help="override the workloads' batch size (smaller captures for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -161,6 +161,38 @@ typedef struct fa_tensor {
 } fa_tensor;
 
 /* ----------------------------------------------------------------------- */
+/* Per-call options of flexattn_forward (pass NULL for the defaults).       */
+/* ----------------------------------------------------------------------- */
+enum {
+  /* The caller promises that every query row has at least one visible key
+   * whose transformed score is finite ("PyTorch Flex Attention complete
+   * guide" section 5, ROWS_GUARANTEED_SAFE, default off; "flexattention-
+   * score-mod-block-mask", "Correctness checks come before performance": a
+   * property the caller has proven, not a speed switch).  The kernels then
+   * drop their guard for rows without a visible key (the -inf tests of the
+   * running maximum and the zero / -inf substitution at the end); a row that
+   * breaks the promise gets unspecified out, lse and max_scores values,
+   * possibly NaN. */
+  FA_FLAG_ROWS_GUARANTEED_SAFE = 1
+};
+
+typedef struct fa_forward_options {
+  float* max_scores;    /* optional device fp32 [B, Hq, L], contiguous (NULL: not written):
+                           per row, the largest transformed score g_ij among the visible
+                           keys, in the units of lse (natural log scale); -inf for a row
+                           without a visible key ("PyTorch Flex Attention complete guide"
+                           section 2, AuxRequest / AuxOutput max_scores)                   */
+  int64_t wait_cycles;  /* budget of each device-side wait on the main path, in GPU clock
+                           cycles; 0 = the default (about 2 s).  A small budget makes the
+                           first wait that is not already satisfied give up, so that the
+                           timeout path (FA_ERR_TIMEOUT in the device status word, outputs
+                           unspecified) can be exercised; the waits that drain a CTA's own
+                           copies and MMAs before it exits keep the default budget       */
+  int32_t flags;        /* FA_FLAG_*                                                        */
+  int32_t reserved;     /* must be 0                                                        */
+} fa_forward_options;
+
+/* ----------------------------------------------------------------------- */
 /* Entry points                                                             */
 /* ----------------------------------------------------------------------- */
 
@@ -202,7 +234,9 @@ int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, cons
  * out_i = 0 and lse_i = -inf, never NaN.
  *
  *   q   (B, Hq, L, E), k (B, Hkv, S, E), v (B, Hkv, S, Ev); out (B, Hq, L, Ev)
- *       with out->dtype == q->dtype; k, v, q share one dtype.
+ *       with out->dtype == q->dtype or FA_DTYPE_F32 (fp32 output from bf16
+ *       inputs: the fp32 result is stored without rounding to bf16); k, v,
+ *       q share one dtype.
  *   lse optional device fp32 [B, Hq, L], contiguous (NULL: not written).
  *   enable_gqa: query head h reads KV head h / (Hq / Hkv) ([guide] 6.1).
  *   block_mask: built for (L, S) with B in {1, B}, H in {1, Hq}; its BM, BN
@@ -214,6 +248,8 @@ int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, cons
  *       the visibility structure changes; the library keeps no cache).
  *   split_kv: 0 = automatic (short queries, L <= 16, use split-KV decode),
  *       1 = never split, n > 1 = split each row of tiles into n parts.
+ *   options: NULL, or max_scores, the rows-guaranteed-safe flag and the wait
+ *       budget (fa_forward_options above).
  *   workspace: device scratch of at least flexattn_forward_workspace_size()
  *       bytes (may be NULL when that size is 0); it must not be used by any
  *       other work in flight on the GPU during the call.
@@ -223,7 +259,8 @@ int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, cons
 int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
                      float* lse, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
                      const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, int32_t split_kv,
-                     void* workspace, size_t workspace_bytes, void* stream);
+                     const fa_forward_options* options, void* workspace, size_t workspace_bytes,
+                     void* stream);
 
 /* The split-KV decode of flexattn_forward, for callers that must not allocate
  * device memory.  The pages have no counterpart of this entry point: it exists
@@ -247,8 +284,11 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
  *
  * Only the decode path runs here (bf16, E == Ev in {64, 128}, L <= 16, one
  * query tile, BN in {64, 128}, split_kv != 1); anything else returns
- * FA_ERR_UNSUPPORTED.  A call needing more than 16 MiB of scratch
- * (B * Hq * L * splits * (Ev + 1) * 4 bytes) returns FA_ERR_WORKSPACE.
+ * FA_ERR_UNSUPPORTED.  With split_kv == 0 the split count is the one
+ * flexattn_forward would choose, lowered to what the scratch holds, and one
+ * split (which needs no scratch) when not even two fit.  A call needing
+ * more than 16 MiB of scratch (B * Hq * L * splits * (Ev + 2) * 4 bytes for
+ * splits > 1) returns FA_ERR_WORKSPACE.
  * Other errors: those of flexattn_forward. */
 int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
                                     float* lse, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,

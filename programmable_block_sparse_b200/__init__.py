@@ -193,23 +193,46 @@ def flexattn_forward_workspace_size(q, k, v, block_mask, split_kv=0):
     return n.value
 
 
-def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=None, enable_gqa=False,
-                     out=None, lse=True, split_kv=0, workspace=None, stream=None):
-    """Run the forward pass; returns ``(out, lse)`` (lse None when ``lse=False``).
+def _options_struct(max_scores, rows_guaranteed_safe, wait_cycles):
+    if max_scores is None and not rows_guaranteed_safe and not wait_cycles:
+        return None
+    o = _abi.fa_forward_options()
+    o.max_scores = None if max_scores is None else max_scores.data_ptr()
+    o.wait_cycles = int(wait_cycles or 0)
+    o.flags = _abi.FA_FLAG_ROWS_GUARANTEED_SAFE if rows_guaranteed_safe else 0
+    o.reserved = 0
+    return o
 
-    ``out`` / ``lse`` may be preallocated tensors; ``workspace`` a uint8 device
-    tensor of at least :func:`flexattn_forward_workspace_size` bytes (allocated
-    here when None and needed).
+
+def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=None, enable_gqa=False,
+                     out=None, lse=True, split_kv=0, workspace=None, stream=None, out_dtype=None,
+                     max_scores=None, rows_guaranteed_safe=False, wait_cycles=0):
+    """Run the forward pass; returns ``(out, lse)`` (lse None when ``lse=False``),
+    or ``(out, lse, max_scores)`` when ``max_scores`` is requested.
+
+    ``out`` / ``lse`` may be preallocated tensors; ``out_dtype`` (torch.float32
+    or the input dtype) picks the output type when ``out`` is None;
+    ``workspace`` a uint8 device tensor of at least
+    :func:`flexattn_forward_workspace_size` bytes (allocated here when None and
+    needed).  ``max_scores``: True (allocate) or an fp32 (B, Hq, L) tensor for
+    the per-row maximum score.  ``rows_guaranteed_safe`` sets
+    FA_FLAG_ROWS_GUARANTEED_SAFE; ``wait_cycles`` the device wait budget.
     """
     import torch
     B, Hq, L, _ = q.shape
     Ev = v.shape[3]
     if out is None:
-        out = torch.empty((B, Hq, L, Ev), dtype=q.dtype, device=q.device)
+        out = torch.empty((B, Hq, L, Ev), dtype=out_dtype or q.dtype, device=q.device)
     if lse is True:
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     elif lse is False:
         lse = None
+    want_max = max_scores is not None and max_scores is not False
+    if max_scores is True:
+        max_scores = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    elif max_scores is False:
+        max_scores = None
+    opts = _options_struct(max_scores, rows_guaranteed_safe, wait_cycles)
     ws_bytes = flexattn_forward_workspace_size(q, k, v, block_mask, split_kv)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
@@ -221,8 +244,10 @@ def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=N
         sc = 0.0
     _check(load_library().flexattn_forward(
         C.byref(qs), C.byref(ks), C.byref(vs), C.byref(os_), _ptr(lse), C.c_float(sc), int(bool(enable_gqa)),
-        C.byref(sm), C.byref(mm), C.byref(bm), int(split_kv), _ptr(workspace),
-        C.c_size_t(workspace.numel() if workspace is not None else 0), _stream_handle(stream)))
+        C.byref(sm), C.byref(mm), C.byref(bm), int(split_kv), None if opts is None else C.byref(opts),
+        _ptr(workspace), C.c_size_t(workspace.numel() if workspace is not None else 0), _stream_handle(stream)))
+    if want_max:
+        return out, lse, max_scores
     return out, lse
 
 

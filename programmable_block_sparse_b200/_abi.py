@@ -15,6 +15,8 @@ FA_ERR_TIMEOUT = 13
 FA_DTYPE_BF16 = 0
 FA_DTYPE_F32 = 1
 
+FA_FLAG_ROWS_GUARANTEED_SAFE = 1
+
 MASK_KIND = {"none": 0, "causal": 1, "sliding_window": 2, "document": 3, "prefix_lm": 4, "chunked": 5}
 SCORE_KIND = {"none": 0, "softcap": 1, "alibi": 2, "cap_then_bias": 3}
 
@@ -49,6 +51,12 @@ class fa_tensor(C.Structure):
     ]
 
 
+class fa_forward_options(C.Structure):
+    _fields_ = [
+        ("max_scores", C.c_void_p), ("wait_cycles", C.c_int64), ("flags", C.c_int32), ("reserved", C.c_int32),
+    ]
+
+
 # (name, restype, argtypes) for every exported entry point.
 PROTOTYPES = [
     ("flexattn_version", C.c_int, []),
@@ -62,7 +70,7 @@ PROTOTYPES = [
     ("flexattn_forward", C.c_int,
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
       C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),
-      C.c_int32, C.c_void_p, C.c_size_t, C.c_void_p]),
+      C.c_int32, C.POINTER(fa_forward_options), C.c_void_p, C.c_size_t, C.c_void_p]),
     ("flexattn_forward_decode_noalloc", C.c_int,
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
       C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),

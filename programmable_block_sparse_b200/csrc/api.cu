@@ -248,6 +248,20 @@ bool aligned16(const fa_tensor* t) {
   return true;
 }
 
+int apply_options(const fa_forward_options* o, FwdArgs* a) {
+  a->max_scores = nullptr;
+  a->rows_safe = 0;
+  a->wait_cycles = kWaitCycles;
+  if (o == nullptr) return FA_OK;
+  if (o->reserved != 0) return fail(FA_ERR_PARAM, "options: reserved field must be 0");
+  if (o->flags & ~FA_FLAG_ROWS_GUARANTEED_SAFE) return fail(FA_ERR_PARAM, "options: unknown flags 0x%x", o->flags);
+  if (o->wait_cycles < 0) return fail(FA_ERR_PARAM, "options: wait_cycles must be >= 0");
+  a->max_scores = o->max_scores;
+  a->rows_safe = (o->flags & FA_FLAG_ROWS_GUARANTEED_SAFE) ? 1 : 0;
+  if (o->wait_cycles > 0) a->wait_cycles = o->wait_cycles;
+  return FA_OK;
+}
+
 int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out, float scale,
             int32_t enable_gqa, const fa_score_mod* score, const fa_mask_mod* mask, const fa_block_mask* bm,
             int32_t split_kv, FwdArgs* a, Path* path) {
@@ -256,7 +270,8 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   if (out != nullptr && (rc = check_tensor(out, "out"))) return rc;
   if (!score || !mask || !bm) return fail(FA_ERR_NULL, "score_mod, mask_mod and block_mask must not be NULL");
   if (k->dtype != q->dtype || v->dtype != q->dtype) return fail(FA_ERR_DTYPE, "q, k and v must share one dtype");
-  if (out && out->dtype != q->dtype) return fail(FA_ERR_DTYPE, "out must have the dtype of q");
+  if (out && out->dtype != q->dtype && out->dtype != FA_DTYPE_F32)
+    return fail(FA_ERR_DTYPE, "out must have the dtype of q, or be fp32");
   const int B = (int)q->size[0], Hq = (int)q->size[1], L = (int)q->size[2], E = (int)q->size[3];
   const int Hkv = (int)k->size[1], S = (int)k->size[2], Ev = (int)v->size[3];
   if (k->size[0] != B || v->size[0] != B) return fail(FA_ERR_BATCH, "q, k and v must have the same batch size");
@@ -301,6 +316,8 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   a->Ev = Ev;
   a->G = Hq / Hkv;
   a->dtype = q->dtype;
+  a->out_f32 = out != nullptr && out->dtype == FA_DTYPE_F32;
+  a->wait_cycles = kWaitCycles;
   a->scale = (scale > 0.0f && !isinf(scale)) ? scale : 1.0f / sqrtf(static_cast<float>(E));
   a->mask = to_device(mask);
   a->score = to_device(score);
@@ -393,13 +410,14 @@ int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, cons
 
 int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out, float* lse,
                      float scale, int32_t enable_gqa, const fa_score_mod* score_mod, const fa_mask_mod* mask_mod,
-                     const fa_block_mask* block_mask, int32_t split_kv, void* workspace, size_t workspace_bytes,
-                     void* stream) {
+                     const fa_block_mask* block_mask, int32_t split_kv, const fa_forward_options* options,
+                     void* workspace, size_t workspace_bytes, void* stream) {
   if (!out) return fail(FA_ERR_NULL, "out is NULL");
   FwdArgs a;
   Path path;
   int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
   if (rc) return rc;
+  if ((rc = apply_options(options, &a))) return rc;
   int serr = 0;
   a.status = status_word(&serr);
   if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
@@ -439,6 +457,7 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
   Path path;
   int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
   if (rc) return rc;
+  if ((rc = apply_options(nullptr, &a))) return rc;
   if (path != Path::kDecode)
     return fail(FA_ERR_UNSUPPORTED,
                 "the no-allocation entry point runs only the split-KV decode path (bf16, E == Ev in {64, 128}, "
@@ -446,10 +465,18 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
   DecodePlan plan;
   plan_decode(a, split_kv, sm_count(), &plan);
   if (split_kv == 0 && plan.workspace_bytes > kNoAllocScratchBytes) {
-    // automatic split count: take the most splits the built-in scratch holds
-    const size_t per_split = static_cast<size_t>(a.B) * a.Hq * a.L * (a.Ev + 1) * sizeof(float);
+    // automatic split count: the most splits the built-in scratch holds, or a
+    // single split (results straight to out / lse, no scratch) when not even
+    // two fit
+    const size_t per_split = static_cast<size_t>(a.B) * a.Hq * a.L * (a.Ev + 2) * sizeof(float);
     const size_t fit = kNoAllocScratchBytes / per_split;
-    if (fit >= 2) plan_decode(a, static_cast<int32_t>(fit < 65536 ? fit : 65536), sm_count(), &plan);
+    if (fit >= 2) {
+      plan_decode(a, static_cast<int32_t>(fit < 65536 ? fit : 65536), sm_count(), &plan);
+    } else {
+      plan.splits = 1;
+      plan.tiles_per_split = a.bm.Nb;
+      plan.workspace_bytes = 0;
+    }
   }
   if (plan.workspace_bytes > kNoAllocScratchBytes)
     return fail(FA_ERR_WORKSPACE,

@@ -20,9 +20,13 @@
 //             HBM, not the tensor pipe); score rule, element mask and online
 //             softmax in registers.  The four warps' (max, sum, O) are merged
 //             through shared memory at the end.
-//   output    one split: out and lse directly.  Several splits: normalised O
-//             and lse per split into the workspace, then combine_kernel merges
-//             them: lse = ln sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
+//   output    one split: out and lse directly.  Several splits: normalised O,
+//             lse and the row maximum per split into the workspace, then
+//             combine_kernel merges them: lse = ln sum_s e^{lse_s},
+//             o = sum_s e^{lse_s - lse} o_s, max_scores = max_s m_s.
+//   abort     when a bounded wait gives up, the consumers skip the merge (it
+//             reuses the stage buffers, which copies in flight may still
+//             fill) and write nothing; the producer drains its own copies.
 #include <math.h>
 
 #include "common.cuh"
@@ -40,6 +44,10 @@ constexpr int kRows = 16;       // query rows per CTA (one m16 fragment)
 constexpr float kLog2eD = 1.4426950408889634f;
 constexpr float kLn2D = 0.6931471805599453f;
 constexpr float kRescaleThresholdD = 8.0f;  // log2 units
+// Start of the running maximum: finite and below any real score (log2
+// units), so that keys hidden from a row give P = 2^-inf = 0 with no test of
+// the maximum, and the first visible key always moves it.
+constexpr float kNoKeyMaxD = -1.0e30f;
 
 template <int D>
 struct DecCfg {
@@ -93,11 +101,11 @@ __device__ __forceinline__ int list_tile(const FwdArgs& a, int64_t brow, int nfu
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_kernel(const FwdArgs a, const DecodePlan p, const __grid_constant__ CUtensorMap map_k,
-                  const __grid_constant__ CUtensorMap map_v, float* ws_o, float* ws_lse) {
+                  const __grid_constant__ CUtensorMap map_v, float* ws_o, float* ws_lse, float* ws_max) {
   using C = DecCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ DecBars bars;
-  __shared__ float s_m[4][kRows], s_l[4][kRows];
+  __shared__ float s_m[4][kRows], s_l[4][kRows], s_t[4][kRows];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       int issued = 0;
       for (int u = 0; u < nsub && !*abort; ++u) {
         const int s = u % kStagesDec;
-        if (u >= kStagesDec && !mbar_wait(&bars.empty[s], ((u / kStagesDec) - 1) & 1, abort, a.status)) break;
+        if (u >= kStagesDec && !mbar_wait(&bars.empty[s], ((u / kStagesDec) - 1) & 1, abort, a.status, a.wait_cycles)) break;
         const int n = list_tile(a, brow, nfull, t0 + u / subs_per_tile);
         const int kv0 = n * a.bm.BN + (u % subs_per_tile) * kSub;
         uint8_t* st = smem + s * C::kStageBytes;
@@ -150,11 +158,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         }
         issued = u + 1;
       }
-      if (*abort) {
-        volatile int never = 0;
-        for (int u = (issued > kStagesDec ? issued - kStagesDec : 0); u < issued; ++u)
-          mbar_wait(&bars.full[u % kStagesDec], (u / kStagesDec) & 1, &never, nullptr);
-      }
+      // Every copy issued lands before this thread leaves, on every path: a
+      // consumer may give up after the loop above has ended, and the CTA must
+      // not exit with copies still in flight.  Only the last kStagesDec can
+      // be pending (each earlier slot was waited free before its reuse), and
+      // on the normal path they have landed already.
+      volatile int never = 0;
+      for (int u = (issued > kStagesDec ? issued - kStagesDec : 0); u < issued; ++u)
+        mbar_wait(&bars.full[u % kStagesDec], (u / kStagesDec) & 1, &never, nullptr);
     }
   } else {
     const int cw = warp - 1;            // consumer warp: keys [16 cw, 16 cw + 16) of each stage
@@ -197,11 +208,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     float o[D / 8][4];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    float m_run[2] = {kNoKeyMaxD, kNoKeyMaxD}, l_run[2] = {0.0f, 0.0f};
+    float m_true[2] = {-INFINITY, -INFINITY};  // exact row maxima (log2 units), for max_scores
 
     for (int u = 0; u < nsub; ++u) {
       const int s = u % kStagesDec;
-      if (!mbar_wait(&bars.full[s], (u / kStagesDec) & 1, abort, a.status)) break;
+      // a warp-uniform result: the lanes leave the loop together or not at all
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[s], (u / kStagesDec) & 1, abort, a.status, a.wait_cycles)))
+        break;
       const int j = t0 + u / subs_per_tile;
       const bool full = j < nfull;
       const int n = list_tile(a, brow, nfull, j);
@@ -254,13 +268,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       for (int half = 0; half < 2; ++half) {
         mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 1));
         mx[half] = fmaxf(mx[half], __shfl_xor_sync(0xffffffffu, mx[half], 2));
+        m_true[half] = fmaxf(m_true[half], mx[half]);
         grow[half] = mx[half] > m_run[half] + kRescaleThresholdD;
       }
       if (__any_sync(0xffffffffu, grow[0] || grow[1])) {
         float alpha[2];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          alpha[half] = grow[half] ? ((m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - mx[half])) : 1.0f;
+          alpha[half] = grow[half] ? ex2f_approx(m_run[half] - mx[half]) : 1.0f;
           if (grow[half]) m_run[half] = mx[half];
           l_run[half] *= alpha[half];
         }
@@ -272,15 +287,12 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           o[i][3] *= alpha[1];
         }
       }
-      float mu[2];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) mu[half] = (m_run[half] == -INFINITY) ? 0.0f : m_run[half];
       float ps[2] = {0.0f, 0.0f};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          sc[nt][e] = ex2f_approx(sc[nt][e] - mu[e >> 1]);
+          sc[nt][e] = ex2f_approx(sc[nt][e] - m_run[e >> 1]);
           ps[e >> 1] += sc[nt][e];
         }
 #pragma unroll
@@ -314,8 +326,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       s_m[cw][r_lo + 8] = m_run[1];
       s_l[cw][r_lo] = l_run[0];
       s_l[cw][r_lo + 8] = l_run[1];
+      s_t[cw][r_lo] = m_true[0];
+      s_t[cw][r_lo + 8] = m_true[1];
     }
     named_bar_sync(1, 128);
+    // Every consumer is past its loop.  A consumer that left it early did so
+    // because a wait gave up, and *abort was set before that; the producer
+    // sets it only while some stage is still unconsumed.  So *abort is now
+    // final for this CTA: on an abort, copies may still be landing in the
+    // stage buffers the merge below reuses, so write nothing.
+    if (*abort) return;
     // merge the four warps: scale each warp's O by 2^(m_w - m) and add in smem
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -323,7 +343,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       float m = -INFINITY;
 #pragma unroll
       for (int w = 0; w < 4; ++w) m = fmaxf(m, s_m[w][rho]);
-      const float f = (m_run[half] == -INFINITY) ? 0.0f : ex2f_approx(m_run[half] - m);
+      const float f = ex2f_approx(m_run[half] - m);
 #pragma unroll
       for (int i = 0; i < D / 8; ++i) {
         o[i][2 * half] *= f;
@@ -349,20 +369,31 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const int hqr = row_head(rho), i = rho % a.L;
       float m = -INFINITY, l = 0.0f;
       for (int w = 0; w < 4; ++w) m = fmaxf(m, s_m[w][rho]);
-      for (int w = 0; w < 4; ++w) l += (s_m[w][rho] == -INFINITY) ? 0.0f : s_l[w][rho] * ex2f_approx(s_m[w][rho] - m);
-      const bool live = l > 0.0f;
+      for (int w = 0; w < 4; ++w) l += s_l[w][rho] * ex2f_approx(s_m[w][rho] - m);
+      float top = -INFINITY;
+      for (int w = 0; w < 4; ++w) top = fmaxf(top, s_t[w][rho]);
+      // a row without a visible key has l = 0: out 0 and lse -inf, unless the
+      // caller promised there is none (rows_safe), which drops this guard
+      const bool live = a.rows_safe || l > 0.0f;
       const float inv = live ? 1.0f / l : 0.0f;
       const float lse = live ? (m + log2f(l)) * kLn2D : -INFINITY;
       const int64_t row_id = (static_cast<int64_t>(b) * a.Hq + hqr) * a.L + i;
       if (p.splits == 1) {
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + hqr * a.o_stride[1] +
-                              i * a.o_stride[2];
-        for (int c = lane; c < D; c += 32) orow[c] = __float2bfloat16_rn(s_o[rho * D + c] * inv);
+        const int64_t off = b * a.o_stride[0] + hqr * a.o_stride[1] + i * a.o_stride[2];
+        if (a.out_f32) {
+          float* orow = static_cast<float*>(a.out) + off;
+          for (int c = lane; c < D; c += 32) orow[c] = s_o[rho * D + c] * inv;
+        } else {
+          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + off;
+          for (int c = lane; c < D; c += 32) orow[c] = __float2bfloat16_rn(s_o[rho * D + c] * inv);
+        }
         if (lane == 0 && a.lse) a.lse[row_id] = lse;
+        if (lane == 0 && a.max_scores) a.max_scores[row_id] = top * kLn2D;
       } else {
         float* wrow = ws_o + (row_id * p.splits + split) * D;
         for (int c = lane; c < D; c += 32) wrow[c] = s_o[rho * D + c] * inv;
         if (lane == 0) ws_lse[row_id * p.splits + split] = lse;
+        if (lane == 0) ws_max[row_id * p.splits + split] = top;
       }
     }
   }
@@ -371,7 +402,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 // One warp per (b, h, i) row: merge the per-split (o_s, lse_s).
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(const FwdArgs a, const DecodePlan p, const float* ws_o,
-                                                      const float* ws_lse) {
+                                                      const float* ws_lse, const float* ws_max) {
   const int64_t row_id = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
@@ -380,17 +411,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const FwdArgs a, const Dec
   const int h = static_cast<int>((row_id / a.L) % a.Hq);
   const int b = static_cast<int>(row_id / (static_cast<int64_t>(a.L) * a.Hq));
   const float* lrow = ws_lse + row_id * p.splits;
-  float m = -INFINITY;
-  for (int s = lane; s < p.splits; s += 32) m = fmaxf(m, lrow[s]);
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const float* trow = ws_max + row_id * p.splits;
+  float m = -INFINITY, top = -INFINITY;
+  for (int s = lane; s < p.splits; s += 32) {
+    m = fmaxf(m, lrow[s]);
+    top = fmaxf(top, trow[s]);
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    top = fmaxf(top, __shfl_xor_sync(0xffffffffu, top, off));
+  }
   float acc[D / 32];
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) acc[c] = 0.0f;
   float tot = 0.0f;
-  if (m != -INFINITY) {
+  if (a.rows_safe || m != -INFINITY) {
     for (int s = 0; s < p.splits; ++s) {
       const float ls = lrow[s];
-      if (ls == -INFINITY) continue;
+      if (!a.rows_safe && ls == -INFINITY) continue;
       const float w = expf(ls - m);
       tot += w;
       const float* orow = ws_o + (row_id * p.splits + s) * D;
@@ -398,12 +436,20 @@ __global__ void __launch_bounds__(256) combine_kernel(const FwdArgs a, const Dec
       for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, orow[lane + 32 * c], acc[c]);
     }
   }
-  const bool live = tot > 0.0f;
+  const bool live = a.rows_safe || tot > 0.0f;
   const float inv = live ? 1.0f / tot : 0.0f;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] + i * a.o_stride[2];
+  const int64_t off = b * a.o_stride[0] + h * a.o_stride[1] + i * a.o_stride[2];
+  if (a.out_f32) {
+    float* out = static_cast<float*>(a.out) + off;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) out[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
+    for (int c = 0; c < D / 32; ++c) out[lane + 32 * c] = acc[c] * inv;
+  } else {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + off;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) out[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
+  }
   if (lane == 0 && a.lse) a.lse[row_id] = live ? m + logf(tot) : -INFINITY;
+  if (lane == 0 && a.max_scores) a.max_scores[row_id] = top * kLn2D;
 }
 
 template <int D>
@@ -411,7 +457,9 @@ cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Ma
                             cudaStream_t stream) {
   const int head_chunks = (a.G + p.heads_per_cta - 1) / p.heads_per_cta;
   float* ws_o = static_cast<float*>(workspace);
-  float* ws_lse = ws_o ? ws_o + static_cast<int64_t>(a.B) * a.Hq * a.L * p.splits * D : nullptr;
+  const int64_t row_splits = static_cast<int64_t>(a.B) * a.Hq * a.L * p.splits;
+  float* ws_lse = ws_o ? ws_o + row_splits * D : nullptr;
+  float* ws_max = ws_o ? ws_lse + row_splits : nullptr;
   auto kern = a.score.kind == FA_SCORE_NONE      ? decode_kernel<D, FA_SCORE_NONE>
               : a.score.kind == FA_SCORE_SOFTCAP ? decode_kernel<D, FA_SCORE_SOFTCAP>
               : a.score.kind == FA_SCORE_ALIBI   ? decode_kernel<D, FA_SCORE_ALIBI>
@@ -419,11 +467,11 @@ cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Ma
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.splits, a.Hkv * head_chunks, a.B);
-  kern<<<grid, kDecThreads, DecCfg<D>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse);
+  kern<<<grid, kDecThreads, DecCfg<D>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse, ws_max);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.splits == 1) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
-  combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(a, p, ws_o, ws_lse);
+  combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(a, p, ws_o, ws_lse, ws_max);
   return cudaGetLastError();
 }
 
@@ -446,7 +494,8 @@ int plan_decode(const FwdArgs& a, int split_kv, int num_sms, DecodePlan* p) {
   }
   p->tiles_per_split = (Nb + splits - 1) / splits;
   p->splits = (Nb + p->tiles_per_split - 1) / p->tiles_per_split;
-  p->workspace_bytes = p->splits > 1 ? static_cast<size_t>(a.B) * a.Hq * a.L * p->splits * (a.Ev + 1) * sizeof(float)
+  // per (row, split): Ev partial outputs, the partial lse and the row maximum
+  p->workspace_bytes = p->splits > 1 ? static_cast<size_t>(a.B) * a.Hq * a.L * p->splits * (a.Ev + 2) * sizeof(float)
                                      : 0;
   return 0;
 }

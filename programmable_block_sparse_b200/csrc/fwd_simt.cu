@@ -72,7 +72,10 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
   const int qpos = query_pos(row, L, S_b);
   const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
   const float slope = distance_slope(h, Hs);
-  float m_run = -INFINITY, l_run = 0.0f;
+  // running maximum from a finite floor below any real score: hidden keys
+  // give exp(-inf) = 0 with no test of the maximum
+  constexpr float kNoKeyMaxS = -1.0e30f;
+  float m_run = kNoKeyMaxS, l_run = 0.0f;
 
   const int bmb = a.bm.B > 1 ? b : 0, bmh = a.bm.H > 1 ? h : 0;
   const int64_t brow = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb + mt;
@@ -108,12 +111,11 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
         cmax = fmaxf(cmax, val);
       }
       const float m_new = fmaxf(m_run, cmax);
-      if (m_new == -INFINITY) continue;  // nothing visible in this row yet
-      const float alpha = (m_run == -INFINITY) ? 0.0f : expf(m_run - m_new);
+      const float alpha = expf(m_run - m_new);
       float psum = 0.0f;
 #pragma unroll
       for (int j = 0; j < kChunk; ++j) {
-        s[j] = (s[j] == -INFINITY) ? 0.0f : expf(s[j] - m_new);
+        s[j] = expf(s[j] - m_new);
         psum += s[j];
       }
       l_run = l_run * alpha + psum;
@@ -127,11 +129,21 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
     }
   }
   if (!active) return;
-  T* ob = static_cast<T*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] + row * a.o_stride[2];
-  const bool live = l_run > 0.0f;
+  const int64_t ooff = b * a.o_stride[0] + h * a.o_stride[1] + row * a.o_stride[2];
+  // a row without a visible key has l_run = 0: out 0 and lse -inf, unless the
+  // caller promised there is none (rows_safe), which drops this guard
+  const bool live = a.rows_safe || l_run > 0.0f;
   const float inv = live ? 1.0f / l_run : 0.0f;
-  for (int d = 0; d < Ev; ++d) store_out<T>(ob + d, live ? so[t * ost + d] * inv : 0.0f);
-  if (a.lse) a.lse[(static_cast<int64_t>(b) * a.Hq + h) * L + row] = live ? m_run + logf(l_run) : -INFINITY;
+  if (a.out_f32) {
+    float* ob = static_cast<float*>(a.out) + ooff;
+    for (int d = 0; d < Ev; ++d) ob[d] = live ? so[t * ost + d] * inv : 0.0f;
+  } else {
+    T* ob = static_cast<T*>(a.out) + ooff;
+    for (int d = 0; d < Ev; ++d) store_out<T>(ob + d, live ? so[t * ost + d] * inv : 0.0f);
+  }
+  const int64_t rid = (static_cast<int64_t>(b) * a.Hq + h) * L + row;
+  if (a.lse) a.lse[rid] = live ? m_run + logf(l_run) : -INFINITY;
+  if (a.max_scores) a.max_scores[rid] = m_run > kNoKeyMaxS ? m_run : -INFINITY;  // the exact running maximum
 }
 
 }  // namespace

@@ -59,6 +59,10 @@ constexpr int kTile = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Start of the running maximum: finite and below any real score (log2
+// units), so that tiles without a visible key for a row give P = 2^-inf = 0
+// with no test of the maximum, and the first visible key always moves it.
+constexpr float kNoKeyMax = -1.0e30f;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -207,30 +211,45 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   const int* doc_row = is_doc ? a.mask.doc_id + static_cast<int64_t>(a.mask.doc_batch > 1 ? b : 0) * a.S : nullptr;
   const int my_doc = (is_doc && row_ok && qpos >= 0) ? __ldg(doc_row + qpos) : -1;
   const KeySpans spans = visible_spans(a.mask, qpos, S_b);
-  float m_ref = -INFINITY, l_sum = 0.0f;
+  float m_ref = kNoKeyMax, l_sum = 0.0f;
+  float m_true = -INFINITY;  // exact row maximum (log2 units), for max_scores
   bool alive = true;
   int cnt = 0;
 
   const int64_t row_x = row_a + X;
   const bool x_on = X == 0 || has_b;
   const int total = x_on ? __ldg(a.bm.full_kv_num_blocks + row_x) + __ldg(a.bm.kv_num_blocks + row_x) : 0;
+  // the four warps of the group stage key-side values for each other when
+  // the rules read positions or document ids (the same for every tile)
+  const bool group_stage = has_pos || is_doc;
+  // A warp leaves this loop only at its top, together with its whole group
+  // when the group stages key-side values (the barrier below): a wait that
+  // gives up inside a tile marks the warp dead, it skips the rest of the tile
+  // and votes false at the next barrier.
   for (; cnt < total; ++cnt) {
-    if (!mbar_wait(&bars.s_full[X], cnt & 1, abort, a.status)) {
-      alive = false;
-      break;
-    }
-    const int info = bars.info[X][cnt & 1];
+    // a warp-uniform result: the lanes leave the loop together or not at all
+    bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[X], cnt & 1, abort, a.status, a.wait_cycles));
+    const int info = ok ? bars.info[X][cnt & 1] : 0;
     const int n = info & (kInfoFull - 1);
     const bool full = (info & kInfoFull) != 0;
     const int kv0 = n * kTile;
     const bool edge = kv0 + kTile > S_b;
     const bool stage_doc = is_doc && (!full || edge);  // the same for every row of the tile
-    if (has_pos || stage_doc) {
-      // this tile's key-side values into smem (double-buffered by cnt & 1)
-      const int kv = kv0 + r;
-      if (has_pos) s_pos[cnt & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
-      if (stage_doc) s_doc[cnt & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
-      named_bar_sync(1 + X, 128);
+    if (group_stage) {
+      // this tile's key-side values into smem (double-buffered by cnt & 1);
+      // every warp of the group reaches the barrier on every tile, and it
+      // also tells each warp whether all four got their S, so that on a
+      // timeout the group leaves together and no warp waits for another
+      if (ok) {
+        const int kv = kv0 + r;
+        if (has_pos) s_pos[cnt & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
+        if (stage_doc) s_doc[cnt & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
+      }
+      ok = named_bar_and(1 + X, 128, ok);
+    }
+    if (!ok) {
+      alive = false;
+      break;
     }
     tc_fence_after();
 
@@ -294,6 +313,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
       tmem_store64(tbase + lane_base + col_s + c0, t);
     }
     tmem_wait_st();
+    m_true = fmaxf(m_true, mx);
 
     // running max: move it (and rescale O) only when it grows past 2^8.  O_X
     // holds the sum through this group's previous tile once that PV is done:
@@ -301,13 +321,15 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     // o_done barrier says so.  No MMA writes O_X until P_X is signalled.
     const bool grow_max = mx > m_ref + kRescaleThreshold;
     const float m_new = grow_max ? mx : m_ref;
-    const bool rescale = grow_max && m_ref != -INFINITY;
+    // O_X holds a sum only after the group's first tile (its first PV
+    // overwrites whatever the columns held)
+    const bool rescale = grow_max && cnt > 0;
     bool pv_done = !kSepP || cnt == 0;
     auto wait_pv = [&]() {
       // the previous tile's PV reads P and writes O; with separate S columns
       // the S of this tile may have landed before that PV finished
       if (!pv_done) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[X], (cnt - 1) & 1, abort, a.status))) alive = false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[X], (cnt - 1) & 1, abort, a.status, a.wait_cycles))) alive = false;
         tc_fence_after();
         pv_done = true;
       }
@@ -315,19 +337,21 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     if (__any_sync(0xffffffffu, rescale)) {
       wait_pv();
       const float f = rescale ? ex2_approx(m_ref - m_new) : 1.0f;
+      if (alive) {
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t rr[16];
-        tmem_ld16(tbase + lane_base + col_o + c * 16, rr);
-        tmem_wait_ld();
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rr[16];
+          tmem_ld16(tbase + lane_base + col_o + c * 16, rr);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
-        tmem_st16(tbase + lane_base + col_o + c * 16, rr);
+          for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+          tmem_st16(tbase + lane_base + col_o + c * 16, rr);
+        }
       }
       l_sum *= f;
     }
     m_ref = m_new;
-    const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+    const float m_use = m_ref;
 
     // pass 2, per half: P = 2^(t - m) as bf16 pairs, 64 columns in all
     // (head dim 128: over the first 64 S columns; half h writes columns
@@ -368,7 +392,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     }
     if (!alive) {
       tmem_wait_st();
-      break;
+      continue;  // leave at the next tile's vote, with the group
     }
     l_sum += psum;
 
@@ -380,18 +404,20 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
 
   // ------------------------------------------------------------- epilogue
   if (alive && cnt > 0) {
-    alive = mbar_wait(&bars.o_final, 0, abort, a.status);
+    alive = mbar_wait(&bars.o_final, 0, abort, a.status, a.wait_cycles);
     tc_fence_after();
   }
   // TMEM loads are warp-collective: every lane takes part, rows past L
   // included; only the stores depend on the row.
   if (__all_sync(0xffffffffu, alive)) {
-    const bool live = l_sum > 0.0f && cnt > 0;
+    // a row without a visible key has l_sum = 0: out 0 and lse -inf, unless
+    // the caller promised there is none (rows_safe), which drops this guard
+    const bool live = (a.rows_safe || l_sum > 0.0f) && cnt > 0;
     const float inv = live ? 1.0f / l_sum : 0.0f;
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] +
-                          static_cast<int64_t>(row_ok ? grow : 0) * a.o_stride[2];
-    if (row_ok && a.lse)
-      a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.L + grow] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
+    const int64_t orow_off = b * a.o_stride[0] + h * a.o_stride[1] + static_cast<int64_t>(row_ok ? grow : 0) * a.o_stride[2];
+    const int64_t rid = (static_cast<int64_t>(b) * a.Hq + h) * a.L + grow;
+    if (row_ok && a.lse) a.lse[rid] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
+    if (row_ok && a.max_scores) a.max_scores[rid] = m_true * kLn2;
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) {
       uint32_t rr[16];
@@ -402,13 +428,22 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
         tmem_wait_ld();
       }
       if (row_ok) {
-        uint32_t pk[8];
+        if (a.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow_off + c * 16);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int i = 0; i < 4; ++i)
+            dst[i] = live ? make_float4(__uint_as_float(rr[4 * i]) * inv, __uint_as_float(rr[4 * i + 1]) * inv,
+                                        __uint_as_float(rr[4 * i + 2]) * inv, __uint_as_float(rr[4 * i + 3]) * inv)
+                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        } else {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow_off + c * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
     }
   }
@@ -486,29 +521,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (has_b)
             tma_load_4d(sQ + C::kTileBytes + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mtB * kTile, h, b);
         }
-        int u = 0, issued = 0;
+        int u = 0, issued_k = 0, issued_v = 0;
         for (; any && !*abort; ++u, any = it.next(n, flags)) {
           const int s = u % NS;
           const uint32_t round = u / NS;
-          if (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status)) break;
+          if (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
           mbar_expect_tx(&bars.k_full[s], C::kTileBytes);
           for (int c = 0; c < C::kBoxes; ++c)
             tma_load_4d(sK + s * C::kTileBytes + c * (kTile * 128), &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
-          issued = u + 1;
-          if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status)) break;
+          issued_k = u + 1;
+          if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
           mbar_expect_tx(&bars.v_full[s], C::kTileBytes);
           for (int c = 0; c < C::kBoxes; ++c)
             tma_load_4d(sV + s * C::kTileBytes + c * (kTile * 128), &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
+          issued_v = u + 1;
         }
-        if (*abort) {
-          // drain: let every copy this thread issued land before the CTA exits
-          volatile int never = 0;
-          mbar_wait(&bars.q_full, 0, &never, nullptr);
-          for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j) {
-            mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
-            mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
-          }
-        }
+        // Drain on every path: each copy this thread issued lands before it
+        // leaves, so the CTA never exits with copies in flight, even when
+        // another warp gives up after this loop has ended.  Only the last NS
+        // of each ring can be pending (earlier slots were waited free before
+        // reuse); on the normal path they have landed already.
+        volatile int never = 0;
+        mbar_wait(&bars.q_full, 0, &never, nullptr);
+        for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
+          mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
+        for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
+          mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -553,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           // keys 64 hf .. 64 hf + 63 once their P is written
-          if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
+          if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status, a.wait_cycles)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
@@ -563,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++pcnt[X];
         return true;
       };
-      bool ok = have_cur && mbar_wait(&bars.q_full, 0, abort, a.status);
+      bool ok = have_cur && mbar_wait(&bars.q_full, 0, abort, a.status, a.wait_cycles);
       if constexpr (D == 64) {
         // S, P and O in separate columns: the next tile's QK of a group goes
         // in as soon as its softmax has read S (s_free), ahead of this
@@ -575,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc0 = acc[X] ? 1u : 0u;
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status)) return false;
+            if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status, a.wait_cycles)) return false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
@@ -588,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto qk_after_free = [&](int X, int s, int n, uint32_t flags) -> bool {
           if (qcnt[X] > 0) {  // the group's previous S must be read out first
-            if (!mbar_wait(&bars.s_free[X], freed[X] & 1, abort, a.status)) return false;
+            if (!mbar_wait(&bars.s_free[X], freed[X] & 1, abort, a.status, a.wait_cycles)) return false;
             ++freed[X];
             tc_fence_after();
           }
@@ -596,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         if (ok) {
-          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
+          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status, a.wait_cycles);
           tc_fence_after();
           if (ok && (f_cur & kInA)) ok = qk_after_free(0, 0, n_cur, f_cur);
           if (ok && (f_cur & kInB)) ok = qk_after_free(1, 0, n_cur, f_cur);
@@ -610,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t in_x = X == 0 ? kInA : kInB;
             if (have_nxt && (f_nxt & in_x)) {
               if (!k_ready) {
-                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
                 tc_fence_after();
                 k_ready = true;
               }
@@ -618,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (ok && (f_cur & in_x)) {
               if (!v_ready) {
-                ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status);
+                ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles);
                 tc_fence_after();
                 v_ready = true;
               }
@@ -629,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every union tile is some group's tile, and so is the next one
           umma_commit(&bars.v_empty[s]);
           if (have_nxt) {
-            if (!k_ready && !mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status)) break;
+            if (!k_ready && !mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles)) break;
             umma_commit(&bars.k_empty[s1]);
           }
           have_cur = have_nxt;
@@ -638,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         if (ok) {
-          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status);
+          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status, a.wait_cycles);
           tc_fence_after();
           if (ok) {
             if (f_cur & kInA) issue_qk(0, 0, n_cur, f_cur);
@@ -650,13 +688,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = u % NS, s1 = (u + 1) % NS;
           const bool have_nxt = it.next(n_nxt, f_nxt);
           bool k_nxt_ready = false;
-          if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status)) break;
+          if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles)) break;
           for (int X = 0; X < 2 && ok; ++X) {
             const uint32_t in_x = X == 0 ? kInA : kInB;
             if (f_cur & in_x) ok = issue_pv(X, s);
             if (ok && have_nxt && (f_nxt & in_x)) {
               if (!k_nxt_ready) {
-                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
                 tc_fence_after();
                 k_nxt_ready = true;
               }
@@ -669,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!k_nxt_ready) {
               // K_{u+1} is listed for neither group's next QK only if a group
               // skips it; it still has to be consumed before its slot is reused
-              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status);
+              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
               if (!ok) break;
             }
             umma_commit(&bars.k_empty[s1]);

@@ -36,6 +36,10 @@ struct FwdArgs {
   const void* v;
   void* out;
   float* lse;                 // [B, Hq, L] or null
+  float* max_scores;          // [B, Hq, L] or null
+  long long wait_cycles;      // budget of each main-path device wait
+  int out_f32;                // out is fp32 (else the input dtype)
+  int rows_safe;              // every row has a visible key: no empty-row guard
   int64_t q_stride[4], k_stride[4], v_stride[4], o_stride[4];
   int B, Hq, Hkv, L, S, E, Ev, G;
   int dtype;                  // FA_DTYPE_*

@@ -30,8 +30,19 @@ int main(void) {
   expect(strlen(flexattn_last_error()) > 0, "a failing call leaves a message");
 
   /* a forward call with NULL tensors is rejected on the host */
-  expect(flexattn_forward(NULL, NULL, NULL, NULL, NULL, 0.0f, 0, NULL, NULL, NULL, 0, NULL, 0, NULL) == FA_ERR_NULL,
+  expect(flexattn_forward(NULL, NULL, NULL, NULL, NULL, 0.0f, 0, NULL, NULL, NULL, 0, NULL, NULL, 0, NULL) ==
+             FA_ERR_NULL,
          "forward with NULL tensors");
+  {
+    /* the options struct is plain C and its defaults are all zero */
+    fa_forward_options opts;
+    memset(&opts, 0, sizeof(opts));
+    opts.flags = FA_FLAG_ROWS_GUARANTEED_SAFE;
+    expect(sizeof(opts) == 24, "fa_forward_options is 24 bytes");
+    expect(flexattn_forward(NULL, NULL, NULL, NULL, NULL, 0.0f, 0, NULL, NULL, NULL, 0, &opts, NULL, 0, NULL) ==
+               FA_ERR_NULL,
+           "forward with options and NULL tensors");
+  }
   expect(flexattn_build_block_mask(NULL, NULL, NULL) == FA_ERR_NULL, "block mask with NULL arguments");
 
   if (failures == 0) printf("ok\n");

@@ -88,18 +88,19 @@ class Case:
         B_mask = B_mask or (self.B if (self.kv_len is not None) else 1)
         return fa.flexattn_build_block_mask(self.dev_mask, B_mask, H_mask, self.L, self.S, BM, BN)
 
-    def run(self, BM, BN, split_kv=0, **kw):
+    def run(self, BM, BN, split_kv=0, bm=None, **kw):
+        """(out, lse), or (out, lse, max_scores) with max_scores=True."""
         import programmable_block_sparse_b200 as fa
-        bm = self.block_mask(BM, BN)
-        out, lse = fa.flexattn_forward(self.q, self.k, self.v, bm, score_mod=self.dev_score, mask_mod=self.dev_mask,
-                                       scale=self.scale32, enable_gqa=self.Hq != self.Hkv, split_kv=split_kv, **kw)
+        bm = bm or self.block_mask(BM, BN)
+        res = fa.flexattn_forward(self.q, self.k, self.v, bm, score_mod=self.dev_score, mask_mod=self.dev_mask,
+                                  scale=self.scale32, enable_gqa=self.Hq != self.Hkv, split_kv=split_kv, **kw)
         torch.cuda.synchronize()
-        return out, lse
+        return res
 
-    def oracle(self):
+    def oracle(self, aux=False):
         import oracle.flex_oracle as o
         return o.forward(self.q_cpu, self.k_cpu, self.v_cpu, self.scale32, self.oracle_mask, self.oracle_score,
-                         kv_len=self.kv_len, enable_gqa=self.Hq != self.Hkv)
+                         kv_len=self.kv_len, enable_gqa=self.Hq != self.Hkv, aux=aux)
 
     def oracle_rows(self, samples):
         import oracle.flex_oracle as o
@@ -107,16 +108,22 @@ class Case:
                                  self.oracle_score, kv_len=self.kv_len, enable_gqa=self.Hq != self.Hkv)
 
 
-def assert_close(case, out, lse, ref_out, ref_lse):
+def out_tolerance(in_dtype, out_is_fp32, ref):
+    """fp32 I/O: 1e-5.  bf16 inputs with an fp32 output: a strict 1e-2 (the
+    arithmetic alone).  bf16 output: 1e-2 plus half a bf16 ulp of ref."""
+    if in_dtype == "fp32":
+        return TOL["fp32"]["out"]
+    return 1e-2 if out_is_fp32 else bf16_tolerance(ref)
+
+
+def assert_close(case, out, lse, ref_out, ref_lse, max_scores=None, ref_max=None):
     """Element-wise comparison with the workload dtype's tolerance."""
+    out_f32 = out.dtype == torch.float32
     out = out.float().cpu().numpy().astype(np.float64)
     lse = lse.cpu().numpy().astype(np.float64)
     assert not np.isnan(out).any(), "NaN in the output"
     assert not np.isnan(lse).any(), "NaN in the lse"
-    if case.dtype == "fp32":
-        tol = TOL["fp32"]["out"]
-    else:
-        tol = bf16_tolerance(ref_out)
+    tol = out_tolerance(case.dtype, out_f32, ref_out)
     err = np.abs(out - ref_out)
     bad = err > tol
     assert not bad.any(), f"max |out - ref| = {err.max():.3e} at {np.argwhere(bad)[0].tolist()} ({bad.sum()} elems)"
@@ -126,4 +133,17 @@ def assert_close(case, out, lse, ref_out, ref_lse):
     if fin.any():
         lerr = np.abs(lse[fin] - ref_lse[fin])
         assert lerr.max() <= TOL[case.dtype]["lse"], f"max |lse - ref| = {lerr.max():.3e}"
+    if max_scores is not None:
+        assert_max_scores(max_scores, ref_max)
     return float(err.max())
+
+
+def assert_max_scores(got, ref, tol=1e-3):
+    """max_scores within the lse tolerance; rows without a visible key -inf."""
+    got = got.cpu().numpy().astype(np.float64) if hasattr(got, "cpu") else np.asarray(got, np.float64)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got), fin), "max_scores finiteness differs"
+    assert np.all(got[~fin] == -np.inf)
+    if fin.any():
+        err = np.abs(got[fin] - ref[fin])
+        assert err.max() <= tol, f"max |max_scores - ref| = {err.max():.3e}"

@@ -46,6 +46,7 @@ def test_struct_layouts_match_header_sizes():
     assert C.sizeof(_abi.fa_score_mod) == 4 * 4 + 8
     assert C.sizeof(_abi.fa_block_mask) == 8 * 4 + 4 * 8
     assert C.sizeof(_abi.fa_tensor) == 8 + 4 + 4 + 8 * 8
+    assert C.sizeof(_abi.fa_forward_options) == 8 + 8 + 4 + 4
 
 
 def test_version(lib):
@@ -84,11 +85,12 @@ def _bm(B, H, L, S, BM, BN):
     return s
 
 
-def _call(lib, q, k, v, out, bm, score=None, mask=None, gqa=0, split=0):
+def _call(lib, q, k, v, out, bm, score=None, mask=None, gqa=0, split=0, opts=None):
     score = score or _abi.fa_score_mod(kind=0)
     mask = mask or _abi.fa_mask_mod(kind=1)
     return lib.flexattn_forward(C.byref(q), C.byref(k), C.byref(v), C.byref(out) if out is not None else None,
-                                None, 0.0, gqa, C.byref(score), C.byref(mask), C.byref(bm), split, None, 0, None)
+                                None, 0.0, gqa, C.byref(score), C.byref(mask), C.byref(bm), split,
+                                C.byref(opts) if opts is not None else None, None, 0, None)
 
 
 def test_forward_rejects_bad_arguments(lib):
@@ -111,7 +113,10 @@ def test_forward_rejects_bad_arguments(lib):
     assert _call(lib, q, k, v, o, bad) == 5
     # dtype
     assert _call(lib, q, _t(2, 4, 256, 64, dtype=_abi.FA_DTYPE_F32), v, o, bm) == 6
-    assert _call(lib, q, k, v, _t(2, 4, 256, 64, dtype=_abi.FA_DTYPE_F32), bm) == 6
+    # fp32 output from bf16 inputs is allowed; bf16 output from fp32 inputs is not
+    f32 = _abi.FA_DTYPE_F32
+    assert _call(lib, _t(2, 4, 256, 64, dtype=f32), _t(2, 4, 256, 64, dtype=f32), _t(2, 4, 256, 64, dtype=f32),
+                 _t(2, 4, 256, 64), bm) == 6
     # head dim
     assert _call(lib, _t(2, 4, 256, 256), _t(2, 4, 256, 256), _t(2, 4, 256, 256), _t(2, 4, 256, 256), bm) == 7
     # strides
@@ -167,3 +172,12 @@ def test_python_binding_rejects_non_4d_tensors(lib):
     import torch
     with pytest.raises(fa.FlexAttnError):
         fa._tensor_struct(torch.zeros(2, 3, 4))
+
+
+def test_forward_rejects_bad_options(lib):
+    q, k, v, o = _t(2, 4, 256, 64), _t(2, 4, 256, 64), _t(2, 4, 256, 64), _t(2, 4, 256, 64)
+    bm = _bm(1, 1, 256, 256, 128, 128)
+    assert _call(lib, q, k, v, o, bm, opts=_abi.fa_forward_options(flags=2)) == 9
+    assert "flags" in fa.flexattn_last_error()
+    assert _call(lib, q, k, v, o, bm, opts=_abi.fa_forward_options(reserved=1)) == 9
+    assert _call(lib, q, k, v, o, bm, opts=_abi.fa_forward_options(wait_cycles=-5)) == 9

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_cases import Case, assert_close, bf16_tolerance
+from gpu_cases import Case, assert_close
 
 pytestmark = pytest.mark.gpu
 
@@ -27,9 +27,13 @@ def test_decode_against_oracle(L, Hq, Hkv, E, split_kv):
     kv_len = [1500, 700, 129, 64]
     case = Case(4, Hq, Hkv, L, 1500, E, E, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=L + E,
                 kv_len=kv_len, sentinel_tail=True)
-    out, lse = case.run(128, 128, split_kv=split_kv)
-    assert_close(case, out, lse, *case.oracle())
+    ro, rl, rm = case.oracle(aux=True)
+    out, lse, mx = case.run(128, 128, split_kv=split_kv, max_scores=True)
+    assert_close(case, out, lse, ro, rl, mx, rm)
     assert out.abs().max().item() < 10.0  # the +-1e4 cache tail never leaks
+    # an fp32 output (from the split path's combine, or straight from one split) within a strict 1e-2
+    out32, lse32 = case.run(128, 128, split_kv=split_kv, out_dtype=torch.float32)
+    assert_close(case, out32, lse32, ro, rl)
     _status_ok()
 
 
@@ -83,21 +87,4 @@ def test_split_counts_agree():
         fa.flexattn_forward(case.q, case.k, case.v, bm, score_mod=case.dev_score, mask_mod=case.dev_mask,
                             enable_gqa=True, split_kv=7, workspace=small)
     assert e.value.status == 10
-    _status_ok()
-
-
-@pytest.mark.parametrize("L", [4, 1])
-def test_decode_workload_full_size(L):
-    case = Case.from_config("decode_kv_cache", L=L)
-    out, lse = case.run(case.BM, case.BN)
-    assert torch.isfinite(lse).all() and not torch.isnan(out).any()
-    assert out.abs().max().item() < 10.0
-    rng = np.random.default_rng(0)
-    samples = sorted({(int(rng.integers(case.B)), int(rng.integers(case.Hq)), int(rng.integers(L))) for _ in range(40)}
-                     | {(0, 0, 0), (case.B - 1, case.Hq - 1, L - 1)})
-    ref_o, ref_l = case.oracle_rows(samples)
-    got_o = np.stack([out[b, h, i].float().cpu().numpy() for b, h, i in samples]).astype(np.float64)
-    got_l = np.array([lse[b, h, i].item() for b, h, i in samples])
-    assert np.all(np.abs(got_o - ref_o) <= bf16_tolerance(ref_o)), np.abs(got_o - ref_o).max()
-    assert np.all(np.abs(got_l - ref_l) <= 1e-3), np.abs(got_l - ref_l).max()
     _status_ok()

@@ -53,3 +53,37 @@ def test_configs_are_complete():
         for key in ("B", "Hq", "Hkv", "L", "S", "E", "Ev", "dtype", "seed", "scale", "BM", "BN", "mask", "score"):
             assert key in c, (name, key)
         assert c["Hq"] % c["Hkv"] == 0
+
+
+def test_oracle_pool_units_equal_whole_tensor_oracle():
+    """The pool's per-unit oracle (slices regenerated per unit in spawned
+    workers) equals the oracle on whole tensors drawn by randn_qkv, for a
+    shrunken copy of each workload kind (slope per head, documents, GQA,
+    per-sequence cache lengths with sentinel tails)."""
+    import numpy as np
+    import torch
+
+    import oracle.flex_oracle as o
+    import workloads as wl
+    from oracle_pool import oracle_units, workload_specs
+
+    cases = [("causal_softcap_alibi", dict(B=2, Hq=3, Hkv=3, L=160, S=160)),
+             ("packed_docs", dict(Hq=2, Hkv=2, L=300, S=300, doc_total=300, doc_lo=20, doc_hi=90)),
+             ("gqa_sliding_window", dict(B=1, Hq=4, Hkv=2, L=200, S=200, mask=dict(kind="sliding_window",
+                                                                                    window=37, n_sink=4))),
+             ("decode_kv_cache", dict(B=3, Hq=4, Hkv=2, L=4, S=300, kv_lo=20, kv_hi=300))]
+    for name, over in cases:
+        c, mask, score, kv_len = workload_specs(name, **over)
+        q, k, v = wl.randn_qkv(c["B"], c["Hq"], c["Hkv"], c["L"], c["S"], c["E"], c["Ev"], seed=c["seed"],
+                               dtype=torch.bfloat16)
+        if kv_len is not None:
+            wl.fill_cache_tail(k, v, kv_len)
+        scale = float(np.float32(c["scale"]))
+        ref_o, ref_l, ref_m = o.forward(q, k, v, scale, mask, score, kv_len=kv_len, enable_gqa=True, aux=True)
+        units = [(b, h) for b in range(c["B"]) for h in range(c["Hq"])]
+        got = oracle_units(name, units, workers=2, **over)
+        for (b, h), (uo, ul, um) in got.items():
+            assert np.allclose(uo, ref_o[b, h], atol=1e-13, rtol=0), (name, b, h)
+            fin = np.isfinite(ref_l[b, h])
+            assert np.array_equal(np.isfinite(ul), fin)
+            assert np.allclose(ul[fin], ref_l[b, h][fin], atol=1e-13) and np.allclose(um[fin], ref_m[b, h][fin])

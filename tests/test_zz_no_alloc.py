@@ -62,7 +62,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 def test_noalloc_refuses_oversized_scratch():
     import programmable_block_sparse_b200 as fa
-    # 8 x 32 heads x 16 rows x 32 splits x 65 floats = 34 MB: above the 16 MiB scratch
+    # 8 x 32 heads x 16 rows x 32 splits x 66 floats = 34.6 MB: above the 16 MiB scratch
     case = Case(8, 32, 32, 16, 4096, 64, 64, "bf16", {"kind": "causal"}, {"kind": "none"}, seed=3)
     bm = case.block_mask(128, 128)
     with pytest.raises(fa.FlexAttnError) as e:
@@ -71,12 +71,43 @@ def test_noalloc_refuses_oversized_scratch():
 
 
 def test_noalloc_automatic_split_count():
-    """With split_kv = 0 the entry point picks its own split count (capped by
-    what the built-in scratch holds) and matches the workspace entry point on
-    a decode-sized cache: 8 sequences of 4096-32768 keys, 64 query heads over
-    8 KV heads, 16 query rows."""
+    """With split_kv = 0 the entry point takes the split count flexattn_forward
+    would choose when its scratch fits the built-in array, and matches the
+    workspace entry point on a decode-sized cache: 8 sequences of 4096-32768
+    keys, 64 query heads over 8 KV heads, 16 query rows (three splits, 6.5 MB
+    of scratch)."""
     rng = np.random.default_rng(5)
     kv_len = rng.integers(4096, 32769, 8).tolist()
     case = Case(8, 64, 8, 16, 32768, 64, 64, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=9,
                 kv_len=kv_len, sentinel_tail=True)
     _compare(case, split_kv=0)
+
+
+def test_noalloc_falls_back_to_one_split():
+    """B=32, Hq=32, Hkv=8, 16 query rows, head dim 128: the automatic plan
+    (1024 CTAs, two splits) would need 16384 rows x 2 x 130 floats = 17.0 MB
+    of scratch, above the 16 MiB array, and not even two splits fit; the entry
+    point then runs one split, which writes out and lse directly and needs no
+    scratch, and matches flexattn_forward."""
+    import programmable_block_sparse_b200 as fa
+    rng = np.random.default_rng(6)
+    kv_len = rng.integers(64, 700, 32).tolist()
+    case = Case(32, 32, 8, 16, 700, 128, 128, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=10,
+                kv_len=kv_len, sentinel_tail=True)
+    bm = case.block_mask(128, 128)
+    need = fa.flexattn_forward_workspace_size(case.q, case.k, case.v, bm, split_kv=0)
+    assert need > 16 << 20, need
+    ref_out, ref_lse = fa.flexattn_forward(case.q, case.k, case.v, bm, score_mod=case.dev_score,
+                                           mask_mod=case.dev_mask, scale=case.scale32, enable_gqa=True)
+    out = torch.full_like(ref_out, float("nan"))
+    lse = torch.full_like(ref_lse, float("nan"))
+    fa.flexattn_forward_decode_noalloc(case.q, case.k, case.v, bm, score_mod=case.dev_score, mask_mod=case.dev_mask,
+                                       scale=case.scale32, enable_gqa=True, out=out, lse=lse, split_kv=0)
+    torch.cuda.synchronize()
+    assert fa.flexattn_poll_device_status() == 0
+    r = ref_out.float().cpu().numpy().astype(np.float64)
+    g = out.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(g - r) <= bf16_tolerance(r)), np.abs(g - r).max()
+    fin = np.isfinite(ref_lse.cpu().numpy())
+    assert np.array_equal(fin, np.isfinite(lse.cpu().numpy()))
+    assert np.all(np.abs(lse.cpu().numpy()[fin] - ref_lse.cpu().numpy()[fin]) <= 1e-3)
