@@ -57,7 +57,10 @@ import numpy as np
 
 NEG_INF = -np.inf
 
-MASK_KINDS = ("none", "causal", "sliding_window", "document", "prefix_lm", "chunked", "dense")
+MASK_KINDS = ("none", "causal", "sliding_window", "document", "prefix_lm", "chunked", "dense",
+              # predicates and combinators for composed masks
+              "distance_below", "key_below", "same_chunk", "same_document", "stride", "head_below",
+              "and", "or", "not")
 SCORE_KINDS = ("none", "softcap", "alibi", "cap_then_bias")
 
 
@@ -121,10 +124,26 @@ def visible(mask, b, h, qp, kv, S_b):
     * dense -- an explicit (L, S) boolean matrix (oracle-only, for the pages'
       key-padding example).
 
+    Composed masks ("PyTorch Flex Attention complete guide" section 4.3:
+    and_masks / or_masks combine any number of mask rules into one, by
+    intersection or union; "Attention expressions", Examples: every fourth
+    key, half the heads global and half local):
+
+    * and / or -- every / any rule of ``masks`` allows the pair; not -- the
+      rule ``mask`` does not.
+    * distance_below -- q - kv < value (no causal bound of its own).
+    * key_below -- kv < value.
+    * same_chunk -- floor(q / value) == floor(kv / value).
+    * same_document -- doc[q] == doc[kv] (no causal bound of its own).
+    * stride -- q - kv is a multiple of value (q = kv modulo value).
+    * head_below -- h < value (the query head).
+
     Keys at or beyond the valid length S_b are invisible under every kind.
     """
-    qp = np.asarray(qp, dtype=np.int64)[:, None]
-    kv = np.asarray(kv, dtype=np.int64)[None, :]
+    qp1 = np.asarray(qp, dtype=np.int64)
+    kv1 = np.asarray(kv, dtype=np.int64)
+    qp = qp1[:, None]
+    kv = kv1[None, :]
     kind = mask["kind"]
     in_range = kv < S_b
     causal = kv <= qp
@@ -150,6 +169,32 @@ def visible(mask, b, h, qp, kv, S_b):
         m = np.asarray(mask["matrix"], dtype=bool)
         rows = mask.get("rows")
         m = m if rows is None else m[np.asarray(rows)]
+    elif kind == "and":
+        m = np.ones(np.broadcast(qp, kv).shape, dtype=bool)
+        for sub in mask["masks"]:
+            m = m & visible(sub, b, h, qp1, kv1, S_b)
+    elif kind == "or":
+        m = np.zeros(np.broadcast(qp, kv).shape, dtype=bool)
+        for sub in mask["masks"]:
+            m = m | visible(sub, b, h, qp1, kv1, S_b)
+    elif kind == "not":
+        m = ~visible(mask["mask"], b, h, qp1, kv1, S_b)
+    elif kind == "distance_below":
+        m = (qp - kv) < int(mask["value"])
+    elif kind == "key_below":
+        m = kv < int(mask["value"])
+    elif kind == "same_chunk":
+        C = int(mask["value"])
+        m = np.floor_divide(qp, C) == np.floor_divide(kv, C)
+    elif kind == "same_document":
+        doc_b = _row_for_batch(mask["doc_id"], b)
+        qi = np.clip(qp, 0, len(doc_b) - 1)
+        ki = np.clip(kv, 0, len(doc_b) - 1)
+        m = (qp >= 0) & (qp < len(doc_b)) & (doc_b[qi] == doc_b[ki])
+    elif kind == "stride":
+        m = np.mod(qp - kv, int(mask["value"])) == 0
+    elif kind == "head_below":
+        m = np.full(np.broadcast(qp, kv).shape, h < int(mask["value"]))
     else:
         raise ValueError(f"unknown mask kind {kind!r}")
     return np.broadcast_to(m, np.broadcast(qp, kv).shape) & in_range
@@ -351,8 +396,9 @@ def block_mask(mask, B, H, L, S, BM, BN, kv_len=None):
     Returns int32 arrays kv_num_blocks (B,H,Mb), kv_indices (B,H,Mb,Nb) of the
     partial tiles, full_kv_num_blocks (B,H,Mb), full_kv_indices (B,H,Mb,Nb),
     indices ascending, unused slots 0.  Tiles at a ragged edge are classified
-    over their in-range cells only.  The menu's masks do not depend on the
-    head, so every head row is the same.
+    over their in-range cells only.  Row h of the arrays is classified for
+    query head h, so a head-dependent rule (head_below) gets per-head lists
+    when H = Hq.
     """
     Mb, Nb = -(-L // BM), -(-S // BN)
     kv_num = np.zeros((B, H, Mb), np.int32)

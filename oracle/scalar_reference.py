@@ -17,9 +17,38 @@ from __future__ import annotations
 import math
 
 
-def _visible(kind, params, b, q, kv, S_b):
+def _rule(params, b, h, q, kv):
+    """A composed rule's verdict for one (query, key) pair, in-range keys only."""
+    kind = params["kind"]
+    if kind == "and":
+        return all(_rule(m, b, h, q, kv) for m in params["masks"])
+    if kind == "or":
+        return any(_rule(m, b, h, q, kv) for m in params["masks"])
+    if kind == "not":
+        return not _rule(params["mask"], b, h, q, kv)
+    if kind == "distance_below":
+        return q - kv < params["value"]
+    if kind == "key_below":
+        return kv < params["value"]
+    if kind == "same_chunk":
+        return math.floor(q / params["value"]) == math.floor(kv / params["value"])
+    if kind == "same_document":
+        doc = params["doc_id"]
+        row = doc[b] if isinstance(doc[0], (list, tuple)) else doc
+        return 0 <= q < len(row) and row[q] == row[kv]
+    if kind == "stride":
+        return (q - kv) % params["value"] == 0
+    if kind == "head_below":
+        return h < params["value"]
+    return _visible(kind, params, b, q, kv, 1 << 62)
+
+
+def _visible(kind, params, b, q, kv, S_b, h=0):
     if kv >= S_b:
         return False
+    if kind in ("and", "or", "not", "distance_below", "key_below", "same_chunk", "same_document", "stride",
+                "head_below"):
+        return _rule(params, b, h, q, kv)
     if kind == "none":
         return True
     if kind == "causal":
@@ -92,7 +121,7 @@ def forward_scalar(q, k, v, scale, mask, score, kv_len=None, with_max=False):
                     for e in range(len(q[b][h][i])):
                         dot += q[b][h][i][e] * k[b][hk][j][e]
                     g = _g(score["kind"], score, scale * dot, b, h, qpos, j, Hq)
-                    scores.append(g if _visible(mask["kind"], mask, b, qpos, j, S_b) else -math.inf)
+                    scores.append(g if _visible(mask["kind"], mask, b, qpos, j, S_b, h) else -math.inf)
                 m = -math.inf
                 for x in scores:
                     if x > m:
@@ -116,7 +145,7 @@ def forward_scalar(q, k, v, scale, mask, score, kv_len=None, with_max=False):
     return (out, lse, top) if with_max else (out, lse)
 
 
-def tile_classes_scalar(mask, L, S, BM, BN, b=0, kv_len=None):
+def tile_classes_scalar(mask, L, S, BM, BN, b=0, kv_len=None, h=0):
     """Tile classes 'F' / 'P' / '0' by visiting every in-range cell of every tile."""
     S_b = S if kv_len is None else int(kv_len[b])
     grid = []
@@ -126,7 +155,7 @@ def tile_classes_scalar(mask, L, S, BM, BN, b=0, kv_len=None):
             seen_vis = seen_hidden = False
             for i in range(m0, min(L, m0 + BM)):
                 for j in range(n0, min(S, n0 + BN)):
-                    if _visible(mask["kind"], mask, b, i + (S_b - L), j, S_b):
+                    if _visible(mask["kind"], mask, b, i + (S_b - L), j, S_b, h):
                         seen_vis = True
                     else:
                         seen_hidden = True

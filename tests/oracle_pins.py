@@ -526,6 +526,94 @@ def check_forward_unit_matches_forward(o):
             assert np.array_equal(np.isfinite(um), fin) and np.allclose(um[fin], mx[b, h][fin], atol=1e-14)
 
 
+def check_composed_masks(o):
+    """and / or / not over predicates ("PyTorch Flex Attention complete guide"
+    section 4.3; "Attention expressions", Examples).
+
+    Pinned by identities with the fixed rules -- causal AND (distance < W OR
+    key < n) is the sliding window with sinks, causal OR key < P is prefix-LM,
+    causal AND same chunk is chunked attention, causal AND same document is
+    the document rule (the guide's and_masks(causal_mask, sliding_window_mask)
+    example) -- by De Morgan, by closed-form counts of the pages' every-fourth-
+    key and half-heads-global examples, by the block-granularity remark (a
+    sliver of every block leaves no full block), and by the scalar loops.
+    """
+    sr = _scalar()
+    T, W, ns, P, C = 70, 9, 3, 11, 16
+    qp, kv = o.query_positions(T, T), np.arange(T)
+    causal = {"kind": "causal"}
+    doc = np.repeat(np.arange(5), [13, 20, 7, 22, 8])
+    ident = [
+        ({"kind": "and", "masks": [causal, {"kind": "or", "masks": [{"kind": "distance_below", "value": W},
+                                                                    {"kind": "key_below", "value": ns}]}]},
+         {"kind": "sliding_window", "window": W, "n_sink": ns}),
+        ({"kind": "or", "masks": [causal, {"kind": "key_below", "value": P}]}, {"kind": "prefix_lm", "prefix": P}),
+        ({"kind": "and", "masks": [causal, {"kind": "same_chunk", "value": C}]}, {"kind": "chunked", "chunk": C}),
+        ({"kind": "and", "masks": [causal, {"kind": "same_document", "doc_id": doc}]},
+         {"kind": "document", "doc_id": doc}),
+    ]
+    for comp, fixed in ident:
+        for S_b in (T, 51):
+            q2 = o.query_positions(T, S_b)
+            assert np.array_equal(o.visible(comp, 0, 0, q2, kv, S_b), o.visible(fixed, 0, 0, q2, kv, S_b)), fixed
+    # chunks are floor-divided: a row at a negative logical position (more
+    # queries than valid keys) shares no chunk with any key, causal bound or not
+    qneg = o.query_positions(T, 40)
+    same = o.visible({"kind": "same_chunk", "value": C}, 0, 0, qneg, kv, 40)
+    assert not same[qneg < 0].any() and same[qneg >= 0].any(axis=1).all()
+    # De Morgan over in-range keys
+    a, bb = {"kind": "stride", "value": 3}, {"kind": "distance_below", "value": 5}
+    lhs = o.visible({"kind": "not", "mask": {"kind": "and", "masks": [a, bb]}}, 0, 0, qp, kv, 60)
+    rhs = o.visible({"kind": "or", "masks": [{"kind": "not", "mask": a}, {"kind": "not", "mask": bb}]}, 0, 0, qp, kv,
+                    60)
+    assert np.array_equal(lhs, rhs) and not lhs[:, 60:].any()
+    # every fourth key, causal: query q sees floor(q / 4) + 1 keys
+    sliver = {"kind": "and", "masks": [causal, {"kind": "stride", "value": 4}]}
+    vis = o.visible(sliver, 0, 0, qp, kv, T)
+    assert vis.sum(axis=1).tolist() == [q // 4 + 1 for q in range(T)]
+    assert vis[T - 1].nonzero()[0].tolist() == list(range((T - 1) % 4, T, 4))
+    # half the heads global, half local (window W), causal on, H = 6
+    H = 6
+    half = {"kind": "and", "masks": [causal, {"kind": "or", "masks": [{"kind": "head_below", "value": H // 2},
+                                                                      {"kind": "distance_below", "value": W}]}]}
+    for h in range(H):
+        n = int(o.visible(half, 0, h, qp, kv, T).sum())
+        assert n == (T * (T + 1) // 2 if h < H // 2 else W * (W + 1) // 2 + (T - W) * W), (h, n)
+    # block granularity: a sliver of every block leaves no full block
+    t = 8
+    bm = o.block_mask(sliver, 1, 1, 8 * t, 8 * t, t, t)
+    assert int(bm["full_kv_num_blocks"].sum()) == 0 and int(bm["kv_num_blocks"].sum()) == 8 * 9 // 2
+    bmh = o.block_mask(half, 1, H, 8 * t, 8 * t, t, t)
+    assert int(bmh["full_kv_num_blocks"][0, 0].sum()) == 8 * 7 // 2  # global heads: causal tiles
+    assert int(bmh["full_kv_num_blocks"][0, 0].sum() + bmh["kv_num_blocks"][0, 0].sum()) == 36
+    assert int(bmh["full_kv_num_blocks"][0, H - 1].sum() + bmh["kv_num_blocks"][0, H - 1].sum()) == 8 + 7
+    # brute force: oracle forward and tile classes against the scalar loops
+    rules = [sliver, half, ident[0][0],
+             {"kind": "not", "mask": {"kind": "or", "masks": [{"kind": "key_below", "value": 2},
+                                                              {"kind": "stride", "value": 3}]}},
+             {"kind": "and", "masks": [{"kind": "same_document", "doc_id": [[0, 0, 1, 1, 1, 2, 2, 2],
+                                                                            [0, 1, 1, 1, 2, 2, 2, 2]]},
+                                       {"kind": "same_chunk", "value": 3}]}]
+    seed = 900
+    for mask in rules:
+        for (L, S, kv_len) in ((8, 8, None), (3, 8, [8, 6])):
+            seed += 1
+            q, k, v = _tiny_case(seed, L, S, 3, 2, Hq=4, Hkv=2)
+            out, lse = o.forward(q, k, v, 0.7, mask, TINY_SCORES[3], kv_len=kv_len, enable_gqa=True)
+            so, sl = sr.forward_scalar(q.tolist(), k.tolist(), v.tolist(), 0.7, mask, TINY_SCORES[3], kv_len)
+            so, sl = np.array(so), np.array(sl)
+            assert np.allclose(out, so, atol=1e-12, rtol=0), mask
+            fin = np.isfinite(sl)
+            assert np.array_equal(fin, np.isfinite(lse)) and np.allclose(lse[fin], sl[fin], atol=1e-12)
+    doc23 = [0] * 5 + [1] * 9 + [2] * 9
+    tile_rules = rules[:4] + [{"kind": "and", "masks": [{"kind": "same_document", "doc_id": doc23},
+                                                        {"kind": "same_chunk", "value": 3}]}]
+    for mask in tile_rules:
+        bm = o.block_mask(mask, 1, 4, 23, 23, 4, 3)
+        for h in range(4):
+            assert o.block_map(bm, 0, h) == sr.tile_classes_scalar(mask, 23, 23, 4, 3, 0, None, h), (mask, h)
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
@@ -533,6 +621,6 @@ ALL_CHECKS = [
     check_alibi_geometric, check_softcap_limits, check_cap_then_bias_order, check_convex_combination,
     check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
     check_split_combine, check_gqa_is_broadcast, check_sampled_rows_match_forward,
-    check_max_scores, check_forward_unit_matches_forward,
+    check_max_scores, check_forward_unit_matches_forward, check_composed_masks,
 ]
 SLOW_CHECKS = [check_workload_tile_counts]

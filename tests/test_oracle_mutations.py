@@ -22,8 +22,10 @@ MUTATIONS = {
     "window_includes_W_plus_1": ("(qp - kv) < W", "(qp - kv) <= W"),
     "sink_off_by_one": ("(kv < n_sink)", "(kv <= n_sink)"),
     "prefix_off_by_one": ("m = causal | (kv < P)", "m = causal | (kv <= P)"),
-    "chunk_ignored": ("np.floor_divide(qp, C) == np.floor_divide(kv, C)", "np.floor_divide(qp, C) >= np.floor_divide(kv, C)"),
-    "document_ignored": ("(doc_b[qi] == doc_b[ki])", "(doc_b[qi] >= doc_b[ki])"),
+    "chunk_ignored": ("m = causal & (np.floor_divide(qp, C) == np.floor_divide(kv, C))",
+                      "m = causal & (np.floor_divide(qp, C) >= np.floor_divide(kv, C))"),
+    "document_ignored": ("m = causal & (qp >= 0) & (doc_b[qi] == doc_b[ki])",
+                         "m = causal & (qp >= 0) & (doc_b[qi] >= doc_b[ki])"),
     "kv_len_ignored": ("in_range = kv < S_b", "in_range = kv >= 0"),
     "alibi_sign": ("return s - slope * (qp - kv)", "return s + slope * (qp - kv)"),
     "slope_index": ("2.0 ** (-8.0 * (h + 1) / H)", "2.0 ** (-8.0 * h / H)"),
@@ -48,6 +50,14 @@ MUTATIONS = {
     "max_scores_unmasked": ("return out, lse, st.max(axis=1)", "return out, lse, g.max(axis=1)"),
     "max_scores_log2_units": ("return out, lse, st.max(axis=1)", "return out, lse, st.max(axis=1) * 1.4426950408889634"),
     "max_scores_raw_score": ("return out, lse, st.max(axis=1)", "return out, lse, np.where(vis, s, NEG_INF).max(axis=1)"),
+    "or_as_and": ("            m = m | visible(sub, b, h, qp1, kv1, S_b)", "            m = m & visible(sub, b, h, qp1, kv1, S_b)"),
+    "not_ignored": ('m = ~visible(mask["mask"], b, h, qp1, kv1, S_b)', 'm = visible(mask["mask"], b, h, qp1, kv1, S_b)'),
+    "distance_below_inclusive": ('m = (qp - kv) < int(mask["value"])', 'm = (qp - kv) <= int(mask["value"])'),
+    "stride_on_key_only": ('m = np.mod(qp - kv, int(mask["value"])) == 0', 'm = np.mod(kv, int(mask["value"])) == 0'),
+    "head_below_inclusive": ('np.full(np.broadcast(qp, kv).shape, h < int(mask["value"]))',
+                             'np.full(np.broadcast(qp, kv).shape, h <= int(mask["value"]))'),
+    "same_chunk_truncated": ('m = np.floor_divide(qp, C) == np.floor_divide(kv, C)\n    elif kind == "same_document"',
+                             'm = np.trunc(qp / C) == np.trunc(kv / C)\n    elif kind == "same_document"'),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
                            "out[live] = outs[:, live].mean(axis=0)"),
 }
