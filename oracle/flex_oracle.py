@@ -380,6 +380,40 @@ def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=
 
 
 # ---------------------------------------------------------------------------
+# Paged KV cache
+# ---------------------------------------------------------------------------
+
+def gather_pages(pool, page_table, page_size, pages_per_seq):
+    """The logical cache (B, H, pages_per_seq * page_size, D) of a paged pool.
+
+    "flexattention-score-mod-block-mask", "At decode, q_idx = 0 is not
+    position 0": in a paged or circular cache layout the storage position
+    has to be mapped back to the logical position.  Reading taken: the pool
+    is (num_pages, H, page_size, D); logical key j of sequence b lives in
+    physical page page_table[b][j // page_size], slot j % page_size.  Every
+    rule (mask, score, valid length) sees logical positions only.
+    """
+    pool = _as_f64(pool)
+    table = np.asarray(page_table, dtype=np.int64)
+    B = table.shape[0]
+    H, D = pool.shape[1], pool.shape[3]
+    out = np.zeros((B, H, pages_per_seq * page_size, D))
+    for b in range(B):
+        for i in range(pages_per_seq):
+            out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]]
+    return out
+
+
+def forward_paged(q, k_pages, v_pages, page_table, page_size, pages_per_seq, scale=None, mask=None, score=None,
+                  kv_len=None, enable_gqa=False, aux=False):
+    """Forward pass against a paged KV cache: :func:`forward` on the logical
+    cache that :func:`gather_pages` reads out of the page pools."""
+    k = gather_pages(k_pages, page_table, page_size, pages_per_seq)
+    v = gather_pages(v_pages, page_table, page_size, pages_per_seq)
+    return forward(q, k, v, scale, mask, score, kv_len=kv_len, enable_gqa=enable_gqa, aux=aux)
+
+
+# ---------------------------------------------------------------------------
 # BlockMask
 # ---------------------------------------------------------------------------
 

@@ -614,6 +614,73 @@ def check_composed_masks(o):
             assert o.block_map(bm, 0, h) == sr.tile_classes_scalar(mask, 23, 23, 4, 3, 0, None, h), (mask, h)
 
 
+def check_paged_cache(o):
+    """A paged cache gives the dense cache's result; storage order is invisible.
+
+    Pinned by: the page's decode example (capacity 8, valid length 6, window
+    3, the query at position 5 sees keys 3, 4, 5) stored in shuffled pages of
+    2; an identity page table over a contiguous pool, and a shuffled pool
+    with its page table, equal the dense forward; a distance bias reads
+    logical, not storage, positions; a circular layout (a ring of pages under
+    a sliding window) whose stale pages hold garbage equals the dense window.
+    """
+    g = load("m3_decode_offset.txt")
+    cap, valid, W = int(g["capacity"]), int(g["valid_length"]), int(g["window"])
+    P = 2
+    perm = np.array([2, 0, 3, 1])                    # logical page i -> physical page perm[i]
+    pos = np.arange(cap, dtype=np.float64)
+    kd = np.zeros((1, 1, cap, 1))                    # q = 0: every score equal
+    vd = pos.reshape(1, 1, cap, 1)                   # each value its logical position
+    kp = np.zeros((4, 1, P, 1))
+    vp = np.zeros((4, 1, P, 1))
+    for i in range(4):
+        vp[perm[i], 0] = vd[0, 0, i * P:(i + 1) * P]
+    mask = {"kind": "sliding_window", "window": W, "n_sink": 0}
+    out, _ = o.forward_paged(np.zeros((1, 1, 1, 1)), kp, vp, perm[None, :], P, 4, 1.0, mask, None, kv_len=[valid])
+    assert abs(out[0, 0, 0, 0] - np.mean(ints(g["visible"]))) < 1e-13  # the mean of keys 3, 4, 5
+    # dense vs paged, identity and shuffled tables, GQA, per-sequence lengths, ALiBi
+    r = np.random.default_rng(33)
+    B, Hq, Hkv, L, P, npg, E = 3, 4, 2, 4, 4, 6, 5
+    q = r.standard_normal((B, Hq, L, E))
+    kd = r.standard_normal((B, Hkv, P * npg, E))
+    vd = r.standard_normal((B, Hkv, P * npg, 3))
+    kv_len = np.array([24, 17, 5])
+    score = {"kind": "cap_then_bias", "cap": 4.0, "slope_heads": 0, "pos": "global"}
+    ref_o, ref_l = o.forward(q, kd, vd, 0.5, {"kind": "causal"}, score, kv_len=kv_len, enable_gqa=True)
+    for shuffle in (False, True):
+        n_pool = B * npg + 3
+        order = r.permutation(n_pool)[:B * npg] if shuffle else np.arange(B * npg)
+        table = order.reshape(B, npg)
+        kp = r.standard_normal((n_pool, Hkv, P, E)) * 50.0   # unused pages hold large values
+        vp = r.standard_normal((n_pool, Hkv, P, 3)) * 50.0
+        for b in range(B):
+            for i in range(npg):
+                kp[table[b, i]] = kd[b, :, i * P:(i + 1) * P]
+                vp[table[b, i]] = vd[b, :, i * P:(i + 1) * P]
+        po, pl = o.forward_paged(q, kp, vp, table, P, npg, 0.5, {"kind": "causal"}, score, kv_len=kv_len,
+                                 enable_gqa=True)
+        assert np.allclose(po, ref_o, atol=1e-13) and np.allclose(pl, ref_l, atol=1e-13)
+        assert np.allclose(o.gather_pages(kp, table, P, npg), kd, atol=0)
+    # circular layout: a window of W = 8 keys over a ring of 3 pages of 4; the
+    # pages the window has left are reused, so a 20-key logical cache needs
+    # logical page i at physical page i mod 3; stale logical pages map to
+    # whatever the ring holds now and must stay hidden by the window
+    P, ring, n_log, Wn = 4, 3, 5, 8
+    kd = r.standard_normal((1, 1, P * n_log, E))
+    vd = r.standard_normal((1, 1, P * n_log, 3))
+    qd = r.standard_normal((1, 1, 1, E))
+    kp = np.zeros((ring, 1, P, E))
+    vp = np.zeros((ring, 1, P, 3))
+    for i in range(n_log):                            # writes in order: the ring keeps the last 3 pages
+        kp[i % ring] = kd[0, :, i * P:(i + 1) * P]
+        vp[i % ring] = vd[0, :, i * P:(i + 1) * P]
+    table = (np.arange(n_log) % ring)[None, :]
+    win = {"kind": "sliding_window", "window": Wn, "n_sink": 0}
+    po, pl = o.forward_paged(qd, kp, vp, table, P, n_log, 0.4, win, None, kv_len=[P * n_log])
+    ro, rl = o.forward(qd, kd, vd, 0.4, win, None, kv_len=[P * n_log])
+    assert np.allclose(po, ro, atol=1e-13) and np.allclose(pl, rl, atol=1e-13)
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
@@ -622,5 +689,6 @@ ALL_CHECKS = [
     check_against_torch_sdpa, check_against_scalar_loops, check_block_mask_against_scalar,
     check_split_combine, check_gqa_is_broadcast, check_sampled_rows_match_forward,
     check_max_scores, check_forward_unit_matches_forward, check_composed_masks,
+    check_paged_cache,
 ]
 SLOW_CHECKS = [check_workload_tile_counts]

@@ -58,6 +58,10 @@ MUTATIONS = {
                              'np.full(np.broadcast(qp, kv).shape, h <= int(mask["value"]))'),
     "same_chunk_truncated": ('m = np.floor_divide(qp, C) == np.floor_divide(kv, C)\n    elif kind == "same_document"',
                              'm = np.trunc(qp / C) == np.trunc(kv / C)\n    elif kind == "same_document"'),
+    "page_slot_order": ("out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]]",
+                        "out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]][:, ::-1]"),
+    "page_table_ignored": ("out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]]",
+                           "out[b, :, i * page_size:(i + 1) * page_size] = pool[b * pages_per_seq + i]"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
                            "out[live] = outs[:, live].mean(axis=0)"),
 }
