@@ -85,8 +85,40 @@ enum {
                                  [expressions] "Examples": a window that keeps sink tokens)      */
   FA_MASK_DOCUMENT = 3,       /* kv <= q && doc_id[b][q] == doc_id[b][kv]  ([charlestar] "Packing") */
   FA_MASK_PREFIX_LM = 4,      /* kv <= q || kv < prefix   (causal off; [expressions] "Examples")   */
-  FA_MASK_CHUNKED = 5         /* kv <= q && q / chunk == kv / chunk  ([expressions] "Examples")    */
+  FA_MASK_CHUNKED = 5,        /* kv <= q && q / chunk == kv / chunk  ([expressions] "Examples")    */
+  FA_MASK_PROGRAM = 6         /* a composed rule: fa_mask_mod.program (below)                      */
 };
+
+/* Instructions of a composed rule ([guide] 4.3: and_masks / or_masks combine
+ * any number of rules by intersection or union; [expressions] "Examples":
+ * every fourth key, half the heads global and half local), in postfix order:
+ * a predicate pushes its verdict for the pair (q, kv) of query head h,
+ * FA_PROG_AND / FA_PROG_OR pop two verdicts and push one, FA_PROG_NOT
+ * negates the top; one verdict must remain.  No predicate carries a causal
+ * bound of its own (add FA_PROG_CAUSAL), and keys kv >= S_b stay invisible
+ * whatever the program says.  The library rewrites the program as an AND of
+ * at most 8 clauses, each an OR of at most 4 predicates or their negations;
+ * a program that needs more returns FA_ERR_UNSUPPORTED. */
+enum {
+  FA_PROG_TRUE = 0,           /* every pair                                                    */
+  FA_PROG_CAUSAL = 1,         /* kv <= q                                                       */
+  FA_PROG_DISTANCE_BELOW = 2, /* q - kv < arg                                                  */
+  FA_PROG_KEY_BELOW = 3,      /* kv < arg                                                      */
+  FA_PROG_SAME_CHUNK = 4,     /* floor(q / arg) == floor(kv / arg), arg >= 1                   */
+  FA_PROG_SAME_DOCUMENT = 5,  /* 0 <= q < S and doc_id[b][q] == doc_id[b][kv] (doc_id needed)  */
+  FA_PROG_STRIDE = 6,         /* q - kv is a multiple of arg, arg >= 1                         */
+  FA_PROG_HEAD_BELOW = 7,     /* h < arg (h is the query head): a head-dependent rule          */
+  FA_PROG_AND = 16,
+  FA_PROG_OR = 17,
+  FA_PROG_NOT = 18
+};
+
+#define FA_MASK_PROGRAM_MAX 16
+
+typedef struct fa_mask_instr {
+  int32_t op;            /* FA_PROG_*                                                      */
+  int32_t arg;           /* the predicate's parameter (unused by the others)               */
+} fa_mask_instr;
 
 typedef struct fa_mask_mod {
   int32_t kind;          /* FA_MASK_*                                                       */
@@ -98,6 +130,10 @@ typedef struct fa_mask_mod {
   const int32_t* doc_id; /* DOCUMENT: device int32 [doc_batch, S], document id per position  */
   const int32_t* kv_len; /* optional device int32 [B]: valid KV length per sequence, values in
                             [0, S] (clamped to that range); NULL means S for every sequence  */
+  int32_t n_instr;       /* PROGRAM: number of instructions, 1..FA_MASK_PROGRAM_MAX         */
+  int32_t reserved;      /* must be 0                                                       */
+  fa_mask_instr program[FA_MASK_PROGRAM_MAX];  /* PROGRAM: postfix instructions (host memory,
+                            read during the call)                                          */
 } fa_mask_mod;
 
 /* ----------------------------------------------------------------------- */
@@ -138,8 +174,9 @@ typedef struct fa_score_mod {
 /* ----------------------------------------------------------------------- */
 typedef struct fa_block_mask {
   int32_t B;                    /* 1 (broadcast over the batch) or the batch size          */
-  int32_t H;                    /* 1 (broadcast over heads) or Hq; the menu's masks do not
-                                   depend on the head, so every head row is identical      */
+  int32_t H;                    /* 1 (broadcast over heads) or Hq; the fixed rules do not
+                                   depend on the head, so their head rows are identical; a
+                                   program with FA_PROG_HEAD_BELOW needs H == Hq           */
   int32_t L, S;                 /* query and key lengths the mask describes                */
   int32_t BM, BN;               /* query and key tile sizes, 1..128                        */
   int32_t Mb, Nb;               /* ceil(L / BM), ceil(S / BN)                              */
@@ -190,6 +227,23 @@ typedef struct fa_forward_options {
                            copies and MMAs before it exits keep the default budget       */
   int32_t flags;        /* FA_FLAG_*                                                        */
   int32_t reserved;     /* must be 0                                                        */
+  /* Paged KV cache ([charlestar] "At decode, q_idx = 0 is not position 0": a
+   * paged or circular layout maps storage positions back to logical ones).
+   * When page_table != NULL, k and v are page pools of shape
+   * (num_pages, Hkv, page_size, E / Ev) -- any strides, so a pool stored as
+   * (num_pages, page_size, Hkv, E) is passed with its strides -- and logical
+   * key j of sequence b is slot j % page_size of page
+   * page_table[b * pages_per_seq + j / page_size].  The logical length
+   * S = pages_per_seq * page_size is what the block mask, kv_len and every
+   * rule see.  A circular cache is a page table whose entries wrap around a
+   * ring of pages; the caller's mask must hide the stale logical pages.
+   * A page id outside [0, num_pages) is clamped into the pool (nothing
+   * outside it is read), FA_ERR_PARAM is recorded in the device status word
+   * and the outputs are unspecified.                                       */
+  const int32_t* page_table;  /* device int32 [B, pages_per_seq], row-major, or NULL        */
+  int32_t page_size;    /* keys per page: a multiple of 64 on the bf16 tensor-core and split-KV
+                           kernels, any size >= 1 on the general kernel                   */
+  int32_t pages_per_seq;/* columns of page_table                                            */
 } fa_forward_options;
 
 /* ----------------------------------------------------------------------- */
@@ -219,9 +273,11 @@ int flexattn_build_block_mask(const fa_mask_mod* mask_mod, const fa_block_mask* 
 
 /* Bytes of device workspace flexattn_forward needs for these arguments
  * (0 when the chosen kernel needs none).  Same argument checks as
- * flexattn_forward. */
+ * flexattn_forward; options (NULL or those of the forward call) matter for a
+ * paged cache. */
 int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
-                                    const fa_block_mask* block_mask, int32_t split_kv, size_t* bytes);
+                                    const fa_block_mask* block_mask, int32_t split_kv,
+                                    const fa_forward_options* options, size_t* bytes);
 
 /* Forward pass ([charlestar] "What one connection goes through"):
  *   s_ij  = scale * q_i . k_j                        (scale <= 0 or NaN: 1/sqrt(E), [guide] 6.2)

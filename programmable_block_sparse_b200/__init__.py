@@ -10,7 +10,13 @@ Specification dicts (the menu of include/flexattn.h):
 
 * mask_mod: ``{"kind": "none" | "causal" | "sliding_window" | "document" |
   "prefix_lm" | "chunked", "window": W, "n_sink": n, "prefix": P,
-  "chunk": C, "doc_id": int32 tensor (B or 1, S), "kv_len": int32 tensor (B,)}``
+  "chunk": C, "doc_id": int32 tensor (B or 1, S), "kv_len": int32 tensor (B,)}``,
+  or a composed rule: ``{"kind": "and" | "or", "masks": [rule, ...]}``,
+  ``{"kind": "not", "mask": rule}`` over the rules above and the predicates
+  ``{"kind": "distance_below" | "key_below" | "same_chunk" | "stride" |
+  "head_below", "value": v}`` and ``{"kind": "same_document", "doc_id": ...}``
+  (see :func:`and_masks`, :func:`or_masks`, :func:`not_mask`); ``kv_len``
+  goes on the outermost rule.
 * score_mod: ``{"kind": "none" | "softcap" | "alibi" | "cap_then_bias",
   "cap": c, "slope_heads": H, "pos": int32 tensor (B or 1, S) or None}``
 """
@@ -25,7 +31,7 @@ from dataclasses import dataclass
 from . import _abi
 
 __all__ = [
-    "BlockMask", "FlexAttnError", "library_path", "load_library",
+    "BlockMask", "FlexAttnError", "library_path", "load_library", "and_masks", "or_masks", "not_mask",
     "flexattn_version", "flexattn_last_error", "flexattn_block_mask_dims", "flexattn_build_block_mask",
     "flexattn_forward_workspace_size", "flexattn_forward", "flexattn_forward_decode_noalloc",
     "flexattn_poll_device_status",
@@ -98,9 +104,86 @@ def _tensor_struct(t):
     return s
 
 
+def and_masks(*rules, **extra):
+    """A rule that allows a pair when every rule does (the guide's and_masks)."""
+    return {"kind": "and", "masks": list(rules), **extra}
+
+
+def or_masks(*rules, **extra):
+    """A rule that allows a pair when any rule does (the guide's or_masks)."""
+    return {"kind": "or", "masks": list(rules), **extra}
+
+
+def not_mask(rule, **extra):
+    """A rule that allows exactly the pairs ``rule`` hides."""
+    return {"kind": "not", "mask": rule, **extra}
+
+
+def _flatten(spec, out, docs):
+    """Postfix instructions of a rule spec (the fixed rules spelled out)."""
+    P = _abi.PROG_PRED
+    k = spec["kind"]
+    if k in ("and", "or"):
+        subs = spec["masks"]
+        op = _abi.PROG_AND if k == "and" else _abi.PROG_OR
+        if not subs:  # the empty AND holds everywhere, the empty OR nowhere
+            out.append((P["true"], 0))
+            if k == "or":
+                out.append((_abi.PROG_NOT, 0))
+            return
+        _flatten(subs[0], out, docs)
+        for sub in subs[1:]:
+            _flatten(sub, out, docs)
+            out.append((op, 0))
+    elif k == "not":
+        _flatten(spec["mask"], out, docs)
+        out.append((_abi.PROG_NOT, 0))
+    elif k == "none":
+        out.append((P["true"], 0))
+    elif k == "causal":
+        out.append((P["causal"], 0))
+    elif k == "sliding_window":
+        out += [(P["causal"], 0), (P["distance_below"], int(spec["window"])),
+                (P["key_below"], int(spec.get("n_sink", 0))), (_abi.PROG_OR, 0), (_abi.PROG_AND, 0)]
+    elif k == "prefix_lm":
+        out += [(P["causal"], 0), (P["key_below"], int(spec["prefix"])), (_abi.PROG_OR, 0)]
+    elif k == "chunked":
+        out += [(P["causal"], 0), (P["same_chunk"], int(spec["chunk"])), (_abi.PROG_AND, 0)]
+    elif k in ("document", "same_document"):
+        docs.append(spec["doc_id"])
+        if k == "document":
+            out += [(P["causal"], 0), (P["same_document"], 0), (_abi.PROG_AND, 0)]
+        else:
+            out.append((P["same_document"], 0))
+    elif k in P:
+        out.append((P[k], int(spec.get("value", 0))))
+    else:
+        raise FlexAttnError(9, f"unknown mask rule {k!r}")
+
+
 def _mask_struct(spec):
     spec = spec or {"kind": "none"}
     m = _abi.fa_mask_mod()
+    if spec["kind"] not in _abi.MASK_KIND or spec["kind"] == "program":
+        prog, docs = [], []
+        _flatten(spec, prog, docs)
+        if len(prog) > _abi.MASK_PROGRAM_MAX:
+            raise FlexAttnError(11, f"the composed rule needs {len(prog)} instructions "
+                                    f"(at most {_abi.MASK_PROGRAM_MAX})")
+        m.kind = _abi.MASK_KIND["program"]
+        m.n_instr = len(prog)
+        for i, (op, arg) in enumerate(prog):
+            m.program[i].op = op
+            m.program[i].arg = arg
+        if docs:
+            if any(d.data_ptr() != docs[0].data_ptr() for d in docs):
+                raise FlexAttnError(9, "a composed rule reads one doc_id tensor")
+            m.doc_id = docs[0].data_ptr()
+            m.doc_batch = docs[0].shape[0] if docs[0].dim() == 2 else 1
+        kv_len = spec.get("kv_len")
+        if kv_len is not None:
+            m.kv_len = kv_len.data_ptr()
+        return m
     m.kind = _abi.MASK_KIND[spec["kind"]]
     m.window = int(spec.get("window", 0))
     m.n_sink = int(spec.get("n_sink", 0))
@@ -185,28 +268,35 @@ def flexattn_build_block_mask(mask_mod, B, H, L, S, BM=128, BN=128, device="cuda
     return out
 
 
-def flexattn_forward_workspace_size(q, k, v, block_mask, split_kv=0):
+def flexattn_forward_workspace_size(q, k, v, block_mask, split_kv=0, paged=None):
     n = C.c_size_t()
     qs, ks, vs, bm = _tensor_struct(q), _tensor_struct(k), _tensor_struct(v), block_mask.as_struct()
+    opts = _options_struct(None, False, 0, paged)
     _check(load_library().flexattn_forward_workspace_size(C.byref(qs), C.byref(ks), C.byref(vs), C.byref(bm),
-                                                          int(split_kv), C.byref(n)))
+                                                          int(split_kv), None if opts is None else C.byref(opts),
+                                                          C.byref(n)))
     return n.value
 
 
-def _options_struct(max_scores, rows_guaranteed_safe, wait_cycles):
-    if max_scores is None and not rows_guaranteed_safe and not wait_cycles:
+def _options_struct(max_scores, rows_guaranteed_safe, wait_cycles, paged=None):
+    if max_scores is None and not rows_guaranteed_safe and not wait_cycles and paged is None:
         return None
     o = _abi.fa_forward_options()
     o.max_scores = None if max_scores is None else max_scores.data_ptr()
     o.wait_cycles = int(wait_cycles or 0)
     o.flags = _abi.FA_FLAG_ROWS_GUARANTEED_SAFE if rows_guaranteed_safe else 0
     o.reserved = 0
+    if paged is not None:
+        table = paged["page_table"]
+        o.page_table = table.data_ptr()
+        o.page_size = int(paged["page_size"])
+        o.pages_per_seq = int(table.shape[-1])
     return o
 
 
 def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=None, enable_gqa=False,
                      out=None, lse=True, split_kv=0, workspace=None, stream=None, out_dtype=None,
-                     max_scores=None, rows_guaranteed_safe=False, wait_cycles=0):
+                     max_scores=None, rows_guaranteed_safe=False, wait_cycles=0, paged=None):
     """Run the forward pass; returns ``(out, lse)`` (lse None when ``lse=False``),
     or ``(out, lse, max_scores)`` when ``max_scores`` is requested.
 
@@ -217,6 +307,8 @@ def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=N
     needed).  ``max_scores``: True (allocate) or an fp32 (B, Hq, L) tensor for
     the per-row maximum score.  ``rows_guaranteed_safe`` sets
     FA_FLAG_ROWS_GUARANTEED_SAFE; ``wait_cycles`` the device wait budget.
+    ``paged``: ``{"page_table": int32 (B, pages_per_seq), "page_size": P}``
+    when k and v are page pools (num_pages, Hkv, P, D).
     """
     import torch
     B, Hq, L, _ = q.shape
@@ -232,8 +324,8 @@ def flexattn_forward(q, k, v, block_mask, score_mod=None, mask_mod=None, scale=N
         max_scores = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     elif max_scores is False:
         max_scores = None
-    opts = _options_struct(max_scores, rows_guaranteed_safe, wait_cycles)
-    ws_bytes = flexattn_forward_workspace_size(q, k, v, block_mask, split_kv)
+    opts = _options_struct(max_scores, rows_guaranteed_safe, wait_cycles, paged)
+    ws_bytes = flexattn_forward_workspace_size(q, k, v, block_mask, split_kv, paged)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     qs, ks, vs, os_ = _tensor_struct(q), _tensor_struct(k), _tensor_struct(v), _tensor_struct(out)

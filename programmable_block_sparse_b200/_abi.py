@@ -17,14 +17,26 @@ FA_DTYPE_F32 = 1
 
 FA_FLAG_ROWS_GUARANTEED_SAFE = 1
 
-MASK_KIND = {"none": 0, "causal": 1, "sliding_window": 2, "document": 3, "prefix_lm": 4, "chunked": 5}
+MASK_KIND = {"none": 0, "causal": 1, "sliding_window": 2, "document": 3, "prefix_lm": 4, "chunked": 5,
+             "program": 6}
+
+# instructions of a composed rule (FA_PROG_*)
+PROG_PRED = {"true": 0, "causal": 1, "distance_below": 2, "key_below": 3, "same_chunk": 4, "same_document": 5,
+             "stride": 6, "head_below": 7}
+PROG_AND, PROG_OR, PROG_NOT = 16, 17, 18
+MASK_PROGRAM_MAX = 16
 SCORE_KIND = {"none": 0, "softcap": 1, "alibi": 2, "cap_then_bias": 3}
+
+
+class fa_mask_instr(C.Structure):
+    _fields_ = [("op", C.c_int32), ("arg", C.c_int32)]
 
 
 class fa_mask_mod(C.Structure):
     _fields_ = [
         ("kind", C.c_int32), ("window", C.c_int32), ("n_sink", C.c_int32), ("prefix", C.c_int32),
         ("chunk", C.c_int32), ("doc_batch", C.c_int32), ("doc_id", C.c_void_p), ("kv_len", C.c_void_p),
+        ("n_instr", C.c_int32), ("reserved", C.c_int32), ("program", fa_mask_instr * MASK_PROGRAM_MAX),
     ]
 
 
@@ -54,6 +66,7 @@ class fa_tensor(C.Structure):
 class fa_forward_options(C.Structure):
     _fields_ = [
         ("max_scores", C.c_void_p), ("wait_cycles", C.c_int64), ("flags", C.c_int32), ("reserved", C.c_int32),
+        ("page_table", C.c_void_p), ("page_size", C.c_int32), ("pages_per_seq", C.c_int32),
     ]
 
 
@@ -66,7 +79,7 @@ PROTOTYPES = [
     ("flexattn_build_block_mask", C.c_int, [C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask), C.c_void_p]),
     ("flexattn_forward_workspace_size", C.c_int,
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_block_mask), C.c_int32,
-      C.POINTER(C.c_size_t)]),
+      C.POINTER(fa_forward_options), C.POINTER(C.c_size_t)]),
     ("flexattn_forward", C.c_int,
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
       C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),

@@ -6,6 +6,7 @@
 
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.h"
@@ -91,8 +92,160 @@ int cuda_fail(cudaError_t e, const char* what) {
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // ----------------------------------------------------------------------------
+// Composed rules: a postfix program of predicates and AND / OR / NOT,
+// rewritten as an AND of clauses, each an OR of (possibly negated)
+// predicates, which the kernels evaluate with fixed, unrolled loops.
+// ----------------------------------------------------------------------------
+struct ProgNode {
+  int op, arg, a, b;  // a, b: operand nodes (-1 when absent)
+};
+struct ProgLit {
+  int op, arg;
+  bool neg;
+  bool operator==(const ProgLit& o) const { return op == o.op && arg == o.arg && neg == o.neg; }
+};
+using ProgClause = std::vector<ProgLit>;
+using ProgCnf = std::vector<ProgClause>;
+constexpr size_t kCnfWork = 256;  // bound on intermediate clause counts
+
+bool prog_is_pred(int op) { return op >= FA_PROG_TRUE && op <= FA_PROG_HEAD_BELOW; }
+
+// Postfix -> tree; false when the stack discipline is broken.
+bool prog_tree(const fa_mask_mod* m, std::vector<ProgNode>* t, int* root) {
+  std::vector<int> st;
+  for (int i = 0; i < m->n_instr; ++i) {
+    const fa_mask_instr& in = m->program[i];
+    if (prog_is_pred(in.op)) {
+      t->push_back({in.op, in.arg, -1, -1});
+    } else if (in.op == FA_PROG_NOT) {
+      if (st.empty()) return false;
+      t->push_back({in.op, 0, st.back(), -1});
+      st.pop_back();
+    } else {  // AND / OR (checked by the caller)
+      if (st.size() < 2) return false;
+      const int b = st.back();
+      st.pop_back();
+      const int a = st.back();
+      st.pop_back();
+      t->push_back({in.op, 0, a, b});
+    }
+    st.push_back(static_cast<int>(t->size()) - 1);
+  }
+  if (st.size() != 1) return false;
+  *root = st[0];
+  return true;
+}
+
+// Negations pushed to the predicates (De Morgan), then AND distributed over
+// OR; false when the clause count would exceed kCnfWork.
+bool prog_cnf(const std::vector<ProgNode>& t, int i, bool neg, ProgCnf* out) {
+  const ProgNode& n = t[i];
+  if (prog_is_pred(n.op)) {
+    *out = ProgCnf{ProgClause{ProgLit{n.op, n.arg, neg}}};
+    return true;
+  }
+  if (n.op == FA_PROG_NOT) return prog_cnf(t, n.a, !neg, out);
+  ProgCnf x, y;
+  if (!prog_cnf(t, n.a, neg, &x) || !prog_cnf(t, n.b, neg, &y)) return false;
+  if ((n.op == FA_PROG_AND) != neg) {  // a conjunction
+    x.insert(x.end(), y.begin(), y.end());
+    *out = std::move(x);
+  } else {  // a disjunction: every clause of x OR every clause of y
+    ProgCnf r;
+    for (const ProgClause& cx : x)
+      for (const ProgClause& cy : y) {
+        ProgClause c = cx;
+        c.insert(c.end(), cy.begin(), cy.end());
+        r.push_back(std::move(c));
+        if (r.size() > kCnfWork) return false;
+      }
+    *out = std::move(r);
+  }
+  return out->size() <= kCnfWork;
+}
+
+// The composed rule of *m as device clauses; FA_ERR_UNSUPPORTED when it needs
+// more than kMaxClauses clauses or kMaxLits predicates in a clause.
+int prog_compile(const fa_mask_mod* m, MaskParams* p) {
+  std::vector<ProgNode> tree;
+  int root = -1;
+  if (!prog_tree(m, &tree, &root)) return FA_ERR_PARAM;
+  ProgCnf cnf;
+  if (!prog_cnf(tree, root, false, &cnf))
+    return fail(FA_ERR_UNSUPPORTED, "the composed mask rule expands to too many clauses");
+  ProgCnf kept;
+  bool never = false;
+  for (const ProgClause& c : cnf) {
+    ProgClause d;
+    bool always = false;
+    for (const ProgLit& l : c) {
+      if (l.op == FA_PROG_TRUE) {
+        if (!l.neg) always = true;  // the clause holds everywhere
+        continue;                   // a false literal adds nothing to an OR
+      }
+      bool dup = false;
+      for (const ProgLit& e : d) dup = dup || e == l;
+      if (!dup) d.push_back(l);
+    }
+    if (always) continue;
+    if (d.empty()) never = true;  // a clause that holds nowhere: the rule holds nowhere
+    kept.push_back(d);
+  }
+  if (never) kept = ProgCnf{ProgClause{ProgLit{FA_PROG_TRUE, 0, true}}};
+  if (kept.size() > static_cast<size_t>(kMaxClauses))
+    return fail(FA_ERR_UNSUPPORTED, "the composed mask rule needs %zu clauses (at most %d)", kept.size(), kMaxClauses);
+  p->n_clauses = static_cast<int>(kept.size());
+  for (size_t c = 0; c < kept.size(); ++c) {
+    if (kept[c].size() > static_cast<size_t>(kMaxLits))
+      return fail(FA_ERR_UNSUPPORTED, "a clause of the composed mask rule has %zu predicates (at most %d)",
+                  kept[c].size(), kMaxLits);
+    p->clause_len[c] = static_cast<int>(kept[c].size());
+    for (size_t l = 0; l < kept[c].size(); ++l) {
+      const ProgLit& x = kept[c][l];
+      MaskLit& lt = p->lit[c][l];
+      lt.op = x.op | (x.neg ? kLitNeg : 0);
+      lt.arg = x.arg;
+      lt.pat = 0u;
+      if (x.op == FA_PROG_STRIDE && x.arg < 32)
+        for (int k = 0; k < 32; k += x.arg) lt.pat |= 1u << k;
+      p->reads_head |= x.op == FA_PROG_HEAD_BELOW;
+      p->reads_doc |= x.op == FA_PROG_SAME_DOCUMENT;
+    }
+  }
+  return FA_OK;
+}
+
+// ----------------------------------------------------------------------------
 // Parameter checks shared by the build and forward calls.
 // ----------------------------------------------------------------------------
+int check_program(const fa_mask_mod* m, int batch) {
+  if (m->n_instr < 1 || m->n_instr > FA_MASK_PROGRAM_MAX)
+    return fail(FA_ERR_PARAM, "a composed mask rule needs 1..%d instructions (got %d)", FA_MASK_PROGRAM_MAX,
+                m->n_instr);
+  if (m->reserved != 0) return fail(FA_ERR_PARAM, "mask_mod: reserved field must be 0");
+  bool doc = false;
+  for (int i = 0; i < m->n_instr; ++i) {
+    const fa_mask_instr& in = m->program[i];
+    const bool known = prog_is_pred(in.op) || in.op == FA_PROG_AND || in.op == FA_PROG_OR || in.op == FA_PROG_NOT;
+    if (!known) return fail(FA_ERR_PARAM, "composed mask rule: unknown instruction %d at %d", in.op, i);
+    if (in.arg < -(1 << 30) || in.arg > (1 << 30))
+      return fail(FA_ERR_PARAM, "composed mask rule: argument %d at %d is outside [-2^30, 2^30]", in.arg, i);
+    if ((in.op == FA_PROG_SAME_CHUNK || in.op == FA_PROG_STRIDE) && in.arg < 1)
+      return fail(FA_ERR_PARAM, "composed mask rule: chunk and stride need an argument >= 1 (got %d at %d)", in.arg, i);
+    doc = doc || in.op == FA_PROG_SAME_DOCUMENT;
+  }
+  std::vector<ProgNode> tree;
+  int root = -1;
+  if (!prog_tree(m, &tree, &root))
+    return fail(FA_ERR_PARAM, "composed mask rule: the postfix program does not leave exactly one verdict");
+  if (doc) {
+    if (m->doc_id == nullptr) return fail(FA_ERR_PARAM, "a same-document predicate needs doc_id");
+    if (m->doc_batch != 1 && m->doc_batch != batch)
+      return fail(FA_ERR_BATCH, "doc_batch must be 1 or %d (got %d)", batch, m->doc_batch);
+  }
+  return FA_OK;
+}
+
 int check_mask_params(const fa_mask_mod* m, int batch) {
   switch (m->kind) {
     case FA_MASK_NONE:
@@ -113,6 +266,8 @@ int check_mask_params(const fa_mask_mod* m, int batch) {
     case FA_MASK_CHUNKED:
       if (m->chunk < 1) return fail(FA_ERR_PARAM, "chunked mask needs chunk >= 1 (got %d)", m->chunk);
       break;
+    case FA_MASK_PROGRAM:
+      return check_program(m, batch);
     default:
       return fail(FA_ERR_PARAM, "unknown mask kind %d", m->kind);
   }
@@ -151,8 +306,9 @@ int check_block_mask_dims(const fa_block_mask* bm) {
   return FA_OK;
 }
 
-MaskParams to_device(const fa_mask_mod* m) {
-  MaskParams p;
+// The mask parameters as the kernels read them (after check_mask_params).
+int mask_to_device(const fa_mask_mod* m, MaskParams* out) {
+  MaskParams p{};
   p.kind = m->kind;
   p.window = m->window;
   p.n_sink = m->n_sink;
@@ -161,7 +317,12 @@ MaskParams to_device(const fa_mask_mod* m) {
   p.doc_batch = m->doc_batch;
   p.doc_id = m->doc_id;
   p.kv_len = m->kv_len;
-  return p;
+  if (m->kind == FA_MASK_PROGRAM) {
+    const int rc = prog_compile(m, &p);
+    if (rc) return rc;
+  }
+  *out = p;
+  return FA_OK;
 }
 
 ScoreParams to_device(const fa_score_mod* s) {
@@ -264,7 +425,7 @@ int apply_options(const fa_forward_options* o, FwdArgs* a) {
 
 int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out, float scale,
             int32_t enable_gqa, const fa_score_mod* score, const fa_mask_mod* mask, const fa_block_mask* bm,
-            int32_t split_kv, FwdArgs* a, Path* path) {
+            int32_t split_kv, const fa_forward_options* opt, FwdArgs* a, Path* path) {
   int rc;
   if ((rc = check_tensor(q, "q")) || (rc = check_tensor(k, "k")) || (rc = check_tensor(v, "v"))) return rc;
   if (out != nullptr && (rc = check_tensor(out, "out"))) return rc;
@@ -273,12 +434,26 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   if (out && out->dtype != q->dtype && out->dtype != FA_DTYPE_F32)
     return fail(FA_ERR_DTYPE, "out must have the dtype of q, or be fp32");
   const int B = (int)q->size[0], Hq = (int)q->size[1], L = (int)q->size[2], E = (int)q->size[3];
-  const int Hkv = (int)k->size[1], S = (int)k->size[2], Ev = (int)v->size[3];
-  if (k->size[0] != B || v->size[0] != B) return fail(FA_ERR_BATCH, "q, k and v must have the same batch size");
+  const int Hkv = (int)k->size[1], Ev = (int)v->size[3];
+  const bool paged = opt != nullptr && opt->page_table != nullptr;
+  int S = (int)k->size[2];
+  if (paged) {
+    // k and v are page pools (num_pages, Hkv, page_size, E); S is the logical length
+    if (opt->page_size < 1 || opt->pages_per_seq < 1)
+      return fail(FA_ERR_PARAM, "paged cache: page_size and pages_per_seq must be >= 1 (got %d, %d)", opt->page_size,
+                  opt->pages_per_seq);
+    if (static_cast<int64_t>(opt->page_size) * opt->pages_per_seq > INT32_MAX / 2)
+      return fail(FA_ERR_SHAPE, "paged cache: logical length page_size * pages_per_seq is too large");
+    if (k->size[2] != opt->page_size || v->size[2] != opt->page_size || v->size[0] != k->size[0])
+      return fail(FA_ERR_SHAPE, "paged cache: k and v must be pools of (num_pages, Hkv, page_size, dim)");
+    S = opt->page_size * opt->pages_per_seq;
+  } else if (k->size[0] != B || v->size[0] != B) {
+    return fail(FA_ERR_BATCH, "q, k and v must have the same batch size");
+  }
   // launch grids carry the batch and the head count in their y / z extents
   if (B > 65535 || Hq > 65535) return fail(FA_ERR_SHAPE, "batch and head counts above 65535 are not supported");
   if (k->size[3] != E) return fail(FA_ERR_SHAPE, "k head dim %lld != q head dim %d", (long long)k->size[3], E);
-  if (v->size[1] != Hkv || v->size[2] != S) return fail(FA_ERR_SHAPE, "v must be (B, Hkv, S, Ev) like k");
+  if (v->size[1] != Hkv || v->size[2] != k->size[2]) return fail(FA_ERR_SHAPE, "v must be (B, Hkv, S, Ev) like k");
   if (out && (out->size[0] != B || out->size[1] != Hq || out->size[2] != L || out->size[3] != Ev))
     return fail(FA_ERR_SHAPE, "out must be (B, Hq, L, Ev)");
   if (Hq != Hkv) {
@@ -319,17 +494,29 @@ int prepare(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa
   a->out_f32 = out != nullptr && out->dtype == FA_DTYPE_F32;
   a->wait_cycles = kWaitCycles;
   a->scale = (scale > 0.0f && !isinf(scale)) ? scale : 1.0f / sqrtf(static_cast<float>(E));
-  a->mask = to_device(mask);
+  if (paged) {
+    a->page_table = opt->page_table;
+    a->page_size = opt->page_size;
+    a->pages_per_seq = opt->pages_per_seq;
+    a->num_pages = static_cast<int>(k->size[0]);
+  }
+  if ((rc = mask_to_device(mask, &a->mask))) return rc;
+  if (a->mask.reads_head && bm->H != Hq && Hq > 1)
+    return fail(FA_ERR_MASK_SHAPE, "a rule that reads the query head needs a per-head block mask (H = %d, got %d)", Hq,
+                bm->H);
   a->score = to_device(score);
   a->bm = BlockMaskView{bm->B, bm->H, bm->Mb, bm->Nb, bm->BM, bm->BN, bm->kv_num_blocks, bm->kv_indices,
                         bm->full_kv_num_blocks, bm->full_kv_indices};
 
-  const bool tc_shape = q->dtype == FA_DTYPE_BF16 && E == Ev && (E == 64 || E == 128);
+  // the tensor-core kernels read a paged pool in 64-key boxes
+  const bool tc_shape = q->dtype == FA_DTYPE_BF16 && E == Ev && (E == 64 || E == 128) &&
+                        (!paged || opt->page_size % 64 == 0);
   const bool tma_ok = aligned16(q) && aligned16(k) && aligned16(v);
   if (split_kv < 0) return fail(FA_ERR_PARAM, "split_kv must be >= 0");
   if (split_kv > 1 && !(tc_shape && L <= kDecodeMaxRows && bm->Mb == 1 && bm->BN % 64 == 0))
     return fail(FA_ERR_UNSUPPORTED,
-                "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16, one query tile and BN in {64, 128}");
+                "split_kv > 1 needs bf16, E == Ev in {64,128}, L <= 16, one query tile, BN in {64, 128} and, for "
+                "a paged cache, pages of a multiple of 64 keys");
   if (split_kv > 1 && !tma_ok) return fail(FA_ERR_ALIGN, "split_kv > 1 needs 16-byte aligned q, k, v and strides");
   const bool out_ok = out == nullptr || aligned16(out);
   const bool decode_ok = tc_shape && tma_ok && L <= kDecodeMaxRows && bm->Mb == 1 && bm->BN % 64 == 0;
@@ -372,7 +559,7 @@ int flexattn_build_block_mask(const fa_mask_mod* mask_mod, const fa_block_mask* 
   int serr = 0;
   a.status = status_word(&serr);
   if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
-  a.mask = to_device(mask_mod);
+  if ((rc = mask_to_device(mask_mod, &a.mask))) return rc;
   a.B = bm->B;
   a.H = bm->H;
   a.L = bm->L;
@@ -391,13 +578,15 @@ int flexattn_build_block_mask(const fa_mask_mod* mask_mod, const fa_block_mask* 
 }
 
 int flexattn_forward_workspace_size(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
-                                    const fa_block_mask* block_mask, int32_t split_kv, size_t* bytes) {
+                                    const fa_block_mask* block_mask, int32_t split_kv,
+                                    const fa_forward_options* options, size_t* bytes) {
   if (!bytes) return fail(FA_ERR_NULL, "bytes must not be NULL");
   fa_score_mod none_score{FA_SCORE_NONE, 0.0f, 0, 0, nullptr};
-  fa_mask_mod none_mask{FA_MASK_NONE, 0, 0, 0, 0, 0, nullptr, nullptr};
+  fa_mask_mod none_mask{};
+  none_mask.kind = FA_MASK_NONE;
   FwdArgs a;
   Path path;
-  int rc = prepare(q, k, v, nullptr, 0.0f, 1, &none_score, &none_mask, block_mask, split_kv, &a, &path);
+  int rc = prepare(q, k, v, nullptr, 0.0f, 1, &none_score, &none_mask, block_mask, split_kv, options, &a, &path);
   if (rc) return rc;
   *bytes = 0;
   if (path == Path::kDecode) {
@@ -415,7 +604,7 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
   if (!out) return fail(FA_ERR_NULL, "out is NULL");
   FwdArgs a;
   Path path;
-  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
+  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, options, &a, &path);
   if (rc) return rc;
   if ((rc = apply_options(options, &a))) return rc;
   int serr = 0;
@@ -426,8 +615,9 @@ int flexattn_forward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v,
   cudaError_t e;
   if (path == Path::kSm100) {
     Sm100Maps maps;
-    if ((rc = encode_bf16_map(&maps.q, q, 128)) || (rc = encode_bf16_map(&maps.k, k, 128)) ||
-        (rc = encode_bf16_map(&maps.v, v, 128)))
+    const int kv_box = a.page_table ? 64 : 128;  // a paged pool is read in 64-key boxes
+    if ((rc = encode_bf16_map(&maps.q, q, 128)) || (rc = encode_bf16_map(&maps.k, k, kv_box)) ||
+        (rc = encode_bf16_map(&maps.v, v, kv_box)))
       return rc;
     e = launch_fwd_sm100(a, maps, st);
   } else if (path == Path::kDecode) {
@@ -455,7 +645,7 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
   if (!out) return fail(FA_ERR_NULL, "out is NULL");
   FwdArgs a;
   Path path;
-  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, &a, &path);
+  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, split_kv, nullptr, &a, &path);
   if (rc) return rc;
   if ((rc = apply_options(nullptr, &a))) return rc;
   if (path != Path::kDecode)

@@ -14,7 +14,10 @@
 // of at most two key intervals, so a tile is classified from per-row
 // intersection counts (BM work per tile instead of BM x BN).  The document
 // rule counts the same way over runs of equal document id (see
-// classify_tile_document).
+// classify_tile_document).  A composed rule (FA_MASK_PROGRAM) is decided per
+// tile by three-valued logic over the tile's bounds, exact where it says all
+// or nothing, and otherwise by evaluating the tile's cells 32 keys at a time;
+// when it reads the query head, every head row is classified for its head.
 #include "common.cuh"
 #include "launch.h"
 #include "mods.cuh"
@@ -111,6 +114,48 @@ __device__ uint8_t classify_tile_document(const MaskParams& m, int b, int r0, in
   return all_full ? kFull : (any_vis ? kPartial : kEmpty);
 }
 
+// Composed rule: rows [r0, r1] x keys [c0, c1] (inclusive, in range) of head
+// h.  Keys >= S_b are invisible; the caller has handled c0 >= S_b.
+__device__ uint8_t classify_tile_program(const MaskParams& m, int b, int h, int r0, int r1, int c0, int c1, int L,
+                                         int S, int S_b, int* doc_keys) {
+  const int lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  const int chi = min(c1, S_b - 1);  // last key that can be visible
+  const int v = program_box(m, h, query_pos(r0, L, S_b), query_pos(r1, L, S_b), c0, chi);
+  if (v == 0) return kEmpty;
+  if (v == 1) return chi == c1 ? kFull : kPartial;
+  // mixed or undecided: count visible keys row by row, 32 keys per word
+  const int* d = m.reads_doc ? m.doc_id + static_cast<int64_t>(m.doc_batch > 1 ? b : 0) * S : nullptr;
+  if (d) {
+    for (int c = c0 + lane; c <= c1; c += 32) doc_keys[c - c0] = __ldg(d + c);
+    __syncwarp();
+  }
+  const int width = c1 - c0 + 1;
+  bool all_full = true, any_vis = false;
+  for (int r = r0 + lane; r <= r1; r += 32) {
+    const int q = query_pos(r, L, S_b);
+    const int dq = (d && q >= 0 && q < S) ? __ldg(d + q) : 0;
+    int cnt = 0;
+    for (int base = c0; base <= c1; base += 32) {
+      uint32_t same = 0xFFFFFFFFu;
+      if (d) {
+        same = 0u;
+        const int nk = min(32, c1 - base + 1);
+        for (int i = 0; i < nk; ++i) same |= (doc_keys[base - c0 + i] == dq ? 1u : 0u) << i;
+        if (q < 0 || q >= S) same = 0u;
+      }
+      const uint32_t bits = program_bits(m, h, q, base, same) & span_bits(-1, chi - base) & span_bits(-1, c1 - base);
+      cnt += __popc(bits);
+    }
+    all_full &= (cnt == width);
+    any_vis |= (cnt > 0);
+  }
+  all_full = __all_sync(full, all_full);
+  any_vis = __any_sync(full, any_vis);
+  __syncwarp();  // doc_keys is rewritten for the warp's next tile
+  return all_full ? kFull : (any_vis ? kPartial : kEmpty);
+}
+
 __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs a) {
   extern __shared__ uint8_t cls[];
   __shared__ int s_run_a[kClassifyThreads / 32][129];
@@ -126,57 +171,66 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs
   const bool causal_family = a.mask.kind == FA_MASK_CAUSAL || a.mask.kind == FA_MASK_SLIDING_WINDOW ||
                              a.mask.kind == FA_MASK_DOCUMENT || a.mask.kind == FA_MASK_CHUNKED;
 
-  for (int n = warp; n < a.Nb; n += nwarps) {
-    const int c0 = n * a.BN;
-    const int c1 = min(a.S, c0 + a.BN) - 1;        // inclusive
-    uint8_t k;
-    if (c0 >= S_b || (causal_family && c0 > q_hi)) {
-      k = kEmpty;
-    } else if (a.mask.kind == FA_MASK_DOCUMENT) {
-      k = classify_tile_document(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b, s_run_a[warp], s_run_id[warp]);
-    } else {
-      k = classify_tile_intervals(a.mask, r0, r1, c0, c1, a.L, S_b);
-    }
-    if (lane == 0) cls[n] = k;
-  }
-  __syncthreads();
-
-  // Ordered lists: warp 0 scans the classes 32 tiles at a time.
+  // a rule that reads the query head is classified for each head row; any
+  // other is classified once and its lists written to every head row
+  const bool per_head = a.mask.kind == FA_MASK_PROGRAM && a.mask.reads_head && a.H > 1;
   __shared__ int s_counts[2];
-  if (warp == 0) {
-    int nfull = 0, npart = 0;
-    for (int base = 0; base < a.Nb; base += 32) {
-      const int n = base + lane;
-      const uint8_t k = n < a.Nb ? cls[n] : kEmpty;
-      const unsigned fb = __ballot_sync(0xffffffffu, k == kFull);
-      const unsigned pb = __ballot_sync(0xffffffffu, k == kPartial);
-      const unsigned below = (1u << lane) - 1u;
-      for (int h = 0; h < a.H; ++h) {
-        const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
-        if (k == kFull) a.full_kv_indices[row * a.Nb + nfull + __popc(fb & below)] = n;
-        if (k == kPartial) a.kv_indices[row * a.Nb + npart + __popc(pb & below)] = n;
+  for (int hc = 0; hc < (per_head ? a.H : 1); ++hc) {
+    for (int n = warp; n < a.Nb; n += nwarps) {
+      const int c0 = n * a.BN;
+      const int c1 = min(a.S, c0 + a.BN) - 1;        // inclusive
+      uint8_t k;
+      if (c0 >= S_b || (causal_family && c0 > q_hi)) {
+        k = kEmpty;
+      } else if (a.mask.kind == FA_MASK_DOCUMENT) {
+        k = classify_tile_document(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b, s_run_a[warp], s_run_id[warp]);
+      } else if (a.mask.kind == FA_MASK_PROGRAM) {
+        k = classify_tile_program(a.mask, b, hc, r0, r1, c0, c1, a.L, a.S, S_b, s_run_id[warp]);
+      } else {
+        k = classify_tile_intervals(a.mask, r0, r1, c0, c1, a.L, S_b);
       }
-      nfull += __popc(fb);
-      npart += __popc(pb);
+      if (lane == 0) cls[n] = k;
     }
-    if (lane == 0) {
-      s_counts[0] = nfull;
-      s_counts[1] = npart;
-      for (int h = 0; h < a.H; ++h) {
-        const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
-        a.full_kv_num_blocks[row] = nfull;
-        a.kv_num_blocks[row] = npart;
+    __syncthreads();
+
+    // Ordered lists: warp 0 scans the classes 32 tiles at a time.
+    const int h_lo = per_head ? hc : 0, h_hi = per_head ? hc + 1 : a.H;
+    if (warp == 0) {
+      int nfull = 0, npart = 0;
+      for (int base = 0; base < a.Nb; base += 32) {
+        const int n = base + lane;
+        const uint8_t k = n < a.Nb ? cls[n] : kEmpty;
+        const unsigned fb = __ballot_sync(0xffffffffu, k == kFull);
+        const unsigned pb = __ballot_sync(0xffffffffu, k == kPartial);
+        const unsigned below = (1u << lane) - 1u;
+        for (int h = h_lo; h < h_hi; ++h) {
+          const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+          if (k == kFull) a.full_kv_indices[row * a.Nb + nfull + __popc(fb & below)] = n;
+          if (k == kPartial) a.kv_indices[row * a.Nb + npart + __popc(pb & below)] = n;
+        }
+        nfull += __popc(fb);
+        npart += __popc(pb);
+      }
+      if (lane == 0) {
+        s_counts[0] = nfull;
+        s_counts[1] = npart;
+        for (int h = h_lo; h < h_hi; ++h) {
+          const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+          a.full_kv_num_blocks[row] = nfull;
+          a.kv_num_blocks[row] = npart;
+        }
       }
     }
-  }
-  __syncthreads();
-  const int nfull = s_counts[0], npart = s_counts[1];
-  for (int h = 0; h < a.H; ++h) {
-    const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
-    for (int i = threadIdx.x; i < a.Nb; i += blockDim.x) {
-      if (i >= nfull) a.full_kv_indices[row * a.Nb + i] = 0;
-      if (i >= npart) a.kv_indices[row * a.Nb + i] = 0;
+    __syncthreads();
+    const int nfull = s_counts[0], npart = s_counts[1];
+    for (int h = h_lo; h < h_hi; ++h) {
+      const int64_t row = (static_cast<int64_t>(b) * a.H + h) * a.Mb + mt;
+      for (int i = threadIdx.x; i < a.Nb; i += blockDim.x) {
+        if (i >= nfull) a.full_kv_indices[row * a.Nb + i] = 0;
+        if (i >= npart) a.kv_indices[row * a.Nb + i] = 0;
+      }
     }
+    __syncthreads();  // cls and s_counts are rewritten for the next head
   }
 }
 

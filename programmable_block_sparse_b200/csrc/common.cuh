@@ -18,6 +18,21 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Physical page of logical key kv of sequence b in a paged cache (see
+// FwdArgs): the table entry of the key's logical page, the logical page
+// clamped to the table's row and the id clamped into the pool; an id outside
+// the pool records FA_ERR_PARAM.
+__device__ __forceinline__ int cache_page(const int* table, int pages_per_seq, int page_size, int num_pages,
+                                          int* status, int b, int kv) {
+  const int lp = min(kv / page_size, pages_per_seq - 1);
+  int pg = __ldg(table + static_cast<int64_t>(b) * pages_per_seq + lp);
+  if (pg < 0 || pg >= num_pages) {
+    record_error(status, FA_ERR_PARAM);
+    pg = pg < 0 ? 0 : num_pages - 1;
+  }
+  return pg;
+}
+
 // A wait gives up after this many clock64 cycles (about 2 s at 1.9 GHz).
 constexpr long long kWaitCycles = 4000000000ll;
 
@@ -65,12 +80,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // (after `budget` clock64 cycles) it records FA_ERR_TIMEOUT, sets *abort
 // (CTA-shared) and returns false; once *abort is set by any thread of the
 // CTA, other waits give up at once.
+// A budget below the default polls with the non-blocking test (try_wait may
+// suspend inside the hardware for longer than a short budget).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
                                           long long budget = kWaitCycles) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool poll = budget < kWaitCycles;
+  if (poll ? mbar_test(bar, parity) : mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll ? mbar_test(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > budget) {
       record_error(status, FA_ERR_TIMEOUT);

@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   const int b = blockIdx.z;
   const int S_b = seq_len_b(a.mask, b, a.S);
   const int bmb = a.bm.B > 1 ? b : 0;
-  const int64_t brow = static_cast<int64_t>(bmb) * a.bm.H * a.bm.Mb;  // head row 0, tile row 0
+  // a per-head block mask (a head-dependent rule) gives each CTA one query
+  // head (the plan sets heads_per_cta = 1), whose row it reads
+  const int bmh = a.bm.H > 1 ? hk * a.G + hc * p.heads_per_cta : 0;
+  const int64_t brow = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb;  // tile row 0
   const int nfull = __ldg(a.bm.full_kv_num_blocks + brow);
   const int ntiles = nfull + __ldg(a.bm.kv_num_blocks + brow);
   const int t0 = split * p.tiles_per_split;
@@ -150,11 +153,17 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         if (u >= kStagesDec && !mbar_wait(&bars.empty[s], ((u / kStagesDec) - 1) & 1, abort, a.status, a.wait_cycles)) break;
         const int n = list_tile(a, brow, nfull, t0 + u / subs_per_tile);
         const int kv0 = n * a.bm.BN + (u % subs_per_tile) * kSub;
+        // dense cache: rows kv0.. of (b, hk); paged: the 64 keys sit in one page
+        int row = kv0, outer = b;
+        if (a.page_table) {
+          outer = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, kv0);
+          row = kv0 % a.page_size;
+        }
         uint8_t* st = smem + s * C::kStageBytes;
         mbar_expect_tx(&bars.full[s], C::kStageBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(st + c * C::kBoxBytes, &map_k, &bars.full[s], c * 64, kv0, hk, b);
-          tma_load_4d(st + C::kTileBytes + c * C::kBoxBytes, &map_v, &bars.full[s], c * 64, kv0, hk, b);
+          tma_load_4d(st + c * C::kBoxBytes, &map_k, &bars.full[s], c * 64, row, hk, outer);
+          tma_load_4d(st + C::kTileBytes + c * C::kBoxBytes, &map_v, &bars.full[s], c * 64, row, hk, outer);
         }
         issued = u + 1;
       }
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           } else {
             g = score_apply<false>(a.score, sc[nt][e] * a.scale, b, qpos[half], kv, a.S, slope2[half]) * kLog2eD;
           }
-          const bool vis = rok[half] && (!need_mask || mask_visible(a.mask, b, qpos[half], kv, S_b, a.S));
+          const bool vis = rok[half] && (!need_mask || mask_visible(a.mask, b, hq[half], qpos[half], kv, S_b, a.S));
           g = vis ? g : -INFINITY;
           sc[nt][e] = g;
           mx[half] = fmaxf(mx[half], g);
@@ -479,6 +488,7 @@ cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Ma
 
 int plan_decode(const FwdArgs& a, int split_kv, int num_sms, DecodePlan* p) {
   p->heads_per_cta = a.G < kRows / a.L ? a.G : kRows / a.L;
+  if (a.bm.H > 1) p->heads_per_cta = 1;  // per-head tile lists: one query head per CTA
   p->rows_per_cta = p->heads_per_cta * a.L;
   const int head_chunks = (a.G + p->heads_per_cta - 1) / p->heads_per_cta;
   const int units = a.B * a.Hkv * head_chunks;

@@ -90,8 +90,24 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
     for (int cc = cb; cc < ce; cc += kChunk) {
       const int nk = min(kChunk, ce - cc);
       __syncthreads();
-      for (int i = t; i < nk * E; i += blockDim.x) sk[i] = to_f(kb[(cc + i / E) * a.k_stride[2] + i % E]);
-      for (int i = t; i < nk * Ev; i += blockDim.x) sv[i] = to_f(vb[(cc + i / Ev) * a.v_stride[2] + i % Ev]);
+      if (a.page_table) {
+        // paged pools: key j is slot j % page_size of its page
+        const T* kp = static_cast<const T*>(a.k) + hk * a.k_stride[1];
+        const T* vp = static_cast<const T*>(a.v) + hk * a.v_stride[1];
+        for (int i = t; i < nk * E; i += blockDim.x) {
+          const int j = cc + i / E;
+          const int pg = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, j);
+          sk[i] = to_f(kp[pg * a.k_stride[0] + (j % a.page_size) * a.k_stride[2] + i % E]);
+        }
+        for (int i = t; i < nk * Ev; i += blockDim.x) {
+          const int j = cc + i / Ev;
+          const int pg = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, j);
+          sv[i] = to_f(vp[pg * a.v_stride[0] + (j % a.page_size) * a.v_stride[2] + i % Ev]);
+        }
+      } else {
+        for (int i = t; i < nk * E; i += blockDim.x) sk[i] = to_f(kb[(cc + i / E) * a.k_stride[2] + i % E]);
+        for (int i = t; i < nk * Ev; i += blockDim.x) sv[i] = to_f(vb[(cc + i / Ev) * a.v_stride[2] + i % Ev]);
+      }
       __syncthreads();
       if (!active) continue;
       float s[kChunk];
@@ -104,7 +120,7 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
           for (int e = 0; e < E; ++e) dot = fmaf(sq[t * qst + e], sk[j * E + e], dot);
           const int kv = cc + j;
           const float g = score_apply<true>(a.score, dot * a.scale, b, qpos, kv, S, slope);
-          const bool vis = is_full ? (kv < S_b) : mask_visible(a.mask, b, qpos, kv, S_b, S);
+          const bool vis = is_full ? (kv < S_b) : mask_visible(a.mask, b, h, qpos, kv, S_b, S);
           val = vis ? g : -INFINITY;
         }
         s[j] = val;

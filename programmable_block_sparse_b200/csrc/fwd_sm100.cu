@@ -47,6 +47,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "launch.h"
 #include "mods.cuh"
 
@@ -144,15 +145,6 @@ struct UnionIter {
   }
 };
 
-// Bits [lo, hi] of a 32-bit word (positions relative to the word's first column).
-__device__ __forceinline__ uint32_t span_bits(int lo, int hi) {
-  lo = max(lo, 0);
-  hi = min(hi, 31);
-  if (hi < lo) return 0u;
-  const uint32_t upto = hi == 31 ? 0xFFFFFFFFu : ((2u << hi) - 1u);
-  return upto & ~((1u << lo) - 1u);
-}
-
 // 64 consecutive fp32 TMEM columns of this thread's row into registers: four
 // loads in flight, one wait.  The empty asm statements after the wait carry
 // the registers as read-write operands so no use is scheduled before it.
@@ -207,7 +199,10 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   }
   const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
   const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
-  const bool is_doc = a.mask.kind == FA_MASK_DOCUMENT;
+  const bool is_prog = a.mask.kind == FA_MASK_PROGRAM;
+  // document ids are staged for the document rule and for composed rules
+  // that compare documents
+  const bool is_doc = a.mask.kind == FA_MASK_DOCUMENT || (is_prog && a.mask.reads_doc);
   const int* doc_row = is_doc ? a.mask.doc_id + static_cast<int64_t>(a.mask.doc_batch > 1 ? b : 0) * a.S : nullptr;
   const int my_doc = (is_doc && row_ok && qpos >= 0) ? __ldg(doc_row + qpos) : -1;
   const KeySpans spans = visible_spans(a.mask, qpos, S_b);
@@ -254,35 +249,66 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     tc_fence_after();
 
     // pass 1, per 64-column half: score rule on every cell, element mask on
-    // partial tiles / ragged edges / rows past L, row max; the transformed
-    // scores go back to TMEM for pass 2
+    // partial tiles / ragged edges / rows past L, row max.  The transformed
+    // scores t = g log2(e) go back to TMEM for pass 2 already shifted by
+    // m_fold (the running maximum, or 0 before the first visible key), so
+    // that pass 2 subtracts nothing unless the maximum moves.  Arithmetic in
+    // f32x2 pairs; maxima as trees of three-input maxima.
     const bool need_mask = !full || edge || !row_ok;
-    float mx = -INFINITY;
+    const float m_fold = (m_ref == kNoKeyMax) ? 0.0f : m_ref;
+    float mx = -INFINITY;  // maximum of t - m_fold over this tile
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       float t[64];
       const int c0 = 64 * half;
       tmem_load64(tbase + lane_base + col_s + c0, t);
+      float2* t2 = reinterpret_cast<float2*>(t);
       if constexpr (SCORE == FA_SCORE_NONE) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) t[c] *= c_out;
-      } else if constexpr (SCORE == FA_SCORE_SOFTCAP) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) t[c] = c_out * tanh_fast(t[c] * c_in);
+        for (int i = 0; i < 32; ++i) t2[i] = fma2(t2[i], splat2(c_out), splat2(-m_fold));
       } else if constexpr (SCORE == FA_SCORE_ALIBI) {
-        const float bias0 = slope2 * static_cast<float>(kv0 + c0 - qpos);
+        // bias of column c: slope2 (kv0 + c0 + c - q) - m_fold
+        const float2 b0 = splat2(slope2 * static_cast<float>(kv0 + c0 - qpos) - m_fold);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) t[c] = fmaf(t[c], c_out, fmaf(slope2, static_cast<float>(c), bias0));
+        for (int i = 0; i < 32; ++i) {
+          const float2 col = make_float2(static_cast<float>(2 * i), static_cast<float>(2 * i + 1));
+          t2[i] = fma2(t2[i], splat2(c_out), fma2(splat2(slope2), col, b0));
+        }
       } else {
-        if (has_pos) {
-          const float* pk = s_pos[cnt & 1] + c0;
+        // soft-cap on the FMA pipe: c tanh(s / c) with tanh's odd series,
+        // exact enough for |s / c| <= kTanhPolyMax; a half whose largest
+        // argument is beyond that is redone with the hardware tanh
+        float2* th = t2;  // tanh(s / c), computed in place
+        float umax = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), pk[c] - pq_scaled);
+        for (int i = 0; i < 32; i += 2) {
+          float2 u0, u1;
+          th[i] = tanh_poly2(mul2(t2[i], splat2(c_in)), u0);
+          th[i + 1] = tanh_poly2(mul2(t2[i + 1], splat2(c_in)), u1);
+          umax = max3f(umax, fmaxf(u0.x, u0.y), fmaxf(u1.x, u1.y));
+        }
+        if (__any_sync(0xffffffffu, !(umax <= kTanhPolyMax * kTanhPolyMax))) {
+          // rare: reload the raw scores (still in TMEM) for the hardware tanh
+          tmem_load64(tbase + lane_base + col_s + c0, t);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) t[c] = tanh_fast(t[c] * c_in);
+        }
+        if constexpr (SCORE == FA_SCORE_SOFTCAP) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), splat2(-m_fold));
+        } else if (has_pos) {
+          // bias of column c: slope2 (p[kv] - p[q]) - m_fold, p[kv] staged in smem
+          const float2* pk = reinterpret_cast<const float2*>(s_pos[cnt & 1] + c0);
+          const float2 b0 = splat2(-pq_scaled - m_fold);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), add2(pk[i], b0));
         } else {
-          const float bias0 = slope2 * static_cast<float>(kv0 + c0 - qpos);
+          const float2 b0 = splat2(slope2 * static_cast<float>(kv0 + c0 - qpos) - m_fold);
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            t[c] = fmaf(c_out, tanh_fast(t[c] * c_in), fmaf(slope2, static_cast<float>(c), bias0));
+          for (int i = 0; i < 32; ++i) {
+            const float2 col = make_float2(static_cast<float>(2 * i), static_cast<float>(2 * i + 1));
+            t2[i] = fma2(th[i], splat2(c_out), fma2(splat2(slope2), col, b0));
+          }
         }
       }
       if (need_mask) {
@@ -290,29 +316,31 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const int base = kv0 + c0 + 32 * w;
-          bits[w] = row_ok ? (span_bits(spans.a0 - base, spans.a1 - base) |
-                              span_bits(spans.b0 - base, spans.b1 - base))
-                           : 0u;
-        }
-        if (stage_doc) {
-          const int* dk = s_doc[cnt & 1] + c0;
+          uint32_t same = 0xFFFFFFFFu;  // same-document bits of the word's keys
+          if (stage_doc) {
+            const int* dk = s_doc[cnt & 1] + c0 + 32 * w;
+            same = 0u;
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            uint32_t same = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) same |= (dk[32 * w + i] == my_doc ? 1u : 0u) << i;
-            bits[w] &= same;
+            for (int i = 0; i < 32; ++i) same |= (dk[i] == my_doc ? 1u : 0u) << i;
+            if (qpos < 0) same = 0u;
+          }
+          if (is_prog) {
+            bits[w] = row_ok ? (program_bits(a.mask, h, qpos, base, same) & span_bits(-1, S_b - 1 - base)) : 0u;
+          } else {
+            bits[w] = row_ok ? ((span_bits(spans.a0 - base, spans.a1 - base) |
+                                 span_bits(spans.b0 - base, spans.b1 - base)) & same)
+                             : 0u;
           }
         }
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (!((bits[c >> 5] >> (c & 31)) & 1u)) t[c] = -INFINITY;
       }
-#pragma unroll
-      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, t[c]);
+      mx = fmaxf(mx, max64(t));
       tmem_store64(tbase + lane_base + col_s + c0, t);
     }
     tmem_wait_st();
+    mx += m_fold;  // the tile's true maximum (log2 units), -inf without a visible key
     m_true = fmaxf(m_true, mx);
 
     // running max: move it (and rescale O) only when it grows past 2^8.  O_X
@@ -351,7 +379,10 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
       l_sum *= f;
     }
     m_ref = m_new;
-    const float m_use = m_ref;
+    // TMEM holds t - m_fold; P = 2^(t - m_ref) needs a further shift only
+    // when the maximum moved (or before the first visible key)
+    const float delta = m_ref - m_fold;
+    const bool shift = __any_sync(0xffffffffu, delta != 0.0f);
 
     // pass 2, per half: P = 2^(t - m) as bf16 pairs, 64 columns in all
     // (head dim 128: over the first 64 S columns; half h writes columns
@@ -367,11 +398,14 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free[X]);
       }
+      if (shift) {
+        float2* t2 = reinterpret_cast<float2*>(t);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        t[c] = ex2_approx(t[c] - m_use);
-        psum += t[c];
+        for (int i = 0; i < 32; ++i) t2[i] = add2(t2[i], splat2(-delta));
       }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) t[c] = ex2_approx(t[c]);
+      psum += sum64(t);
       if (half == 0) wait_pv();
       if (!alive) break;
 #pragma unroll
@@ -526,14 +560,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = u % NS;
           const uint32_t round = u / NS;
           if (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
+          // a paged pool is read in two 64-key boxes per tile, each from its
+          // own page (the swizzle follows the smem address, so the halves
+          // land exactly as one 128-row box would)
+          int pg0 = b, pg1 = b, row0 = n * kTile, row1 = n * kTile + 64;
+          if (a.page_table) {
+            pg0 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, n * kTile);
+            pg1 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, n * kTile + 64);
+            row0 = (n * kTile) % a.page_size;
+            row1 = (n * kTile + 64) % a.page_size;
+          }
           mbar_expect_tx(&bars.k_full[s], C::kTileBytes);
-          for (int c = 0; c < C::kBoxes; ++c)
-            tma_load_4d(sK + s * C::kTileBytes + c * (kTile * 128), &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
+          for (int c = 0; c < C::kBoxes; ++c) {
+            uint8_t* dst = sK + s * C::kTileBytes + c * (kTile * 128);
+            if (a.page_table) {
+              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, row0, hk, pg0);
+              tma_load_4d(dst + 64 * 128, &map_k, &bars.k_full[s], c * 64, row1, hk, pg1);
+            } else {
+              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
+            }
+          }
           issued_k = u + 1;
           if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
           mbar_expect_tx(&bars.v_full[s], C::kTileBytes);
-          for (int c = 0; c < C::kBoxes; ++c)
-            tma_load_4d(sV + s * C::kTileBytes + c * (kTile * 128), &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
+          for (int c = 0; c < C::kBoxes; ++c) {
+            uint8_t* dst = sV + s * C::kTileBytes + c * (kTile * 128);
+            if (a.page_table) {
+              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, row0, hk, pg0);
+              tma_load_4d(dst + 64 * 128, &map_v, &bars.v_full[s], c * 64, row1, hk, pg1);
+            } else {
+              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
+            }
+          }
           issued_v = u + 1;
         }
         // Drain on every path: each copy this thread issued lands before it

@@ -40,6 +40,11 @@ struct FwdArgs {
   long long wait_cycles;      // budget of each main-path device wait
   int out_f32;                // out is fp32 (else the input dtype)
   int rows_safe;              // every row has a visible key: no empty-row guard
+  // paged KV cache (page_table == null: k, v are (B, Hkv, S, D)): logical key
+  // j of sequence b is slot j % page_size of page page_table[b * pages_per_seq
+  // + j / page_size] of the pools k, v (num_pages, Hkv, page_size, D)
+  const int* page_table;
+  int page_size, pages_per_seq, num_pages;
   int64_t q_stride[4], k_stride[4], v_stride[4], o_stride[4];
   int B, Hq, Hkv, L, S, E, Ev, G;
   int dtype;                  // FA_DTYPE_*

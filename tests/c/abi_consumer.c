@@ -38,7 +38,7 @@ int main(void) {
     fa_forward_options opts;
     memset(&opts, 0, sizeof(opts));
     opts.flags = FA_FLAG_ROWS_GUARANTEED_SAFE;
-    expect(sizeof(opts) == 24, "fa_forward_options is 24 bytes");
+    expect(sizeof(opts) == 40, "fa_forward_options is 40 bytes");
     expect(flexattn_forward(NULL, NULL, NULL, NULL, NULL, 0.0f, 0, NULL, NULL, NULL, 0, &opts, NULL, 0, NULL) ==
                FA_ERR_NULL,
            "forward with options and NULL tensors");

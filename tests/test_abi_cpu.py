@@ -42,11 +42,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_struct_layouts_match_header_sizes():
-    assert C.sizeof(_abi.fa_mask_mod) == 6 * 4 + 2 * 8
+    assert C.sizeof(_abi.fa_mask_mod) == 6 * 4 + 2 * 8 + 2 * 4 + 16 * 8
     assert C.sizeof(_abi.fa_score_mod) == 4 * 4 + 8
     assert C.sizeof(_abi.fa_block_mask) == 8 * 4 + 4 * 8
     assert C.sizeof(_abi.fa_tensor) == 8 + 4 + 4 + 8 * 8
-    assert C.sizeof(_abi.fa_forward_options) == 8 + 8 + 4 + 4
+    assert C.sizeof(_abi.fa_forward_options) == 8 + 8 + 4 + 4 + 8 + 4 + 4
 
 
 def test_version(lib):
@@ -181,3 +181,66 @@ def test_forward_rejects_bad_options(lib):
     assert "flags" in fa.flexattn_last_error()
     assert _call(lib, q, k, v, o, bm, opts=_abi.fa_forward_options(reserved=1)) == 9
     assert _call(lib, q, k, v, o, bm, opts=_abi.fa_forward_options(wait_cycles=-5)) == 9
+
+
+def _prog(*instrs, doc=None):
+    m = _abi.fa_mask_mod(kind=6)
+    m.n_instr = len(instrs)
+    for i, (op, arg) in enumerate(instrs):
+        m.program[i].op, m.program[i].arg = op, arg
+    if doc is not None:
+        m.doc_id, m.doc_batch = doc, 1
+    return m
+
+
+def test_composed_rules_checked_on_the_host(lib):
+    q, k, v, o = _t(2, 4, 256, 64), _t(2, 4, 256, 64), _t(2, 4, 256, 64), _t(2, 4, 256, 64)
+    bm = _bm(1, 1, 256, 256, 128, 128)
+    AND, OR, NOT = 16, 17, 18
+    # broken postfix: two verdicts left, an operator without operands, no instruction
+    assert _call(lib, q, k, v, o, bm, mask=_prog((1, 0), (6, 4))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog((1, 0), (AND, 0))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog()) == 9
+    # bad arguments and unknown instructions; same-document without ids
+    assert _call(lib, q, k, v, o, bm, mask=_prog((6, 0))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog((4, -3))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog((2, (1 << 30) + 1))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog((12, 0))) == 9
+    assert _call(lib, q, k, v, o, bm, mask=_prog((5, 0))) == 9
+    # a head-dependent rule needs a per-head block mask
+    assert _call(lib, q, k, v, o, bm, mask=_prog((1, 0), (7, 2), (AND, 0))) == 5
+    assert "per-head" in fa.flexattn_last_error()
+    # an OR of four ANDs of two predicates needs 2^4 = 16 clauses in AND-of-OR form
+    big = []
+    for i in range(4):
+        big += [(2, 10 + i), (3, 20 + i), (AND, 0)]
+        if i:
+            big.append((OR, 0))
+    assert _call(lib, q, k, v, o, bm, mask=_prog(*big)) == 11
+    assert "clauses" in fa.flexattn_last_error()
+    # a valid rule passes the host checks and reaches the launch-free build check
+    bm2 = _bm(1, 1, 64, 64, 16, 16)
+    bm2.Mb = 5
+    assert lib.flexattn_build_block_mask(C.byref(_prog((1, 0), (6, 4), (AND, 0))), C.byref(bm2), None) == 5
+
+
+def test_paged_cache_checked_on_the_host(lib):
+    q, o = _t(2, 4, 4, 64), _t(2, 4, 4, 64)
+    kp, vp = _t(10, 2, 64, 64), _t(10, 2, 64, 64)   # pools of 10 pages of 64 keys
+    bm = _bm(2, 1, 4, 256, 128, 128)                  # logical length 4 pages x 64
+    opts = _abi.fa_forward_options(page_table=FAKE, page_size=64, pages_per_seq=4)
+    # pools whose slot extent is not the page size, or k and v of different pool sizes
+    assert _call(lib, q, _t(10, 2, 32, 64), _t(10, 2, 32, 64), o, bm, gqa=1, opts=opts) == 2
+    assert _call(lib, q, kp, _t(9, 2, 64, 64), o, bm, gqa=1, opts=opts) == 2
+    # page size or table width below 1
+    assert _call(lib, q, kp, vp, o, bm, gqa=1,
+                 opts=_abi.fa_forward_options(page_table=FAKE, page_size=0, pages_per_seq=4)) == 9
+    # the block mask must describe the logical length
+    assert _call(lib, q, kp, vp, o, _bm(2, 1, 4, 640, 128, 128), gqa=1, opts=opts) == 5
+    # forced splits need pages of a multiple of 64 keys
+    odd = _abi.fa_forward_options(page_table=FAKE, page_size=48, pages_per_seq=4)
+    assert _call(lib, q, _t(10, 2, 48, 64), _t(10, 2, 48, 64), o, _bm(2, 1, 4, 192, 128, 128), gqa=1, split=3,
+                 opts=odd) == 11
+    n = C.c_size_t()
+    assert lib.flexattn_forward_workspace_size(C.byref(q), C.byref(_t(10, 2, 32, 64)), C.byref(vp), C.byref(bm), 0,
+                                               C.byref(opts), C.byref(n)) == 2
