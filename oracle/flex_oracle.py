@@ -380,6 +380,120 @@ def forward_sampled(q, k, v, samples, scale=None, mask=None, score=None, kv_len=
 
 
 # ---------------------------------------------------------------------------
+# Backward pass
+# ---------------------------------------------------------------------------
+
+def score_mod_slope(score, s):
+    """dg/ds of the score rule at the scaled scores ``s``.
+
+    The distance biases do not depend on s (slope 1); the soft-cap
+    g = c tanh(s / c) has dg/ds = 1 - tanh(s / c)^2.
+    """
+    kind = score["kind"]
+    if kind in ("softcap", "cap_then_bias"):
+        c = float(score["cap"])
+        return 1.0 - np.tanh(s / c) ** 2
+    if kind in ("none", "alibi"):
+        return np.ones_like(s)
+    raise ValueError(f"unknown score kind {kind!r}")
+
+
+def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score):
+    """Gradients of one (batch b, query head h) unit: (dq (L,E), dk (S,E), dv (S,Ev)).
+
+    "flexattention-score-mod-block-mask" shows the loss's backward call
+    through flex_attention; the gradients are those of the forward
+    definition ("What one connection goes through"), by the chain rule:
+    with P the softmax weights (0 on hidden keys) and O = P V,
+        dV = P^T dO,  dP = dO V^T,  D_i = sum_e dO_ie O_ie,
+        dS~ = P * (dP - D),  ds = dS~ * dg/ds,
+        dQ = scale ds K,  dK = scale ds^T Q.
+    A row without a visible key has P = 0 and contributes nothing.  k and v
+    gradients are those of this unit alone; GQA sums them over the query
+    heads that share a KV head (:func:`backward`).
+    """
+    q_bh, k_bh, v_bh, do_bh = _as_f64(q_bh), _as_f64(k_bh), _as_f64(v_bh), _as_f64(do_bh)
+    L, S = q_bh.shape[0], k_bh.shape[0]
+    qp = query_positions(L, S_b)
+    kv = np.arange(S, dtype=np.int64)
+    s = scale * (q_bh @ k_bh.T)
+    g = score_mod(score, s, b, h, qp, kv, Hq)
+    vis = visible(mask, b, h, qp, kv, S_b)
+    masked = np.where(vis, g, NEG_INF)
+    m = masked.max(axis=1)
+    p = np.zeros_like(s)
+    live = m > NEG_INF
+    if live.any():
+        e = np.exp(masked[live] - m[live, None])
+        p[live] = e / e.sum(axis=1, keepdims=True)
+    o = p @ v_bh
+    dv = p.T @ do_bh
+    dp = do_bh @ v_bh.T
+    D = (do_bh * o).sum(axis=1)
+    dst = p * (dp - D[:, None])
+    ds = dst * score_mod_slope(score, s)
+    dq = scale * (ds @ k_bh)
+    dk = scale * (ds.T @ q_bh)
+    return dq, dk, dv
+
+
+def backward(q, k, v, do, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False):
+    """fp64 gradients (dq (B,Hq,L,E), dk (B,Hkv,S,E), dv (B,Hkv,S,Ev)) of
+    sum(out * do) for the forward of :func:`forward`; GQA sums dk and dv over
+    the query heads of each KV head ("PyTorch Flex Attention complete guide"
+    section 6.1: the KV heads are broadcast to the query heads)."""
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, Hq, L, E = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if Hq != Hkv:
+        assert enable_gqa and Hq % Hkv == 0, "Hq != Hkv needs enable_gqa and Hq % Hkv == 0"
+    G = Hq // Hkv
+    mask = mask or {"kind": "none"}
+    score = score or {"kind": "none"}
+    scale = 1.0 / math.sqrt(E) if scale is None else float(scale)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
+        for h in range(Hq):
+            kvh = h // G
+            uq, uk, uv = backward_unit(q[b, h], k[b, kvh], v[b, kvh], do[b, h], b, h, Hq, S_b, scale, mask, score)
+            dq[b, h] = uq
+            dk[b, kvh] += uk
+            dv[b, kvh] += uv
+    return dq, dk, dv
+
+
+def transpose_block_mask(bm):
+    """Query-side lists of a BlockMask: for every key tile n, the query tiles
+    m whose row lists n as full or as partial, ascending, unused slots 0.
+
+    "PyTorch Flex Attention complete guide" section 3.3: from_kv_blocks
+    derives the query-side block information (_transpose_ordered) that the
+    backward pass walks.  Returns q_num_blocks (B,H,Nb), q_indices (B,H,Nb,Mb),
+    full_q_num_blocks, full_q_indices.
+    """
+    B, H, Mb = bm["kv_num_blocks"].shape
+    Nb = bm["Nb"]
+    out = {"q_num_blocks": np.zeros((B, H, Nb), np.int32), "q_indices": np.zeros((B, H, Nb, Mb), np.int32),
+           "full_q_num_blocks": np.zeros((B, H, Nb), np.int32),
+           "full_q_indices": np.zeros((B, H, Nb, Mb), np.int32)}
+    for b in range(B):
+        for h in range(H):
+            for kind, cnt, idx in (("", "kv_num_blocks", "kv_indices"),
+                                   ("full_", "full_kv_num_blocks", "full_kv_indices")):
+                lists = [[] for _ in range(Nb)]
+                for m in range(Mb):
+                    for i in range(int(bm[cnt][b, h, m])):
+                        lists[int(bm[idx][b, h, m, i])].append(m)
+                for n in range(Nb):
+                    out[kind + "q_num_blocks"][b, h, n] = len(lists[n])
+                    out[kind + "q_indices"][b, h, n, :len(lists[n])] = sorted(lists[n])
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Paged KV cache
 # ---------------------------------------------------------------------------
 

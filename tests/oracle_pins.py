@@ -681,6 +681,112 @@ def check_paged_cache(o):
     assert np.allclose(po, ro, atol=1e-13) and np.allclose(pl, rl, atol=1e-13)
 
 
+def check_backward(o):
+    """Gradients of sum(out * W) for a random W.
+
+    Pinned by central finite differences of the oracle's forward (step 1e-5,
+    fp64) on tiny shapes for every score kind and several masks; by torch
+    autograd (CPU, fp64) through a plain torch statement of the forward
+    (scores, score rule, mask, softmax, values); by closed forms (a row with
+    one visible key passes dO straight to that key's value and gives q and k
+    nothing; a row with no visible key gives nothing at all); and by GQA
+    (dk, dv of a KV head = the sum over its query heads).
+    """
+    import torch
+    r = np.random.default_rng(61)
+    B, Hq, Hkv, L, S, E, Ev = 1, 4, 2, 5, 7, 3, 2
+    masks = [{"kind": "causal"}, {"kind": "sliding_window", "window": 3, "n_sink": 1},
+             {"kind": "and", "masks": [{"kind": "causal"}, {"kind": "stride", "value": 2}]}]
+    scores = [{"kind": "none"}, {"kind": "softcap", "cap": 1.5}, {"kind": "alibi"},
+              {"kind": "cap_then_bias", "cap": 2.0, "slope_heads": 0, "pos": "global"}]
+    for mask in masks:
+        for score in scores:
+            q = r.standard_normal((B, Hq, L, E))
+            k = r.standard_normal((B, Hkv, S, E))
+            v = r.standard_normal((B, Hkv, S, Ev))
+            W = r.standard_normal((B, Hq, L, Ev))
+            kv_len = [6]
+            dq, dk, dv = o.backward(q, k, v, W, 0.8, mask, score, kv_len=kv_len, enable_gqa=True)
+
+            def loss(q_, k_, v_):
+                out, _ = o.forward(q_, k_, v_, 0.8, mask, score, kv_len=kv_len, enable_gqa=True)
+                return float((out * W).sum())
+            eps = 1e-5
+            for x, gx in ((q, dq), (k, dk), (v, dv)):
+                num = np.zeros_like(x)
+                for idx in np.ndindex(x.shape):
+                    xp = x.copy()
+                    xp[idx] += eps
+                    args_p = [xp if y is x else y for y in (q, k, v)]
+                    xm = x.copy()
+                    xm[idx] -= eps
+                    args_m = [xm if y is x else y for y in (q, k, v)]
+                    num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+                assert np.allclose(num, gx, atol=1e-7, rtol=1e-6), (mask["kind"], score["kind"])
+            # torch autograd through a plain statement of the forward
+            tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+            G = Hq // Hkv
+            kk = tk.repeat_interleave(G, dim=1)
+            vv = tv.repeat_interleave(G, dim=1)
+            sc = 0.8 * tq @ kk.transpose(-1, -2)
+            qpos = torch.arange(L) + (kv_len[0] - L)
+            kpos = torch.arange(S)
+            if score["kind"] in ("softcap", "cap_then_bias"):
+                g = score["cap"] * torch.tanh(sc / score["cap"])
+            else:
+                g = sc
+            if score["kind"] in ("alibi", "cap_then_bias"):
+                slope = torch.tensor([2.0 ** (-8.0 * (hh + 1) / Hq) for hh in range(Hq)], dtype=torch.float64)
+                dist = (qpos[:, None] - kpos[None, :]).to(torch.float64)
+                g = g - slope[None, :, None, None] * dist if score["kind"] == "alibi" else \
+                    g + slope[None, :, None, None] * (-dist)
+            vis = torch.from_numpy(o.visible(mask, 0, 0, qpos.numpy(), kpos.numpy(), kv_len[0]))
+            out = torch.softmax(g.masked_fill(~vis, float("-inf")), dim=-1) @ vv
+            (out * torch.from_numpy(W)).sum().backward()
+            for t, gx in ((tq, dq), (tk, dk), (tv, dv)):
+                assert np.allclose(t.grad.numpy(), gx, atol=1e-12), (mask["kind"], score["kind"])
+    # one visible key (row 0, causal): dv gets dO, q gets nothing from that row
+    q = r.standard_normal((1, 1, 4, 3))
+    k = r.standard_normal((1, 1, 4, 3))
+    v = r.standard_normal((1, 1, 4, 2))
+    W = np.zeros((1, 1, 4, 2))
+    W[0, 0, 0] = [1.5, -2.0]
+    dq, dk, dv = o.backward(q, k, v, W, 1.0, {"kind": "causal"}, {"kind": "softcap", "cap": 3.0})
+    assert np.allclose(dv[0, 0, 0], [1.5, -2.0], atol=0) and np.all(dv[0, 0, 1:] == 0)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    # rows without a visible key (bottom-right, 3 keys for 5 queries) give nothing
+    q = r.standard_normal((1, 1, 5, 3))
+    k = r.standard_normal((1, 1, 3, 3))
+    v = r.standard_normal((1, 1, 3, 2))
+    W = np.zeros((1, 1, 5, 2))
+    W[0, 0, :2] = 1.0
+    dq, dk, dv = o.backward(q, k, v, W, 1.0, {"kind": "causal"}, None)
+    assert np.all(dq == 0) and np.all(dk == 0) and np.all(dv == 0)
+    # GQA: dk, dv of a KV head are the sums over its query heads
+    q, k, v = _tiny_case(8, 5, 6, 3, 2, B=1, Hq=6, Hkv=2)
+    W = r.standard_normal((1, 6, 5, 2))
+    a = o.backward(q, k, v, W, 0.5, {"kind": "causal"}, {"kind": "alibi"}, enable_gqa=True)
+    bq, bk, bv = o.backward(q, np.repeat(k, 3, axis=1), np.repeat(v, 3, axis=1), W, 0.5, {"kind": "causal"},
+                            {"kind": "alibi"})
+    assert np.allclose(a[0], bq, atol=1e-14)
+    assert np.allclose(a[1], bk.reshape(1, 2, 3, 6, 3).sum(axis=2), atol=1e-13)
+    assert np.allclose(a[2], bv.reshape(1, 2, 3, 6, 2).sum(axis=2), atol=1e-13)
+    # query-side lists: the transpose of the tile map, ascending
+    doc = np.repeat(np.arange(4), [9, 14, 5, 12])
+    for mask in ({"kind": "causal"}, {"kind": "document", "doc_id": doc},
+                 {"kind": "sliding_window", "window": 9, "n_sink": 2}):
+        bm = o.block_mask(mask, 1, 1, 40, 40, 4, 8)
+        tq = o.transpose_block_mask(bm)
+        grid = o.block_map(bm)
+        for n in range(bm["Nb"]):
+            part = [m for m in range(bm["Mb"]) if grid[m][n] == "P"]
+            full = [m for m in range(bm["Mb"]) if grid[m][n] == "F"]
+            assert tq["q_indices"][0, 0, n, :len(part)].tolist() == part and tq["q_num_blocks"][0, 0, n] == len(part)
+            assert tq["full_q_indices"][0, 0, n, :len(full)].tolist() == full
+            assert tq["full_q_num_blocks"][0, 0, n] == len(full)
+            assert np.all(tq["q_indices"][0, 0, n, len(part):] == 0)
+
+
 ALL_CHECKS = [
     check_m1_six_token_tiles, check_m6_packed_documents, check_m2_softcap_after_mask,
     check_m3_decode_offset, check_m4_bottom_right, check_m5_left_padding,
@@ -691,4 +797,4 @@ ALL_CHECKS = [
     check_max_scores, check_forward_unit_matches_forward, check_composed_masks,
     check_paged_cache,
 ]
-SLOW_CHECKS = [check_workload_tile_counts]
+SLOW_CHECKS = [check_workload_tile_counts, check_backward]

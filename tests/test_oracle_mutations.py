@@ -62,6 +62,12 @@ MUTATIONS = {
                         "out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]][:, ::-1]"),
     "page_table_ignored": ("out[b, :, i * page_size:(i + 1) * page_size] = pool[table[b, i]]",
                            "out[b, :, i * page_size:(i + 1) * page_size] = pool[b * pages_per_seq + i]"),
+    "backward_slope_dropped": ("ds = dst * score_mod_slope(score, s)", "ds = dst"),
+    "backward_rowsum_dropped": ("dst = p * (dp - D[:, None])", "dst = p * dp"),
+    "backward_dk_unscaled": ("dk = scale * (ds.T @ q_bh)", "dk = ds.T @ q_bh"),
+    "backward_gqa_overwrite": ("dk[b, kvh] += uk", "dk[b, kvh] = uk"),
+    "backward_cap_slope": ("return 1.0 - np.tanh(s / c) ** 2", "return 1.0 - np.tanh(s / c)"),
+    "transpose_unsorted": ("= sorted(lists[n])", "= lists[n][::-1]"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
                            "out[live] = outs[:, live].mean(axis=0)"),
 }
