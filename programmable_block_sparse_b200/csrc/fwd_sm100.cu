@@ -145,6 +145,31 @@ struct UnionIter {
   }
 };
 
+// Rarely run paths, kept out of line so the softmax loop stays compact in the
+// instruction cache: a composed mask rule's bits for one 32-key word, and the
+// hardware tanh of 64 columns (for a half whose arguments exceed the
+// polynomial's range).
+__device__ __noinline__ uint32_t program_word(const MaskParams* m, int h, int q, int base, uint32_t same, int S_b) {
+  return program_bits(*m, h, q, base, same) & span_bits(-1, S_b - 1 - base);
+}
+// In place in TMEM: the 64 columns at taddr become tanh(column * c_in).
+__device__ __noinline__ void tanh_hw_tmem(uint32_t taddr, float c_in) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[16];
+    tmem_ld16(taddr + 16 * c, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float y;
+      asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(__uint_as_float(r[i]) * c_in));
+      r[i] = __float_as_uint(y);
+    }
+    tmem_st16(taddr + 16 * c, r);
+  }
+  tmem_wait_st();
+}
+
 // 64 consecutive fp32 TMEM columns of this thread's row into registers: four
 // loads in flight, one wait.  The empty asm statements after the wait carry
 // the registers as read-write operands so no use is scheduled before it.
@@ -289,9 +314,8 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
         }
         if (__any_sync(0xffffffffu, !(umax <= kTanhPolyMax * kTanhPolyMax))) {
           // rare: reload the raw scores (still in TMEM) for the hardware tanh
+          tanh_hw_tmem(tbase + lane_base + col_s + c0, c_in);
           tmem_load64(tbase + lane_base + col_s + c0, t);
-#pragma unroll
-          for (int c = 0; c < 64; ++c) t[c] = tanh_fast(t[c] * c_in);
         }
         if constexpr (SCORE == FA_SCORE_SOFTCAP) {
 #pragma unroll
@@ -325,7 +349,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
             if (qpos < 0) same = 0u;
           }
           if (is_prog) {
-            bits[w] = row_ok ? (program_bits(a.mask, h, qpos, base, same) & span_bits(-1, S_b - 1 - base)) : 0u;
+            bits[w] = row_ok ? program_word(&a.mask, h, qpos, base, same, S_b) : 0u;
           } else {
             bits[w] = row_ok ? ((span_bits(spans.a0 - base, spans.a1 - base) |
                                  span_bits(spans.b0 - base, spans.b1 - base)) & same)
@@ -405,7 +429,6 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
       }
 #pragma unroll
       for (int c = 0; c < 64; ++c) t[c] = ex2_approx(t[c]);
-      psum += sum64(t);
       if (half == 0) wait_pv();
       if (!alive) break;
 #pragma unroll
@@ -415,25 +438,20 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[32 * g + 2 * i], t[32 * g + 2 * i + 1]);
         tmem_st16(tbase + lane_base + col_p + 32 * half + 16 * g, pk);
       }
-      if (half == 0) {
-        // P of keys 0-63 is in TMEM: the first half of PV can run while
-        // the second half of P is computed
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_half[X]);
-      }
+      // this half of P is in TMEM: signal the MMA thread first (half 0 lets
+      // the first half of PV run while the second half of P is computed),
+      // then add up the row sum, which nothing waits for
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(half == 0 ? &bars.p_half[X] : &bars.p_full[X]);
+      psum += sum64(t);
     }
     if (!alive) {
       tmem_wait_st();
       continue;  // leave at the next tile's vote, with the group
     }
     l_sum += psum;
-
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.p_full[X]);
   }
 
   // ------------------------------------------------------------- epilogue
@@ -485,7 +503,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
 
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_sm100_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap map_q,
+    fwd_sm100_kernel(const __grid_constant__ FwdArgs a, const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
   using C = Cfg<D>;
   constexpr int NS = C::kStages;
