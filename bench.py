@@ -68,7 +68,7 @@ HEADLINE = BENCH_ITEMS[0][0]
 NCU_TRAFFIC = {}
 
 KERNEL_SOURCES = {
-    "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh"),
+    "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh", "fastmath.cuh"),
     "decode": ("decode.cu", "mods.cuh", "common.cuh"),
     "general": ("fwd_simt.cu", "mods.cuh", "common.cuh"),
 }

@@ -351,6 +351,58 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
                                     const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, int32_t split_kv,
                                     void* stream);
 
+/* ----------------------------------------------------------------------- */
+/* Backward pass                                                            */
+/* ----------------------------------------------------------------------- */
+
+/* Query-side lists of a BlockMask ([guide] 3.3: from_kv_blocks derives them
+ * for the backward pass): for key tile n of row (b, h), the query tiles m
+ * whose row lists n as partial (q_indices, counted in q_num_blocks) or as
+ * full (full_q_indices, full_q_num_blocks), ascending, unused slots 0.
+ * B, H, Mb, Nb are those of the BlockMask it is built from; all four arrays
+ * are caller-allocated device int32, row-major. */
+typedef struct fa_block_mask_q {
+  int32_t B, H, Mb, Nb;
+  int32_t* q_num_blocks;        /* [B, H, Nb]     */
+  int32_t* q_indices;           /* [B, H, Nb, Mb] */
+  int32_t* full_q_num_blocks;   /* [B, H, Nb]     */
+  int32_t* full_q_indices;      /* [B, H, Nb, Mb] */
+} fa_block_mask_q;
+
+/* Fill the query-side lists of `block_mask` on the GPU.
+ * Errors: FA_ERR_NULL, FA_ERR_SHAPE, FA_ERR_MASK_SHAPE (dims disagree), FA_ERR_CUDA. */
+int flexattn_transpose_block_mask(const fa_block_mask* block_mask, const fa_block_mask_q* q_side, void* stream);
+
+/* Bytes of device workspace flexattn_backward needs (fp32 D = rowsum(dout * out),
+ * [B, Hq, L]). */
+int flexattn_backward_workspace_size(const fa_tensor* q, size_t* bytes);
+
+/* Backward pass: the gradients of sum(out * dout) with respect to q, k and v
+ * for the forward pass of flexattn_forward with the same arguments
+ * ([charlestar] calls backward on the loss through flex_attention).  With P
+ * the softmax weights recomputed from lse (0 on hidden keys),
+ *   dv = P^T dout,  dP = dout v^T,  D = rowsum(dout * out),
+ *   dS = P (dP - D) dg/ds  (dg/ds = 1 - tanh(s / cap)^2 under a soft-cap, else 1),
+ *   dq = scale dS k,  dk = scale dS^T q;
+ * dk and dv sum over the query heads that share a KV head (GQA).  The dk / dv
+ * kernel walks each key tile's query-side list and the dq kernel each query
+ * tile's key-side list, so every gradient is written once, in a fixed order
+ * (deterministic; [guide] 5, WRITE_DQ).
+ *   q, k, v, out (forward output), dout (B, Hq, L, Ev): bf16, E == Ev in
+ *       {64, 128}; lse: the forward's fp32 [B, Hq, L].
+ *   dq (B, Hq, L, E), dk (B, Hkv, S, E), dv (B, Hkv, S, Ev): bf16 or fp32,
+ *       written in full.
+ *   block_mask / block_mask_q: 128 x 128 tiles, with the query-side lists
+ *       from flexattn_transpose_block_mask.
+ *   workspace: flexattn_backward_workspace_size() bytes.
+ * No paged cache.  Errors: those of flexattn_forward, and FA_ERR_UNSUPPORTED
+ * for other dtypes, head dims or tile sizes. */
+int flexattn_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
+                      const fa_tensor* dout, const float* lse, const fa_tensor* dq, const fa_tensor* dk,
+                      const fa_tensor* dv, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
+                      const fa_mask_mod* mask_mod, const fa_block_mask* block_mask,
+                      const fa_block_mask_q* block_mask_q, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Wait for `stream`, then read and clear the device status word that the
  * kernels set when a bounded wait runs out (FA_ERR_TIMEOUT) or an index check
  * fails.  *status receives FA_OK or the first error recorded since the last

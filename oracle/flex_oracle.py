@@ -398,7 +398,7 @@ def score_mod_slope(score, s):
     raise ValueError(f"unknown score kind {kind!r}")
 
 
-def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score):
+def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score, out_bh=None):
     """Gradients of one (batch b, query head h) unit: (dq (L,E), dk (S,E), dv (S,Ev)).
 
     "flexattention-score-mod-block-mask" shows the loss's backward call
@@ -411,6 +411,11 @@ def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score):
     A row without a visible key has P = 0 and contributes nothing.  k and v
     gradients are those of this unit alone; GQA sums them over the query
     heads that share a KV head (:func:`backward`).
+
+    ``out_bh`` is the forward output as the caller stored it (for bf16
+    outputs, O rounded to bf16).  A backward call receives the stored output
+    and forms D from it, so D carries that rounding; by default D uses the
+    exact O.
     """
     q_bh, k_bh, v_bh, do_bh = _as_f64(q_bh), _as_f64(k_bh), _as_f64(v_bh), _as_f64(do_bh)
     L, S = q_bh.shape[0], k_bh.shape[0]
@@ -426,7 +431,7 @@ def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score):
     if live.any():
         e = np.exp(masked[live] - m[live, None])
         p[live] = e / e.sum(axis=1, keepdims=True)
-    o = p @ v_bh
+    o = p @ v_bh if out_bh is None else _as_f64(out_bh)
     dv = p.T @ do_bh
     dp = do_bh @ v_bh.T
     D = (do_bh * o).sum(axis=1)
@@ -437,11 +442,13 @@ def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score):
     return dq, dk, dv
 
 
-def backward(q, k, v, do, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False):
+def backward(q, k, v, do, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, out=None):
     """fp64 gradients (dq (B,Hq,L,E), dk (B,Hkv,S,E), dv (B,Hkv,S,Ev)) of
     sum(out * do) for the forward of :func:`forward`; GQA sums dk and dv over
     the query heads of each KV head ("PyTorch Flex Attention complete guide"
-    section 6.1: the KV heads are broadcast to the query heads)."""
+    section 6.1: the KV heads are broadcast to the query heads).  ``out``
+    (B,Hq,L,Ev), optional: the stored forward output that D is formed from
+    (see :func:`backward_unit`)."""
     q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
     B, Hq, L, E = q.shape
     Hkv, S = k.shape[1], k.shape[2]
@@ -458,7 +465,8 @@ def backward(q, k, v, do, scale=None, mask=None, score=None, kv_len=None, enable
         S_b = S if kv_len is None else int(np.asarray(kv_len)[b])
         for h in range(Hq):
             kvh = h // G
-            uq, uk, uv = backward_unit(q[b, h], k[b, kvh], v[b, kvh], do[b, h], b, h, Hq, S_b, scale, mask, score)
+            uq, uk, uv = backward_unit(q[b, h], k[b, kvh], v[b, kvh], do[b, h], b, h, Hq, S_b, scale, mask, score,
+                                       None if out is None else out[b, h])
             dq[b, h] = uq
             dk[b, kvh] += uk
             dv[b, kvh] += uv

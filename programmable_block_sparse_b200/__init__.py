@@ -34,7 +34,7 @@ __all__ = [
     "BlockMask", "FlexAttnError", "library_path", "load_library", "and_masks", "or_masks", "not_mask",
     "flexattn_version", "flexattn_last_error", "flexattn_block_mask_dims", "flexattn_build_block_mask",
     "flexattn_forward_workspace_size", "flexattn_forward", "flexattn_forward_decode_noalloc",
-    "flexattn_poll_device_status",
+    "flexattn_poll_device_status", "BlockMaskQ", "flexattn_transpose_block_mask", "flexattn_backward",
 ]
 
 _LIB = None
@@ -373,3 +373,70 @@ def flexattn_poll_device_status(stream=None):
     st = C.c_int32()
     _check(load_library().flexattn_poll_device_status(_stream_handle(stream), C.byref(st)))
     return st.value
+
+
+@dataclass
+class BlockMaskQ:
+    """Device-resident query-side lists of a BlockMask (for the backward pass)."""
+
+    B: int
+    H: int
+    Mb: int
+    Nb: int
+    q_num_blocks: object
+    q_indices: object
+    full_q_num_blocks: object
+    full_q_indices: object
+
+    def as_struct(self):
+        s = _abi.fa_block_mask_q()
+        s.B, s.H, s.Mb, s.Nb = self.B, self.H, self.Mb, self.Nb
+        s.q_num_blocks = self.q_num_blocks.data_ptr()
+        s.q_indices = self.q_indices.data_ptr()
+        s.full_q_num_blocks = self.full_q_num_blocks.data_ptr()
+        s.full_q_indices = self.full_q_indices.data_ptr()
+        return s
+
+
+def flexattn_transpose_block_mask(block_mask, stream=None, out=None):
+    """Query-side lists of ``block_mask`` (allocated here unless ``out`` is given)."""
+    import torch
+    bm = block_mask
+    if out is None:
+        z = dict(dtype=torch.int32, device=bm.kv_num_blocks.device)
+        out = BlockMaskQ(bm.B, bm.H, bm.Mb, bm.Nb, torch.empty((bm.B, bm.H, bm.Nb), **z),
+                         torch.empty((bm.B, bm.H, bm.Nb, bm.Mb), **z), torch.empty((bm.B, bm.H, bm.Nb), **z),
+                         torch.empty((bm.B, bm.H, bm.Nb, bm.Mb), **z))
+    s, q = bm.as_struct(), out.as_struct()
+    _check(load_library().flexattn_transpose_block_mask(C.byref(s), C.byref(q), _stream_handle(stream)))
+    return out
+
+
+def flexattn_backward(q, k, v, out, dout, lse, block_mask, q_side=None, score_mod=None, mask_mod=None, scale=None,
+                      enable_gqa=False, dq=None, dk=None, dv=None, grad_dtype=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the forward pass with the
+    same arguments; ``lse`` is the forward's.  ``q_side`` defaults to the
+    transposed lists of ``block_mask``; gradients are allocated in
+    ``grad_dtype`` (default: the input dtype) unless given."""
+    import torch
+    gd = grad_dtype or q.dtype
+    dq = torch.empty(q.shape, dtype=gd, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=gd, device=q.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=gd, device=q.device) if dv is None else dv
+    if q_side is None:
+        q_side = flexattn_transpose_block_mask(block_mask, stream=stream)
+    n = C.c_size_t()
+    qs = _tensor_struct(q)
+    _check(load_library().flexattn_backward_workspace_size(C.byref(qs), C.byref(n)))
+    if workspace is None:
+        workspace = torch.empty(max(1, n.value), dtype=torch.uint8, device=q.device)
+    ks, vs, os_, ds = _tensor_struct(k), _tensor_struct(v), _tensor_struct(out), _tensor_struct(dout)
+    gq, gk, gv = _tensor_struct(dq), _tensor_struct(dk), _tensor_struct(dv)
+    bm, qsd = block_mask.as_struct(), q_side.as_struct()
+    sm, mm = _score_struct(score_mod), _mask_struct(mask_mod)
+    sc = 0.0 if scale is None or math.isnan(float(scale)) else float(scale)
+    _check(load_library().flexattn_backward(
+        C.byref(qs), C.byref(ks), C.byref(vs), C.byref(os_), C.byref(ds), _ptr(lse), C.byref(gq), C.byref(gk),
+        C.byref(gv), C.c_float(sc), int(bool(enable_gqa)), C.byref(sm), C.byref(mm), C.byref(bm), C.byref(qsd),
+        _ptr(workspace), C.c_size_t(workspace.numel()), _stream_handle(stream)))
+    return dq, dk, dv

@@ -70,6 +70,14 @@ class fa_forward_options(C.Structure):
     ]
 
 
+class fa_block_mask_q(C.Structure):
+    _fields_ = [
+        ("B", C.c_int32), ("H", C.c_int32), ("Mb", C.c_int32), ("Nb", C.c_int32),
+        ("q_num_blocks", C.c_void_p), ("q_indices", C.c_void_p),
+        ("full_q_num_blocks", C.c_void_p), ("full_q_indices", C.c_void_p),
+    ]
+
+
 # (name, restype, argtypes) for every exported entry point.
 PROTOTYPES = [
     ("flexattn_version", C.c_int, []),
@@ -88,6 +96,13 @@ PROTOTYPES = [
      [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_void_p,
       C.c_float, C.c_int32, C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask),
       C.c_int32, C.c_void_p]),
+    ("flexattn_transpose_block_mask", C.c_int, [C.POINTER(fa_block_mask), C.POINTER(fa_block_mask_q), C.c_void_p]),
+    ("flexattn_backward_workspace_size", C.c_int, [C.POINTER(fa_tensor), C.POINTER(C.c_size_t)]),
+    ("flexattn_backward", C.c_int,
+     [C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor),
+      C.c_void_p, C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.POINTER(fa_tensor), C.c_float, C.c_int32,
+      C.POINTER(fa_score_mod), C.POINTER(fa_mask_mod), C.POINTER(fa_block_mask), C.POINTER(fa_block_mask_q),
+      C.c_void_p, C.c_size_t, C.c_void_p]),
     ("flexattn_poll_device_status", C.c_int, [C.c_void_p, C.POINTER(C.c_int32)]),
 ]
 

@@ -686,6 +686,126 @@ int flexattn_forward_decode_noalloc(const fa_tensor* q, const fa_tensor* k, cons
   return FA_OK;
 }
 
+int flexattn_transpose_block_mask(const fa_block_mask* bm, const fa_block_mask_q* qs, void* stream) {
+  if (!bm || !qs) return fail(FA_ERR_NULL, "block_mask and q_side must not be NULL");
+  int rc;
+  if ((rc = check_block_mask_dims(bm))) return rc;
+  if (qs->B != bm->B || qs->H != bm->H || qs->Mb != bm->Mb || qs->Nb != bm->Nb)
+    return fail(FA_ERR_MASK_SHAPE, "query-side lists must have the block mask's B, H, Mb, Nb");
+  if (!qs->q_num_blocks || !qs->q_indices || !qs->full_q_num_blocks || !qs->full_q_indices)
+    return fail(FA_ERR_NULL, "query-side arrays must not be NULL");
+  TransposeArgs t{bm->B, bm->H, bm->Mb, bm->Nb, bm->kv_num_blocks, bm->kv_indices, bm->full_kv_num_blocks,
+                  bm->full_kv_indices, qs->q_num_blocks, qs->q_indices, qs->full_q_num_blocks, qs->full_q_indices};
+  cudaError_t e = launch_transpose(t, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block-mask transpose launch");
+  return FA_OK;
+}
+
+int flexattn_backward_workspace_size(const fa_tensor* q, size_t* bytes) {
+  if (!bytes) return fail(FA_ERR_NULL, "bytes must not be NULL");
+  int rc;
+  if ((rc = check_tensor(q, "q"))) return rc;
+  *bytes = static_cast<size_t>(q->size[0]) * q->size[1] * q->size[2] * sizeof(float);
+  return FA_OK;
+}
+
+int flexattn_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,
+                      const fa_tensor* dout, const float* lse, const fa_tensor* dq, const fa_tensor* dk,
+                      const fa_tensor* dv, float scale, int32_t enable_gqa, const fa_score_mod* score_mod,
+                      const fa_mask_mod* mask_mod, const fa_block_mask* block_mask, const fa_block_mask_q* qs,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!out || !dout || !dq || !dk || !dv || !lse || !qs) return fail(FA_ERR_NULL, "backward arguments must not be NULL");
+  FwdArgs f;
+  Path path;
+  int rc = prepare(q, k, v, out, scale, enable_gqa, score_mod, mask_mod, block_mask, 1, nullptr, &f, &path);
+  if (rc) return rc;
+  if ((rc = check_tensor(dout, "dout")) || (rc = check_tensor(dq, "dq")) || (rc = check_tensor(dk, "dk")) ||
+      (rc = check_tensor(dv, "dv")))
+    return rc;
+  const int B = f.B, Hq = f.Hq, Hkv = f.Hkv, L = f.L, S = f.S, E = f.E;
+  if (q->dtype != FA_DTYPE_BF16 || out->dtype != FA_DTYPE_BF16 || dout->dtype != FA_DTYPE_BF16)
+    return fail(FA_ERR_UNSUPPORTED, "the backward pass takes bf16 q, k, v, out and dout");
+  if (f.E != f.Ev || (E != 64 && E != 128))
+    return fail(FA_ERR_UNSUPPORTED, "the backward pass needs E == Ev in {64, 128}");
+  if (block_mask->BM != 128 || block_mask->BN != 128)
+    return fail(FA_ERR_UNSUPPORTED, "the backward pass needs 128 x 128 tiles");
+  for (int i = 0; i < 4; ++i)
+    if (dout->size[i] != out->size[i]) return fail(FA_ERR_SHAPE, "dout must have the shape of out");
+  const int64_t want_q[4] = {B, Hq, L, E}, want_k[4] = {B, Hkv, S, E};
+  for (int i = 0; i < 4; ++i) {
+    if (dq->size[i] != want_q[i]) return fail(FA_ERR_SHAPE, "dq must be (B, Hq, L, E)");
+    if (dk->size[i] != want_k[i] || dv->size[i] != want_k[i]) return fail(FA_ERR_SHAPE, "dk and dv must be (B, Hkv, S, E)");
+  }
+  for (const fa_tensor* g : {dq, dk, dv})
+    if (g->dtype != FA_DTYPE_BF16 && g->dtype != FA_DTYPE_F32) return fail(FA_ERR_DTYPE, "gradients are bf16 or fp32");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return fail(FA_ERR_ALIGN, "the backward pass needs 16-byte aligned tensors and strides");
+  if (qs->B != block_mask->B || qs->H != block_mask->H || qs->Mb != block_mask->Mb || qs->Nb != block_mask->Nb)
+    return fail(FA_ERR_MASK_SHAPE, "query-side lists must have the block mask's B, H, Mb, Nb");
+  if (!qs->q_num_blocks || !qs->q_indices || !qs->full_q_num_blocks || !qs->full_q_indices)
+    return fail(FA_ERR_NULL, "query-side arrays must not be NULL");
+  const size_t need = static_cast<size_t>(B) * Hq * L * sizeof(float);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(FA_ERR_WORKSPACE, "the backward pass needs %zu bytes of workspace (got %zu)", need,
+                workspace ? workspace_bytes : static_cast<size_t>(0));
+  if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(FA_ERR_ALIGN, "workspace must be 16-byte aligned");
+  if (B > 65535 || Hq > 65535 || block_mask->Nb > 65535) return fail(FA_ERR_SHAPE, "grid extents above 65535");
+
+  BwdArgs a{};
+  int serr = 0;
+  a.status = status_word(&serr);
+  if (serr) return fail(FA_ERR_CUDA, "cannot locate the device status word");
+  a.wait_cycles = kWaitCycles;
+  a.q = q->data;
+  a.k = k->data;
+  a.v = v->data;
+  a.out = out->data;
+  a.dout = dout->data;
+  a.lse = lse;
+  a.dsum = static_cast<float*>(workspace);
+  a.dq = dq->data;
+  a.dk = dk->data;
+  a.dv = dv->data;
+  for (int i = 0; i < 4; ++i) {
+    a.q_stride[i] = q->stride[i];
+    a.k_stride[i] = k->stride[i];
+    a.v_stride[i] = v->stride[i];
+    a.o_stride[i] = out->stride[i];
+    a.do_stride[i] = dout->stride[i];
+    a.dq_stride[i] = dq->stride[i];
+    a.dk_stride[i] = dk->stride[i];
+    a.dv_stride[i] = dv->stride[i];
+  }
+  a.dq_f32 = dq->dtype == FA_DTYPE_F32;
+  a.dk_f32 = dk->dtype == FA_DTYPE_F32;
+  a.dv_f32 = dv->dtype == FA_DTYPE_F32;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.S = S;
+  a.E = E;
+  a.G = f.G;
+  a.scale = f.scale;
+  a.mask = f.mask;
+  a.score = f.score;
+  a.bm = f.bm;
+  a.qB = qs->B;
+  a.qH = qs->H;
+  a.q_num_blocks = qs->q_num_blocks;
+  a.q_indices = qs->q_indices;
+  a.full_q_num_blocks = qs->full_q_num_blocks;
+  a.full_q_indices = qs->full_q_indices;
+  BwdMaps maps;
+  if ((rc = encode_bf16_map(&maps.q, q, 128)) || (rc = encode_bf16_map(&maps.k, k, 128)) ||
+      (rc = encode_bf16_map(&maps.v, v, 128)) || (rc = encode_bf16_map(&maps.dout, dout, 128)))
+    return rc;
+  cudaError_t e = launch_bwd(a, maps, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return FA_OK;
+}
+
 int flexattn_poll_device_status(void* stream, int32_t* status) {
   if (!status) return fail(FA_ERR_NULL, "status must not be NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

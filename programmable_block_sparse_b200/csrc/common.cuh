@@ -206,6 +206,34 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
   return r != 0;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 64 consecutive fp32 TMEM columns of this thread's row into registers: four
+// loads in flight, one wait.  The empty asm statements after the wait carry
+// the registers as read-write operands so no use is scheduled before it.
+__device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&t)[64]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(t);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(u + c * 16));
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t* x = u + c * 16;
+    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),
+                 "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]),
+                 "+r"(x[14]), "+r"(x[15]));
+  }
+}
+__device__ __forceinline__ void tmem_store64(uint32_t taddr, const float (&t)[64]) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(t);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_st16(taddr + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(u + c * 16));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

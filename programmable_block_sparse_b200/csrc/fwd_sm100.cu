@@ -89,12 +89,6 @@ struct Barriers {
   int abort;
 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // Walks the union of the two query tiles' full and partial lists in
 // descending key order (for causal-like rules the nearest, highest-scoring
 // keys come first, so the running max rarely has to move afterwards).
@@ -168,28 +162,6 @@ __device__ __noinline__ void tanh_hw_tmem(uint32_t taddr, float c_in) {
     tmem_st16(taddr + 16 * c, r);
   }
   tmem_wait_st();
-}
-
-// 64 consecutive fp32 TMEM columns of this thread's row into registers: four
-// loads in flight, one wait.  The empty asm statements after the wait carry
-// the registers as read-write operands so no use is scheduled before it.
-__device__ __forceinline__ void tmem_load64(uint32_t taddr, float (&t)[64]) {
-  uint32_t* u = reinterpret_cast<uint32_t*>(t);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(u + c * 16));
-  tmem_wait_ld();
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t* x = u + c * 16;
-    asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),
-                 "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]),
-                 "+r"(x[14]), "+r"(x[15]));
-  }
-}
-__device__ __forceinline__ void tmem_store64(uint32_t taddr, const float (&t)[64]) {
-  const uint32_t* u = reinterpret_cast<const uint32_t*>(t);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_st16(taddr + c * 16, *reinterpret_cast<const uint32_t(*)[16]>(u + c * 16));
 }
 
 // Softmax and epilogue of one 128-row query tile; runs on one warpgroup.

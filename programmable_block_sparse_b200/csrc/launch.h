@@ -77,4 +77,37 @@ int plan_decode(const FwdArgs& a, int split_kv, int num_sms, DecodePlan* plan);
 cudaError_t launch_decode(const FwdArgs& a, const DecodePlan& plan, const Sm100Maps& maps, void* workspace,
                           cudaStream_t stream);
 
+// Backward pass (bf16, E = Ev in {64, 128}, 128 x 128 tiles).
+struct BwdArgs {
+  int* status;  // device status word
+  long long wait_cycles;
+  const void *q, *k, *v, *out, *dout;
+  const float* lse;  // [B, Hq, L] from the forward pass
+  float* dsum;       // workspace: D = rowsum(dout * out), [B, Hq, L]
+  void *dq, *dk, *dv;
+  int64_t q_stride[4], k_stride[4], v_stride[4], o_stride[4], do_stride[4];
+  int64_t dq_stride[4], dk_stride[4], dv_stride[4];
+  int dq_f32, dk_f32, dv_f32;  // gradient storage: fp32, else bf16
+  int B, Hq, Hkv, L, S, E, G;
+  float scale;
+  MaskParams mask;
+  ScoreParams score;
+  BlockMaskView bm;  // key-side lists (the forward's)
+  // query-side lists: for key tile n of row (b, h), the query tiles listing it
+  int qB, qH;
+  const int *q_num_blocks, *q_indices, *full_q_num_blocks, *full_q_indices;
+};
+struct BwdMaps {
+  CUtensorMap q, k, v, dout;
+};
+cudaError_t launch_bwd(const BwdArgs& a, const BwdMaps& maps, cudaStream_t stream);
+
+// Query-side lists from the key-side lists of a BlockMask.
+struct TransposeArgs {
+  int B, H, Mb, Nb;
+  const int *kv_num_blocks, *kv_indices, *full_kv_num_blocks, *full_kv_indices;
+  int *q_num_blocks, *q_indices, *full_q_num_blocks, *full_q_indices;
+};
+cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t stream);
+
 }  // namespace fa

@@ -228,6 +228,77 @@ __device__ __forceinline__ int program_box(const MaskParams& m, int h, int q0, i
   return res;
 }
 
+// The transposed view, for the backward pass over key rows: one predicate
+// over the 32 queries at logical positions qbase .. qbase + 31 for key kv.
+__device__ __forceinline__ uint32_t prog_pred_bits_q(const MaskLit& lt, int h, int kv, int qbase, uint32_t same_doc) {
+  const int op = lt.op & 0xff, arg = lt.arg;
+  switch (op) {
+    case FA_PROG_TRUE:
+      return 0xFFFFFFFFu;
+    case FA_PROG_CAUSAL:  // q >= kv
+      return span_bits(kv - qbase, 31);
+    case FA_PROG_DISTANCE_BELOW:  // q < kv + arg
+      return span_bits(-1, kv + arg - 1 - qbase);
+    case FA_PROG_KEY_BELOW:
+      return kv < arg ? 0xFFFFFFFFu : 0u;
+    case FA_PROG_SAME_CHUNK: {
+      const int c0 = floor_div(kv, arg) * arg;
+      return span_bits(c0 - qbase, c0 + arg - 1 - qbase);
+    }
+    case FA_PROG_SAME_DOCUMENT:
+      return same_doc;
+    case FA_PROG_STRIDE: {  // queries qbase + i with i = kv - qbase (mod arg)
+      const int r = mod_pos(kv - qbase, arg);
+      return arg < 32 ? (lt.pat << r) : (r < 32 ? (1u << r) : 0u);
+    }
+    case FA_PROG_HEAD_BELOW:
+      return h < arg ? 0xFFFFFFFFu : 0u;
+    default:
+      return 0u;
+  }
+}
+
+__device__ __forceinline__ uint32_t program_bits_q(const MaskParams& m, int h, int kv, int qbase, uint32_t same_doc) {
+  uint32_t res = 0xFFFFFFFFu;
+#pragma unroll
+  for (int c = 0; c < kMaxClauses; ++c) {
+    if (c >= m.n_clauses) break;
+    uint32_t cl = 0u;
+#pragma unroll
+    for (int l = 0; l < kMaxLits; ++l) {
+      if (l >= m.clause_len[c]) break;
+      const MaskLit lt = m.lit[c][l];
+      const uint32_t v = prog_pred_bits_q(lt, h, kv, qbase, same_doc);
+      cl |= (lt.op & kLitNeg) ? ~v : v;
+    }
+    res &= cl;
+  }
+  return res;
+}
+
+// Fixed rules over the 32 queries qbase .. qbase + 31 for key kv (kv < S_b;
+// the caller clears queries outside the valid rows and applies same_doc for
+// the document rule).
+__device__ __forceinline__ uint32_t fixed_bits_q(const MaskParams& m, int kv, int qbase) {
+  switch (m.kind) {
+    case FA_MASK_NONE:
+      return 0xFFFFFFFFu;
+    case FA_MASK_CAUSAL:
+    case FA_MASK_DOCUMENT:
+      return span_bits(kv - qbase, 31);
+    case FA_MASK_SLIDING_WINDOW:
+      return kv < m.n_sink ? span_bits(kv - qbase, 31) : span_bits(kv - qbase, kv + m.window - 1 - qbase);
+    case FA_MASK_PREFIX_LM:
+      return kv < m.prefix ? 0xFFFFFFFFu : span_bits(kv - qbase, 31);
+    case FA_MASK_CHUNKED: {
+      const int c0 = (kv / m.chunk) * m.chunk;  // kv >= 0
+      return span_bits(kv - qbase, c0 + m.chunk - 1 - qbase);
+    }
+    default:
+      return 0u;
+  }
+}
+
 // M(b, h, q, kv): visibility of key kv for the query at logical position q
 // of query head h.  The caller guarantees 0 <= kv; keys at or beyond S_b are
 // invisible.

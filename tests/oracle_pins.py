@@ -689,8 +689,9 @@ def check_backward(o):
     autograd (CPU, fp64) through a plain torch statement of the forward
     (scores, score rule, mask, softmax, values); by closed forms (a row with
     one visible key passes dO straight to that key's value and gives q and k
-    nothing; a row with no visible key gives nothing at all); and by GQA
-    (dk, dv of a KV head = the sum over its query heads).
+    nothing; a row with no visible key gives nothing at all); by GQA
+    (dk, dv of a KV head = the sum over its query heads); and, for D formed
+    from a stored output, by the closed-form shift that a changed D gives dq.
     """
     import torch
     r = np.random.default_rng(61)
@@ -771,6 +772,22 @@ def check_backward(o):
     assert np.allclose(a[0], bq, atol=1e-14)
     assert np.allclose(a[1], bk.reshape(1, 2, 3, 6, 3).sum(axis=2), atol=1e-13)
     assert np.allclose(a[2], bv.reshape(1, 2, 3, 6, 2).sum(axis=2), atol=1e-13)
+    # the stored output: D is formed from the out the caller passes.  With
+    # out = O + c_i dO_i / |dO_i|^2 (so D grows by c_i), dv is unchanged and,
+    # with no score rule, dq_i moves by -scale c_i sum_j P_ij k_j, which is the
+    # forward's output for v = k.
+    q, k, v = _tiny_case(9, 6, 8, 3, 2, B=1, Hq=2, Hkv=2)
+    W = r.standard_normal((1, 2, 6, 2))
+    c = r.standard_normal((1, 2, 6))
+    out, _ = o.forward(q, k, v, 0.7, {"kind": "causal"}, None)
+    stored = out + c[..., None] * W / (W * W).sum(axis=-1, keepdims=True)
+    ex = o.backward(q, k, v, W, 0.7, {"kind": "causal"}, None)
+    st = o.backward(q, k, v, W, 0.7, {"kind": "causal"}, None, out=stored)
+    same = o.backward(q, k, v, W, 0.7, {"kind": "causal"}, None, out=out)
+    pk, _ = o.forward(q, k, k, 0.7, {"kind": "causal"}, None)
+    assert np.allclose(st[2], ex[2], atol=1e-14)
+    assert np.allclose(st[0] - ex[0], -0.7 * c[..., None] * pk, atol=1e-12)
+    assert all(np.allclose(a_, b_, atol=1e-14) for a_, b_ in zip(same, ex))
     # query-side lists: the transpose of the tile map, ascending
     doc = np.repeat(np.arange(4), [9, 14, 5, 12])
     for mask in ({"kind": "causal"}, {"kind": "document", "doc_id": doc},

@@ -244,3 +244,45 @@ def test_paged_cache_checked_on_the_host(lib):
     n = C.c_size_t()
     assert lib.flexattn_forward_workspace_size(C.byref(q), C.byref(_t(10, 2, 32, 64)), C.byref(vp), C.byref(bm), 0,
                                                C.byref(opts), C.byref(n)) == 2
+
+
+def _bq(B, H, Mb, Nb):
+    s = _abi.fa_block_mask_q()
+    s.B, s.H, s.Mb, s.Nb = B, H, Mb, Nb
+    s.q_num_blocks = s.q_indices = s.full_q_num_blocks = s.full_q_indices = FAKE
+    return s
+
+
+def test_backward_checked_on_the_host(lib):
+    q, k, v, o, do = (_t(2, 4, 256, 64) for _ in range(5))
+    dq, dk, dv = _t(2, 4, 256, 64), _t(2, 4, 256, 64), _t(2, 4, 256, 64)
+    bm, bq = _bm(1, 1, 256, 256, 128, 128), _bq(1, 1, 2, 2)
+    sc, mk = _abi.fa_score_mod(kind=0), _abi.fa_mask_mod(kind=1)
+
+    def call(q=q, k=k, v=v, o=o, do=do, dq=dq, dk=dk, dv=dv, bm=bm, bq=bq, ws=FAKE, ws_bytes=1 << 20, lse=FAKE):
+        return lib.flexattn_backward(C.byref(q), C.byref(k), C.byref(v), C.byref(o), C.byref(do), lse, C.byref(dq),
+                                     C.byref(dk), C.byref(dv), 0.0, 0, C.byref(sc), C.byref(mk), C.byref(bm),
+                                     C.byref(bq), ws, ws_bytes, None)
+    f32 = _abi.FA_DTYPE_F32
+    assert call(q=_t(2, 4, 256, 64, dtype=f32), k=_t(2, 4, 256, 64, dtype=f32), v=_t(2, 4, 256, 64, dtype=f32),
+                o=_t(2, 4, 256, 64, dtype=f32)) == 11                       # fp32 inputs
+    assert call(q=_t(2, 4, 256, 96), k=_t(2, 4, 256, 96), v=_t(2, 4, 256, 96), o=_t(2, 4, 256, 96),
+                do=_t(2, 4, 256, 96), dq=_t(2, 4, 256, 96), dk=_t(2, 4, 256, 96), dv=_t(2, 4, 256, 96)) == 11
+    assert call(bm=_bm(1, 1, 256, 256, 64, 64), bq=_bq(1, 1, 4, 4)) == 11  # other tiles
+    assert call(dq=_t(2, 4, 255, 64)) == 2                                  # gradient shapes
+    assert call(do=_t(2, 4, 128, 64)) == 2
+    assert call(bq=_bq(1, 1, 2, 3)) == 5                                    # lists of another mask
+    assert call(ws_bytes=16) == 10                                          # workspace
+    assert call(lse=None) == 1
+    assert call(dk=_t(2, 4, 256, 64, stride=(4 * 256 * 64, 256 * 64, 64, 2))) == 8
+    n = C.c_size_t()
+    assert lib.flexattn_backward_workspace_size(C.byref(q), C.byref(n)) == 0 and n.value == 2 * 4 * 256 * 4
+
+
+def test_transpose_checked_on_the_host(lib):
+    bm = _bm(1, 1, 256, 256, 128, 128)
+    assert lib.flexattn_transpose_block_mask(C.byref(bm), C.byref(_bq(1, 1, 2, 3)), None) == 5
+    assert lib.flexattn_transpose_block_mask(None, C.byref(_bq(1, 1, 2, 2)), None) == 1
+    nul = _bq(1, 1, 2, 2)
+    nul.q_indices = None
+    assert lib.flexattn_transpose_block_mask(C.byref(bm), C.byref(nul), None) == 1

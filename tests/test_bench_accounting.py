@@ -43,7 +43,7 @@ def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     import bench
     csrc = tmp_path / "programmable_block_sparse_b200" / "csrc"
     csrc.mkdir(parents=True)
-    for name in ("fwd_sm100.cu", "mods.cuh", "common.cuh"):
+    for name in bench.KERNEL_SOURCES["prefill"]:
         (csrc / name).write_text("int f(int x) {\n  return x + 1;  // add one\n}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h0 = bench.kernel_source_hash("prefill")

@@ -66,6 +66,7 @@ MUTATIONS = {
     "backward_rowsum_dropped": ("dst = p * (dp - D[:, None])", "dst = p * dp"),
     "backward_dk_unscaled": ("dk = scale * (ds.T @ q_bh)", "dk = ds.T @ q_bh"),
     "backward_gqa_overwrite": ("dk[b, kvh] += uk", "dk[b, kvh] = uk"),
+    "backward_stored_out_ignored": ("o = p @ v_bh if out_bh is None else _as_f64(out_bh)", "o = p @ v_bh"),
     "backward_cap_slope": ("return 1.0 - np.tanh(s / c) ** 2", "return 1.0 - np.tanh(s / c)"),
     "transpose_unsorted": ("= sorted(lists[n])", "= lists[n][::-1]"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',
