@@ -57,6 +57,9 @@ BENCH_ITEMS = [
     ("decode_kv_cache", "decode_kv_cache", {}),
     ("decode_kv_cache_q1", "decode_kv_cache", {"L": 1}),
     ("fp32_causal_small", "fp32_causal_small", {}),
+    # the backward pass (dq, dk, dv of sum(out * dout)) of two workloads
+    ("backward_causal_softcap_alibi", "causal_softcap_alibi", {"backward": True}),
+    ("backward_packed_docs", "packed_docs", {"backward": True}),
 ]
 HEADLINE = BENCH_ITEMS[0][0]
 
@@ -69,9 +72,15 @@ NCU_TRAFFIC = {}
 
 KERNEL_SOURCES = {
     "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh", "fastmath.cuh"),
-    "decode": ("decode.cu", "mods.cuh", "common.cuh"),
+    "decode": ("decode.cu", "mods.cuh", "common.cuh", "fastmath.cuh"),
     "general": ("fwd_simt.cu", "mods.cuh", "common.cuh"),
+    "backward": ("bwd_sm100.cu", "mods.cuh", "common.cuh", "fastmath.cuh"),
 }
+
+
+def config_over(over):
+    """A bench item's overrides of the workload config (its mode keys removed)."""
+    return {k: v for k, v in over.items() if k != "backward"}
 
 
 def kernel_source_hash(kind="prefill"):
@@ -262,9 +271,10 @@ class OracleSampler:
     prefill, or the unit's share of its KV head's valid cache bytes for decode.
     """
 
-    def __init__(self, name, **over):
+    def __init__(self, name, backward=False, **over):
         import torch
         self.name = name
+        self.backward = backward
         self.c = c = wl.config(name, **over)
         self.kv_len = self.doc_lengths = None
         if name == "decode_kv_cache":
@@ -284,6 +294,8 @@ class OracleSampler:
         self.counts = [visible_counts_rows(c, b, self.kv_len, self.doc_lengths) for b in range(c["B"])]
         self.unit_desc = ("one (batch, query head) unit, all its query rows" if self.decode else
                           f"a block of {self.rows} query rows of one (batch, query head) unit, every row in full")
+        if backward:
+            self.unit_desc += " (the backward: dq of the rows and their parts of dk, dv)"
 
     def block(self, i):
         """(work, seconds) of the i-th sample; samples are spread over units and rows."""
@@ -307,6 +319,12 @@ class OracleSampler:
         kn = k.to(torch.float64).numpy()
         vn = v.to(torch.float64).numpy()
         qp = o.query_positions(c["L"], S_b)[r0:r1]
+        if self.backward:
+            don = wl.randn_slice(c["seed"], 3, b, h, c["L"], c["Ev"], self.dt)[r0:r1].to(torch.float64).numpy()
+            t0 = time.perf_counter()
+            o.backward_rows(qn, kn, vn, don, c["scale"], self.mask, self.score, b, h, qp, S_b, c["Hq"])
+            el = time.perf_counter() - t0
+            return float(self.counts[b][r0:r1].sum()) * (6 * c["E"] + 4 * c["Ev"]), el
         t0 = time.perf_counter()
         o.attention_rows(qn, kn, vn, c["scale"], self.mask, self.score, b, h, qp, S_b, c["Hq"])
         el = time.perf_counter() - t0
@@ -335,7 +353,7 @@ class OracleSampler:
 
 def cpu_baseline(label, target_s):
     _, name, over = item(label)
-    s = OracleSampler(name, **over)
+    s = OracleSampler(name, backward=over.get("backward", False), **config_over(over))
     rate, el, n = s.rate(target_s)
     return {"value": rate, "unit": s.unit, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
             "sample": f"{n} samples of {s.unit_desc}, spread over the workload's units and rows", "seconds": el}
@@ -347,8 +365,8 @@ def run_reference(args):
         return 0
     label = HEADLINE if args.workload == "all" else args.workload
     _, name, over = item(label)
-    c = wl.config(name, **over)
-    s = OracleSampler(name, **over)
+    c = wl.config(name, **config_over(over))
+    s = OracleSampler(name, backward=over.get("backward", False), **config_over(over))
     for i in range(args.warmup):
         s.block(i)
     times, works = [], []
@@ -412,8 +430,9 @@ class Workload:
         self.fa = fa
         self.label = label
         _, self.name, over = item(label)
+        self.backward = over.get("backward", False)
         (self.c, (self.q_h, self.k_h, self.v_h), self.mask, self.score, self.kv_len,
-         self.doc_lengths) = make_inputs(self.name, dev, seed_offset=rank, batch=batch, **over)
+         self.doc_lengths) = make_inputs(self.name, dev, seed_offset=rank, batch=batch, **config_over(over))
         c = self.c
         self.B_mask = c["B"] if self.kv_len is not None else 1
         self.gqa = c["Hq"] != c["Hkv"]
@@ -435,15 +454,39 @@ class Workload:
         self.visited_flops = cells * fp
         self.kv_bytes = (int(np.sum(self.kv_len)) * c["Hkv"] * (c["E"] + c["Ev"]) * self.q.element_size()
                          if self.decode else None)
+        if self.backward:
+            # the forward's out and lse once, then the backward is the timed call:
+            # the query-side lists (as the block-mask step) and the gradients
+            self.forward_call()
+            self.dout = wl.randn_dout(c["B"], c["Hq"], c["L"], c["Ev"], seed=c["seed"] + rank).to(dev)
+            self.q_side = fa.flexattn_transpose_block_mask(self.bm)
+            self.grads = tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (self.q, self.k, self.v))
+            self.bwd_ws = torch.empty(c["B"] * c["Hq"] * c["L"] * 4, dtype=torch.uint8, device=dev)
+            self.launches_per_step = 4  # query-side lists, D = rowsum(dout * out), dk / dv, dq
+            bf = 6 * c["E"] + 4 * c["Ev"]  # five products per cell: S, dP, dV, dK, dQ
+            self.vis_flops = self.vis_flops // fp * bf
+            self.visited_flops = cells * bf
 
     def build(self):
         c = self.c
+        if self.backward:
+            self.fa.flexattn_transpose_block_mask(self.bm, out=self.q_side)
+            return
         self.fa.flexattn_build_block_mask(self.mask, self.B_mask, 1, c["L"], c["S"], c["BM"], c["BN"], out=self.bm)
 
-    def forward(self):
+    def forward_call(self):
         self.fa.flexattn_forward(self.q, self.k, self.v, self.bm, score_mod=self.score, mask_mod=self.mask,
                                  scale=self.c["scale"], enable_gqa=self.gqa, out=self.out, lse=self.lse,
                                  workspace=self.ws)
+
+    def forward(self):
+        """The timed call: the forward, or for a backward item the backward."""
+        if not self.backward:
+            return self.forward_call()
+        dq, dk, dv = self.grads
+        self.fa.flexattn_backward(self.q, self.k, self.v, self.out, self.dout, self.lse, self.bm, q_side=self.q_side,
+                                  score_mod=self.score, mask_mod=self.mask, scale=self.c["scale"],
+                                  enable_gqa=self.gqa, dq=dq, dk=dk, dv=dv, workspace=self.bwd_ws)
 
     def step(self):
         self.build()
@@ -455,6 +498,8 @@ class Workload:
         (block mask bit for bit, out within 1e-2, lse within 1e-3)."""
         import torch
         fa = self.fa
+        if self.backward:
+            return self._capture_backward()
         try:
             out_ref, lse_ref = self.out.float().clone(), self.lse.clone()
             bm_ref = [t.clone() for t in (self.bm.kv_num_blocks, self.bm.kv_indices, self.bm.full_kv_num_blocks,
@@ -485,6 +530,40 @@ class Workload:
         except Exception as exc:  # capture unsupported here: keep the eager launches
             torch.cuda.synchronize()
             return None, f"eager (graph capture failed: {type(exc).__name__})"
+
+
+def _capture_backward(self):
+    """Graphs of the two backward calls, used only when a replay into cleared
+    query-side lists and gradients reproduces the eager result bit for bit
+    (the backward kernels write every gradient once, in a fixed order)."""
+    import torch
+    fa = self.fa
+    try:
+        qs = self.q_side
+        lists = (qs.q_num_blocks, qs.q_indices, qs.full_q_num_blocks, qs.full_q_indices)
+        ref = [t.clone() for t in lists + self.grads]
+        g_lists, g_bwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_lists, capture_error_mode="relaxed"):
+            self.build()
+        with torch.cuda.graph(g_bwd, capture_error_mode="relaxed"):
+            self.forward()
+        for t in lists:
+            t.fill_(-1)
+        for t in self.grads:
+            t.zero_()
+        g_lists.replay()
+        g_bwd.replay()
+        torch.cuda.synchronize()
+        same = all(torch.equal(a, b) for a, b in zip(ref, lists + self.grads))
+        if same and fa.flexattn_poll_device_status() == 0:
+            return (g_lists, g_bwd), "CUDA graph replay, one graph per call"
+        return None, "eager (graph replay did not reproduce the eager result)"
+    except Exception as exc:
+        torch.cuda.synchronize()
+        return None, f"eager (graph capture failed: {type(exc).__name__})"
+
+
+Workload._capture_backward = _capture_backward
 
 
 def measure(wk, args, dev, world, flush, peaks, peak_src):
@@ -541,7 +620,21 @@ def measure(wk, args, dev, world, flush, peaks, peak_src):
          "ms_per_step": ms_per_step, "forward_ms": fwd_mean, "forward_ms_median": statistics.median(fwd_ms),
          "block_mask_ms": statistics.mean(mask_ms), "gpu_launches": wk.launches_per_step * args.steps,
          "clocks": clocks.summary()}
-    if wk.decode:
+    if wk.backward:
+        r["step"] = "query-side lists + backward (dq, dk, dv in bf16)"
+        r["backward_ms"] = r.pop("forward_ms")
+        r["backward_ms_median"] = r.pop("forward_ms_median")
+        r["transpose_ms"] = r.pop("block_mask_ms")
+        r["value"] = whole_job_rate(wk.vis_flops, world, ms_per_step, 1e12)
+        r["unit"] = "TFLOP/s"
+        achieved = wk.visited_flops / (fwd_mean * 1e-3) / 1e12
+        r["roofline"] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                         "flops_counted_over": "visited-tile cells, (6E + 4Ev) per cell: S, dP, dV, dK, dQ"}
+        r["visible_pairs_flops"] = wk.vis_flops
+        r["visited_cells"] = wk.visited_cells
+        kind = "backward"
+    elif wk.decode:
         r["value"] = whole_job_rate(wk.kv_bytes, world, ms_per_step, 1e9)
         r["unit"] = "GB/s"
         achieved = wk.kv_bytes / (fwd_mean * 1e-3) / 1e9
@@ -648,7 +741,7 @@ def run_gpu(args):
                                                       args.cpu_seconds_other)
     h = per[head]
     _, hname, hover = item(head)
-    hc = wl.config(hname, **hover)
+    hc = wl.config(hname, **config_over(hover))
     line = {
         "metric": METRIC, "value": h["value"], "unit": h["unit"], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True, "scaling": "weak",

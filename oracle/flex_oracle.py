@@ -442,6 +442,34 @@ def backward_unit(q_bh, k_bh, v_bh, do_bh, b, h, Hq, S_b, scale, mask, score, ou
     return dq, dk, dv
 
 
+def backward_rows(q_rows, k, v, do_rows, scale, mask, score, b, h, qp, S_b, Hq, out_rows=None):
+    """The part of one unit's gradients that a set of its query rows gives:
+    (dq of those rows, their contribution to dk (S,E), to dv (S,Ev)).
+
+    The same chain rule as :func:`backward_unit`, restricted to the rows at
+    logical positions ``qp``: every row's dq depends on that row alone, and
+    dk, dv are sums over rows, so a unit's gradients are the row blocks' dq
+    stacked and their dk, dv parts added.  ``out_rows`` is the stored output
+    of those rows (D is formed from it), by default the exact one.
+    """
+    q_rows, k, v, do_rows = _as_f64(q_rows), _as_f64(k), _as_f64(v), _as_f64(do_rows)
+    kv = np.arange(k.shape[0], dtype=np.int64)
+    s = (q_rows @ k.T) * scale
+    g = score_mod(score, s, b, h, qp, kv, Hq)
+    vis = visible(mask, b, h, qp, kv, S_b)
+    masked = np.where(vis, g, NEG_INF)
+    m = masked.max(axis=1)
+    p = np.zeros_like(s)
+    live = m > NEG_INF
+    if live.any():
+        e = np.exp(masked[live] - m[live, None])
+        p[live] = e / e.sum(axis=1, keepdims=True)
+    o = p @ v if out_rows is None else _as_f64(out_rows)
+    D = (do_rows * o).sum(axis=1)
+    ds = p * (do_rows @ v.T - D[:, None]) * score_mod_slope(score, s)
+    return scale * (ds @ k), scale * (ds.T @ q_rows), p.T @ do_rows
+
+
 def backward(q, k, v, do, scale=None, mask=None, score=None, kv_len=None, enable_gqa=False, out=None):
     """fp64 gradients (dq (B,Hq,L,E), dk (B,Hkv,S,E), dv (B,Hkv,S,Ev)) of
     sum(out * do) for the forward of :func:`forward`; GQA sums dk and dv over

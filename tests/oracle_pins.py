@@ -788,6 +788,17 @@ def check_backward(o):
     assert np.allclose(st[2], ex[2], atol=1e-14)
     assert np.allclose(st[0] - ex[0], -0.7 * c[..., None] * pk, atol=1e-12)
     assert all(np.allclose(a_, b_, atol=1e-14) for a_, b_ in zip(same, ex))
+    # row blocks: a unit's dq rows stacked and dk, dv parts summed give the unit
+    q, k, v = _tiny_case(12, 9, 11, 3, 2, B=1, Hq=1, Hkv=1)
+    W = r.standard_normal((1, 1, 9, 2))
+    qp_all = o.query_positions(9, 10)
+    score = {"kind": "cap_then_bias", "cap": 2.0, "slope_heads": 2, "pos": "global"}
+    ref = o.backward_unit(q[0, 0], k[0, 0], v[0, 0], W[0, 0], 0, 1, 2, 10, 0.6, {"kind": "causal"}, score)
+    parts = [o.backward_rows(q[0, 0, r0:r1], k[0, 0], v[0, 0], W[0, 0, r0:r1], 0.6, {"kind": "causal"}, score, 0, 1,
+                             qp_all[r0:r1], 10, 2) for r0, r1 in ((0, 4), (4, 5), (5, 9))]
+    assert np.allclose(np.concatenate([pt[0] for pt in parts]), ref[0], atol=1e-13)
+    assert np.allclose(sum(pt[1] for pt in parts), ref[1], atol=1e-13)
+    assert np.allclose(sum(pt[2] for pt in parts), ref[2], atol=1e-13)
     # query-side lists: the transpose of the tile map, ascending
     doc = np.repeat(np.arange(4), [9, 14, 5, 12])
     for mask in ({"kind": "causal"}, {"kind": "document", "doc_id": doc},

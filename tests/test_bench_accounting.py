@@ -51,3 +51,20 @@ def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.kernel_source_hash("prefill") == h0
     (csrc / "fwd_sm100.cu").write_text("int f(int x) {\n  return x + 2;\n}\n")
     assert bench.kernel_source_hash("prefill") != h0
+
+
+def test_backward_items_and_their_oracle_sample():
+    """Backward bench items reuse a workload's config (their mode key is not a
+    config key) and the cpu sample times the oracle's backward of a row
+    block, counting (6E + 4Ev) FLOPs per visible pair (S, dP, dV, dK, dQ)."""
+    back = [it for it in bench.BENCH_ITEMS if it[2].get("backward")]
+    assert back
+    for label, name, over in back:
+        assert bench.config_over(over) == {}
+        wl.config(name, **bench.config_over(over))
+    s = bench.OracleSampler("causal_softcap_alibi", backward=True, L=256, S=256, B=1, Hq=2, Hkv=2)
+    work, el = s.block(0)
+    c = s.c
+    b, h = divmod(0, c["Hq"])
+    assert work == float(s.counts[b][:s.rows].sum()) * (6 * c["E"] + 4 * c["Ev"])
+    assert el > 0

@@ -37,23 +37,35 @@ def test_decode_against_oracle(L, Hq, Hkv, E, split_kv):
     _status_ok()
 
 
-@pytest.mark.parametrize("mask", [{"kind": "none"}, {"kind": "sliding_window", "window": 200, "n_sink": 4},
-                                  {"kind": "chunked", "chunk": 300}, {"kind": "prefix_lm", "prefix": 100}],
-                         ids=lambda m: m["kind"])
-@pytest.mark.parametrize("score", [{"kind": "none"}, {"kind": "alibi"},
-                                   {"kind": "cap_then_bias", "cap": 30.0, "pos": "global"}], ids=lambda s: s["kind"])
-def test_decode_mask_and_score_kinds(mask, score):
-    case = Case(3, 8, 2, 4, 1000, 128, 128, "bf16", mask, score, seed=4, kv_len=[1000, 555, 77], sentinel_tail=True)
-    out, lse = case.run(128, 128, split_kv=4)
-    assert_close(case, out, lse, *case.oracle())
+DECODE_MASKS = [{"kind": "none"}, {"kind": "sliding_window", "window": 200, "n_sink": 4},
+                {"kind": "chunked", "chunk": 300}, {"kind": "prefix_lm", "prefix": 100}, {"kind": "document"}]
+DECODE_SCORES = [{"kind": "none"}, {"kind": "alibi"}, {"kind": "cap_then_bias", "cap": 30.0, "pos": "global"},
+                 {"kind": "cap_then_bias", "cap": 20.0, "pos": "in_doc"}]
+
+
+@pytest.mark.parametrize("E", [64, 128])
+@pytest.mark.parametrize("mask", DECODE_MASKS, ids=lambda m: m["kind"])
+@pytest.mark.parametrize("score", DECODE_SCORES, ids=lambda s: s["kind"] + ("_doc" if s.get("pos") == "in_doc" else ""))
+def test_decode_mask_and_score_kinds(mask, score, E):
+    """The tensor-core decode kernel (tiles of 128 keys) on every mask and
+    score kind, with max_scores."""
+    case = Case(3, 8, 2, 4, 1000, E, E, "bf16", mask, score, seed=4, kv_len=[1000, 555, 77], sentinel_tail=True)
+    out, lse, mx = case.run(128, 128, split_kv=4, max_scores=True)
+    ro, rl, rm = case.oracle(aux=True)
+    assert_close(case, out, lse, ro, rl, mx, rm)
     _status_ok()
 
 
-def test_decode_tiles_of_64_keys():
-    case = Case(2, 4, 1, 1, 640, 128, 128, "bf16", {"kind": "causal"}, {"kind": "none"}, seed=8, kv_len=[640, 100],
+@pytest.mark.parametrize("E", [64, 128])
+@pytest.mark.parametrize("L,Hq,Hkv,split_kv", [(1, 4, 1, 0), (4, 8, 2, 3), (16, 4, 4, 0), (3, 6, 2, 2)])
+@pytest.mark.parametrize("score", [{"kind": "softcap", "cap": 30.0}, {"kind": "alibi"}], ids=lambda s: s["kind"])
+def test_decode_tiles_of_64_keys(L, Hq, Hkv, split_kv, score, E):
+    """Block masks of 64-key tiles take the mma.sync decode kernel."""
+    case = Case(2, Hq, Hkv, L, 640, E, E, "bf16", {"kind": "causal"}, score, seed=8 + L, kv_len=[640, 100],
                 sentinel_tail=True)
-    out, lse = case.run(64, 64, split_kv=0)
-    assert_close(case, out, lse, *case.oracle())
+    out, lse, mx = case.run(64, 64, split_kv=split_kv, max_scores=True)
+    ro, rl, rm = case.oracle(aux=True)
+    assert_close(case, out, lse, ro, rl, mx, rm)
     _status_ok()
 
 

@@ -29,8 +29,11 @@ CASES = {
     # group stage key-side values for one another behind a group barrier
     "tcgen05_documents": (1, 4, 4, 900, 900, 128, {"kind": "document"},
                           {"kind": "cap_then_bias", "cap": 30.0, "slope_heads": 0, "pos": "in_doc"}, None, 1),
+    # head dim 128: the tensor-core decode kernel; head dim 64: the mma.sync one
     "decode": (4, 8, 2, 4, 3000, 128, {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, [3000, 2000, 900, 129],
                4),
+    "decode_e64": (4, 8, 2, 4, 3000, 64, {"kind": "causal"}, {"kind": "softcap", "cap": 50.0},
+                   [3000, 2000, 900, 129], 4),
 }
 
 

@@ -67,6 +67,7 @@ MUTATIONS = {
     "backward_dk_unscaled": ("dk = scale * (ds.T @ q_bh)", "dk = ds.T @ q_bh"),
     "backward_gqa_overwrite": ("dk[b, kvh] += uk", "dk[b, kvh] = uk"),
     "backward_stored_out_ignored": ("o = p @ v_bh if out_bh is None else _as_f64(out_bh)", "o = p @ v_bh"),
+    "backward_rows_rowsum_dropped": ("ds = p * (do_rows @ v.T - D[:, None])", "ds = p * (do_rows @ v.T)"),
     "backward_cap_slope": ("return 1.0 - np.tanh(s / c) ** 2", "return 1.0 - np.tanh(s / c)"),
     "transpose_unsorted": ("= sorted(lists[n])", "= lists[n][::-1]"),
     "combine_unweighted": ('out[live] = np.einsum("sr,sre->re", w, outs[:, live]) / tot[:, None]',

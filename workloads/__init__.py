@@ -33,6 +33,7 @@ __all__ = [
     "slice_seed",
     "randn_slice",
     "randn_qkv",
+    "randn_dout",
     "doc_lengths",
     "doc_ids_from_lengths",
     "in_doc_positions",
@@ -92,6 +93,12 @@ def randn_qkv(B, Hq, Hkv, L, S, E, Ev, seed=0, dtype=torch.bfloat16):
     k = _fill(torch.empty((B, Hkv, S, E), dtype=dtype), seed, 1)
     v = _fill(torch.empty((B, Hkv, S, Ev), dtype=dtype), seed, 2)
     return q, k, v
+
+
+def randn_dout(B, Hq, L, Ev, seed=0, dtype=torch.bfloat16):
+    """iid N(0,1) output gradient (B,Hq,L,Ev), one generator per (b, h) slice
+    (the fourth stream after q, k, v)."""
+    return _fill(torch.empty((B, Hq, L, Ev), dtype=dtype), seed, 3)
 
 
 def doc_lengths(total, lo, hi, seed=0):
