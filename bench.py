@@ -60,7 +60,23 @@ BENCH_ITEMS = [
     # the backward pass (dq, dk, dv of sum(out * dout)) of two workloads
     ("backward_causal_softcap_alibi", "causal_softcap_alibi", {"backward": True}),
     ("backward_packed_docs", "packed_docs", {"backward": True}),
+    # composed rules at the causal workload's shape: a sliver (every fourth
+    # key: every causal tile is partial, the worst case for block sparsity)
+    # and a head-dependent rule (half the heads global, half a 256-key window)
+    ("sliver_every_fourth_key", "causal_softcap_alibi", {"rule": "every_fourth_key"}),
+    ("half_heads_global", "causal_softcap_alibi", {"rule": "half_heads_global"}),
+    # the decode workload against a paged cache: 64-key pages in shuffled order
+    ("decode_kv_cache_paged", "decode_kv_cache", {"paged": 64}),
 ]
+
+# Composed rules of the bench items: (rule spec, reads the query head).
+RULES = {
+    "every_fourth_key": ({"kind": "and", "masks": [{"kind": "causal"}, {"kind": "stride", "value": 4}]}, False),
+    "half_heads_global": ({"kind": "and", "masks": [
+        {"kind": "causal"},
+        {"kind": "or", "masks": [{"kind": "head_below", "value": 8}, {"kind": "distance_below", "value": 256}]}]},
+        True),
+}
 HEADLINE = BENCH_ITEMS[0][0]
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
@@ -80,7 +96,10 @@ KERNEL_SOURCES = {
 
 def config_over(over):
     """A bench item's overrides of the workload config (its mode keys removed)."""
-    return {k: v for k, v in over.items() if k != "backward"}
+    c = {k: v for k, v in over.items() if k not in ("backward", "rule", "paged")}
+    if "rule" in over:
+        c["mask"] = dict(RULES[over["rule"]][0])
+    return c
 
 
 def kernel_source_hash(kind="prefill"):
@@ -116,8 +135,9 @@ def item(label):
 # Work accounting (exact counts from the workload parameters)
 # ---------------------------------------------------------------------------
 
-def visible_counts_rows(c, b, kv_len=None, doc_lengths=None):
-    """Visible keys of every query row of batch b (int64 array of length L)."""
+def visible_counts_rows(c, b, kv_len=None, doc_lengths=None, h=0):
+    """Visible keys of every query row of batch b, query head h (int64 array
+    of length L)."""
     L, S = c["L"], c["S"]
     kind = c["mask"]["kind"]
     S_b = S if kv_len is None else int(kv_len[b])
@@ -133,9 +153,25 @@ def visible_counts_rows(c, b, kv_len=None, doc_lengths=None):
     elif kind == "document":
         starts = np.repeat(np.concatenate([[0], np.cumsum(doc_lengths)[:-1]]), doc_lengths)
         n = q - starts[q] + 1
+    elif c["mask"] == RULES["every_fourth_key"][0]:
+        # keys kv <= q with kv = q (mod 4): q // 4 + 1 of them (S_b = S here)
+        n = np.where(q >= 0, q // 4 + 1, 0)
+    elif c["mask"] == RULES["half_heads_global"][0]:
+        # heads below 8 see every earlier key, the others the last 256
+        n = np.clip(np.minimum(q + 1, S_b), 0, None)
+        if h >= 8:
+            n = np.minimum(n, 256)
     else:
         raise ValueError(kind)
     return n
+
+
+def visible_pairs_all_heads(c, kv_len=None, doc_lengths=None):
+    """Visible pairs over every (b, h); a head-dependent rule counts per head."""
+    if c["mask"] == RULES["half_heads_global"][0]:
+        return sum(int(visible_counts_rows(c, b, kv_len, doc_lengths, h).sum())
+                   for b in range(c["B"]) for h in range(c["Hq"]))
+    return visible_pairs_per_head(c, kv_len, doc_lengths) * c["Hq"]
 
 
 def visible_pairs_per_head(c, kv_len=None, doc_lengths=None):
@@ -291,7 +327,7 @@ class OracleSampler:
         self.rows = c["L"] if self.decode else max(1, min(c["L"], (1 << 21) // c["S"]))
         self.blocks_per_unit = -(-c["L"] // self.rows)
         self.units = c["B"] * c["Hq"]
-        self.counts = [visible_counts_rows(c, b, self.kv_len, self.doc_lengths) for b in range(c["B"])]
+        self.counts = {}
         self.unit_desc = ("one (batch, query head) unit, all its query rows" if self.decode else
                           f"a block of {self.rows} query rows of one (batch, query head) unit, every row in full")
         if backward:
@@ -324,15 +360,22 @@ class OracleSampler:
             t0 = time.perf_counter()
             o.backward_rows(qn, kn, vn, don, c["scale"], self.mask, self.score, b, h, qp, S_b, c["Hq"])
             el = time.perf_counter() - t0
-            return float(self.counts[b][r0:r1].sum()) * (6 * c["E"] + 4 * c["Ev"]), el
+            return float(self.visible(b, h)[r0:r1].sum()) * (6 * c["E"] + 4 * c["Ev"]), el
         t0 = time.perf_counter()
         o.attention_rows(qn, kn, vn, c["scale"], self.mask, self.score, b, h, qp, S_b, c["Hq"])
         el = time.perf_counter() - t0
         if self.decode:
             work = S_b * (c["E"] + c["Ev"]) * 2 / G
         else:
-            work = float(self.counts[b][r0:r1].sum()) * (2 * c["E"] + 2 * c["Ev"])
+            work = float(self.visible(b, h)[r0:r1].sum()) * (2 * c["E"] + 2 * c["Ev"])
         return work, el
+
+    def visible(self, b, h):
+        """Visible keys per query row of unit (b, h) (cached)."""
+        key = (b, h if self.c["mask"] == RULES["half_heads_global"][0] else 0)
+        if key not in self.counts:
+            self.counts[key] = visible_counts_rows(self.c, b, self.kv_len, self.doc_lengths, key[1])
+        return self.counts[key]
 
     def rate(self, target_s):
         """(rate, seconds, samples) running samples until ~target_s of oracle time."""
@@ -435,12 +478,32 @@ class Workload:
          self.doc_lengths) = make_inputs(self.name, dev, seed_offset=rank, batch=batch, **config_over(over))
         c = self.c
         self.B_mask = c["B"] if self.kv_len is not None else 1
+        # a rule that reads the query head needs a block mask per head
+        self.H_mask = c["Hq"] if over.get("rule") and RULES[over["rule"]][1] else 1
         self.gqa = c["Hq"] != c["Hkv"]
         self.q, self.k, self.v = self.q_h.to(dev), self.k_h.to(dev), self.v_h.to(dev)
+        self.paged = None
+        if over.get("paged"):
+            # the cache as a pool of pages in a seeded shuffled order, and its page table
+            P = int(over["paged"])
+            B, Hkv, S = c["B"], c["Hkv"], c["S"]
+            npg = S // P
+            perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(c["seed"] + 7)).to(dev)
+
+            def pool(t):
+                pages = t.view(B, Hkv, npg, P, t.shape[-1]).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, P,
+                                                                                           t.shape[-1])
+                out = torch.empty_like(pages)
+                out[perm] = pages
+                return out
+            self.k, self.v = pool(self.k), pool(self.v)
+            self.k_h, self.v_h = self.k.cpu(), self.v.cpu()  # the host copies the end-to-end leg sends
+            self.paged = {"page_table": perm.view(B, npg).to(torch.int32), "page_size": P}
         self.out = torch.empty((c["B"], c["Hq"], c["L"], c["Ev"]), dtype=self.q.dtype, device=dev)
         self.lse = torch.empty((c["B"], c["Hq"], c["L"]), dtype=torch.float32, device=dev)
-        self.bm = fa.flexattn_build_block_mask(self.mask, self.B_mask, 1, c["L"], c["S"], c["BM"], c["BN"], device=dev)
-        ws = fa.flexattn_forward_workspace_size(self.q, self.k, self.v, self.bm)
+        self.bm = fa.flexattn_build_block_mask(self.mask, self.B_mask, self.H_mask, c["L"], c["S"], c["BM"], c["BN"],
+                                               device=dev)
+        ws = fa.flexattn_forward_workspace_size(self.q, self.k, self.v, self.bm, paged=self.paged)
         self.ws_bytes = ws
         self.ws = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
         self.decode = self.name == "decode_kv_cache"
@@ -448,7 +511,7 @@ class Workload:
         # classifier + forward kernel, + the log-sum-exp combine when decode splits the keys
         self.launches_per_step = 2 + (1 if self.decode and ws > 0 else 0)
         fp = 2 * c["E"] + 2 * c["Ev"]
-        self.vis_flops = visible_pairs_per_head(c, self.kv_len, self.doc_lengths) * c["Hq"] * fp
+        self.vis_flops = visible_pairs_all_heads(c, self.kv_len, self.doc_lengths) * fp
         cells = visited_cells(self.bm) * (c["Hq"] if self.bm.H == 1 else 1) * (c["B"] if self.bm.B == 1 else 1)
         self.visited_cells = cells
         self.visited_flops = cells * fp
@@ -472,12 +535,13 @@ class Workload:
         if self.backward:
             self.fa.flexattn_transpose_block_mask(self.bm, out=self.q_side)
             return
-        self.fa.flexattn_build_block_mask(self.mask, self.B_mask, 1, c["L"], c["S"], c["BM"], c["BN"], out=self.bm)
+        self.fa.flexattn_build_block_mask(self.mask, self.B_mask, self.H_mask, c["L"], c["S"], c["BM"], c["BN"],
+                                          out=self.bm)
 
     def forward_call(self):
         self.fa.flexattn_forward(self.q, self.k, self.v, self.bm, score_mod=self.score, mask_mod=self.mask,
                                  scale=self.c["scale"], enable_gqa=self.gqa, out=self.out, lse=self.lse,
-                                 workspace=self.ws)
+                                 workspace=self.ws, paged=self.paged)
 
     def forward(self):
         """The timed call: the forward, or for a backward item the backward."""

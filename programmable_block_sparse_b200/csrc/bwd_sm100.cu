@@ -21,9 +21,10 @@
 //                    the key-side list: S = Q K^T, dP = dout V^T, then per
 //                    query row dS, then dQ += dS K (TS).
 // Warp roles as in the prefill kernel: warp 0 TMA producer, warp 1 TMEM
-// allocator and MMA issuer (one thread), warps 2-5 one TMEM lane (row) per
-// thread.  TMEM: S at column 0, dP at 128 (P / dS written as bf16 pairs over
-// the columns already read), then the accumulators.  Every mbarrier wait is
+// allocator and MMA issuer (one thread), warps 2-9 the rows, one TMEM lane
+// (row) per thread and two warps per row, each taking half of the columns.
+// TMEM: S at column 0, dP at 128 (P / dS written as bf16 pairs over the
+// columns already read), then the accumulators.  Every mbarrier wait is
 // bounded; a timeout records FA_ERR_TIMEOUT, the producer drains its copies,
 // the MMA thread its MMAs, and the CTA exits.
 #include <math.h>
@@ -37,7 +38,15 @@ namespace fa {
 
 namespace {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
+// Rows of a tile take two warps each (warps 2-9; warp % 4 is the TMEM lane
+// quadrant): math group 0 takes columns 0-63, group 1 columns 64-127, so two
+// warps per SM sub-partition hide each other's latencies.
+constexpr int kMathThreads = 256;
+// TMEM column of the bf16 pairs for keys (or queries) 16 kk .. 16 kk + 15:
+// chunk j = kk / 2 of 32 columns writes its pairs over the first half of its
+// own S columns, which only its own thread has read.
+__device__ __forceinline__ uint32_t pair_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 constexpr int kBT = 128;  // tile rows and columns
 constexpr float kLog2eB = 1.4426950408889634f;
 
@@ -131,7 +140,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars.empty[s], 1);
     }
     mbar_init(&bars.s_full, 2);
-    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.p_full, 8);
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + 256, tbase + kk * 8, dkmn0 + s * kStep + ((kk * 16 * 128) >> 4), idesc_dq,
+          umma_ts(tbase + 256, tbase + pair_col(kk), dkmn0 + s * kStep + ((kk * 16 * 128) >> 4), idesc_dq,
                   (u > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bars.empty[s]);
       }
@@ -209,6 +218,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ rows
     const int quad = warp & 3;
+    const int jg = (warp - 2) >> 2;  // math group: column chunks 2 jg, 2 jg + 1
     const int r = quad * 32 + lane;
     const int grow = mt * kBT + r;
     const bool row_ok = grow < a.L;
@@ -242,12 +252,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool edge = kv0 + kBT > S_b;
       const bool stage_doc = is_doc && (!full || edge);
       if (group_stage) {
-        if (ok) {
+        if (ok && jg == 0) {
           const int kv = kv0 + r;
           if (has_pos) s_pos[cnt & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
           if (stage_doc) s_doc[cnt & 1][r] = kv < a.S ? __ldg(doc_row + kv) : 0;
         }
-        ok = named_bar_and(1, 128, ok);
+        ok = named_bar_and(1, kMathThreads, ok);
       }
       if (!ok) {
         alive = false;
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const bool need_mask = !full || edge || !row_ok;
 #pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 2 * jg; j < 2 * jg + 2; ++j) {
         uint32_t sr[32], dp[32];
         tmem_ld16(tbase + lane_base + 32 * j, *reinterpret_cast<uint32_t(*)[16]>(sr));
         tmem_ld16(tbase + lane_base + 32 * j + 16, *reinterpret_cast<uint32_t(*)[16]>(sr + 16));
@@ -301,7 +311,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[i >> 1] = pack_bf16x2(ds2[0], ds2[1]);
         }
         // dS of these 32 keys as bf16 pairs over S columns already read
-        tmem_st16(tbase + lane_base + 16 * j, pk);
+        tmem_st16(tbase + lane_base + 32 * j, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (__all_sync(0xffffffffu, alive)) {
       const int64_t off = b * a.dq_stride[0] + h * a.dq_stride[1] + static_cast<int64_t>(row_ok ? grow : 0) * a.dq_stride[2];
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = jg * (D / 32); c < (jg + 1) * (D / 32); ++c) {
         uint32_t rr[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) rr[i] = 0u;
@@ -422,7 +432,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars.empty[s], 1);
     }
     mbar_init(&bars.s_full, 2);
-    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.p_full, 8);
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
@@ -494,8 +504,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
           const uint32_t boff = s * kStep + ((kk * 16 * 128) >> 4);
-          umma_ts(tbase + 256, tbase + kk * 8, ddomn0 + boff, idesc_acc, acc);            // dV += P^T dout
-          umma_ts(tbase + 256 + D, tbase + 128 + kk * 8, dqmn0 + boff, idesc_acc, acc);   // dK += dS^T Q
+          umma_ts(tbase + 256, tbase + pair_col(kk), ddomn0 + boff, idesc_acc, acc);          // dV += P^T dout
+          umma_ts(tbase + 256 + D, tbase + 128 + pair_col(kk), dqmn0 + boff, idesc_acc, acc); // dK += dS^T Q
         }
         umma_commit(&bars.empty[s]);
       }
@@ -506,6 +516,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ key rows
     const int quad = warp & 3;
+    const int jg = (warp - 2) >> 2;  // math group: column chunks 2 jg, 2 jg + 1
     const int r = quad * 32 + lane;
     const int kv = n * kBT + r;
     const bool key_ok = kv < S_b;
@@ -531,9 +542,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int g = ok ? bars.info_h[cnt & 1] : 0;
       const int h = hk * a.G + g;
       // the tile's query-side values (lse, D, positions, documents) into smem,
-      // double-buffered by cnt & 1; the group barrier also tells every warp
-      // whether all four got their S, so a timeout is left together
-      if (ok) {
+      // double-buffered by cnt & 1 (math group 0 writes them); the barrier
+      // also tells every warp whether all eight got their S, so a timeout is
+      // left together
+      if (ok && jg == 0) {
         const int i = mq * kBT + r;
         const int64_t rid = (static_cast<int64_t>(b) * a.Hq + h) * a.L + i;
         const float l = i < a.L ? a.lse[rid] : -INFINITY;
@@ -543,7 +555,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (has_pos) s_pq[cnt & 1][r] = static_cast<float>(pos_at(a.score, b, q, a.S));
         if (is_doc) s_doc[cnt & 1][r] = (q >= 0 && q < a.S && i < a.L) ? __ldg(doc_row + q) : 0;
       }
-      ok = named_bar_and(1, 128, ok);
+      ok = named_bar_and(1, kMathThreads, ok);
       if (!ok) {
         alive = false;
         break;
@@ -554,7 +566,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool edge = i0 + kBT > a.L || n * kBT + kBT > S_b;
       const bool need_mask = !full || edge || !key_ok;
 #pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 2 * jg; j < 2 * jg + 2; ++j) {
         uint32_t sr[32], dp[32];
         tmem_ld16(tbase + lane_base + 32 * j, *reinterpret_cast<uint32_t(*)[16]>(sr));
         tmem_ld16(tbase + lane_base + 32 * j + 16, *reinterpret_cast<uint32_t(*)[16]>(sr + 16));
@@ -600,8 +612,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dpk[i >> 1] = pack_bf16x2(d2[0], d2[1]);
         }
         // P^T and dS^T of these 32 queries as bf16 pairs over columns already read
-        tmem_st16(tbase + lane_base + 16 * j, ppk);
-        tmem_st16(tbase + lane_base + 128 + 16 * j, dpk);
+        tmem_st16(tbase + lane_base + 32 * j, ppk);
+        tmem_st16(tbase + lane_base + 128 + 32 * j, dpk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -616,8 +628,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (__all_sync(0xffffffffu, alive)) {
       const bool row_ok = kv < a.S;
       const int kvr = row_ok ? kv : 0;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+      {
+        const int which = jg;  // math group 0 writes dV, group 1 dK
         void* base = which ? a.dk : a.dv;
         const int64_t* st = which ? a.dk_stride : a.dv_stride;
         const bool f32 = which ? a.dk_f32 : a.dv_f32;

@@ -566,6 +566,31 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   };
   auto row_head = [&](int r) { return hk * a.G + hc * p.heads_per_cta + r / a.L; };
 
+  // K (u even) or V (u odd) of tile u / 2 into ring entry u % R
+  auto issue_load = [&](int u) {
+    const int e = u % R, j = u >> 1;
+    const int n = list_tile(a, brow, nfull, t0 + j / subs);
+    const int kv0 = n * a.bm.BN + (j % subs) * kTcKeys;
+    const CUtensorMap* map = (u & 1) ? &map_v : &map_k;
+    uint8_t* dst = sKV + e * C::kEntryBytes;
+    mbar_expect_tx(&bars.full[e], C::kEntryBytes);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      // two 64-key boxes per tile; a paged cache keeps each in one page
+      int row = kv0 + 64 * h2, outer = b;
+      if (a.page_table) {
+        outer = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, row);
+        row = row % a.page_size;
+      }
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_4d(dst + c * (kTcKeys * 128) + h2 * (64 * 128), map, &bars.full[e], c * 64, row, hk, outer);
+    }
+  };
+  // The first R copies need no free entry: thread 0 (the producer) issues
+  // them right after initialising the barriers, so they are in flight while
+  // the CTA stages Q and allocates TMEM.
+  const int first_loads = min(R, 2 * nsub);
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(&bars.full[s], 1);
@@ -580,6 +605,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
+    if (nsub > 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+    }
+    for (int u = 0; u < first_loads; ++u) issue_load(u);
   }
   if (threadIdx.x < kTcRows) {
     const int r = threadIdx.x;
@@ -614,30 +644,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0 && nsub > 0) {
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
-      int issued = 0;
-      for (int u = 0; u < 2 * nsub && !*abort; ++u) {
-        const int e = u % R;
-        if (u >= R && !mbar_wait(&bars.empty[e], ((u / R) - 1) & 1, abort, a.status, a.wait_cycles)) break;
-        const int j = u >> 1;
-        const int n = list_tile(a, brow, nfull, t0 + j / subs);
-        const int kv0 = n * a.bm.BN + (j % subs) * kTcKeys;
-        const CUtensorMap* map = (u & 1) ? &map_v : &map_k;
-        uint8_t* dst = sKV + e * C::kEntryBytes;
-        mbar_expect_tx(&bars.full[e], C::kEntryBytes);
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          // two 64-key boxes per tile; a paged cache keeps each in one page
-          int row = kv0 + 64 * h2, outer = b;
-          if (a.page_table) {
-            outer = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, row);
-            row = row % a.page_size;
-          }
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(dst + c * (kTcKeys * 128) + h2 * (64 * 128), map, &bars.full[e], c * 64, row, hk, outer);
-        }
+      int issued = first_loads;
+      for (int u = first_loads; u < 2 * nsub && !*abort; ++u) {
+        if (!mbar_wait(&bars.empty[u % R], ((u / R) - 1) & 1, abort, a.status, a.wait_cycles)) break;
+        issue_load(u);
         issued = u + 1;
       }
       // every copy issued lands before this thread leaves (only the last R

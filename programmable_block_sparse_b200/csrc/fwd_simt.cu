@@ -47,11 +47,16 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
   const int t = threadIdx.x;
   const int BM = a.bm.BM, BN = a.bm.BN;
   const int E = a.E, Ev = a.Ev;
+  // R threads per query row (R = 128 / BM, at least 1): thread t takes row
+  // t % BM and the keys j = sub (mod R) of every chunk, sub = t / BM; the R
+  // partial (max, sum, O) of a row are merged at the end.
+  const int R = BM >= kSimtThreads ? 1 : kSimtThreads / BM;
   const int qst = E | 1, ost = Ev | 1;  // odd row strides: no bank conflicts across rows
   float* sq = smem;
-  float* so = sq + BM * qst;
-  float* sk = so + BM * ost;
+  float* so = sq + BM * qst;             // [R][BM] partial O rows
+  float* sk = so + R * BM * ost;
   float* sv = sk + kChunk * E;
+  float* sml = sv + kChunk * Ev;          // [R][BM] partial max, then [R][BM] partial sum
 
   const int hk = h / a.G;
   const int S = a.S, L = a.L;
@@ -65,10 +70,13 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
     const int r = i / E, e = i % E;
     sq[r * qst + e] = (r0 + r < L) ? to_f(qb[(r0 + r) * a.q_stride[2] + e]) : 0.0f;
   }
-  for (int i = t; i < BM * Ev; i += blockDim.x) so[(i / Ev) * ost + i % Ev] = 0.0f;
+  for (int i = t; i < R * BM * Ev; i += blockDim.x) so[(i / Ev) * ost + i % Ev] = 0.0f;
 
-  const int row = r0 + t;
-  const bool active = t < BM && row < L;
+  const int rr = t % BM, sub = t / BM;
+  const int row = r0 + rr;
+  const bool active = sub < R && row < L;
+  float* orow = so + (sub * BM + rr) * ost;
+  const float* qrow = sq + rr * qst;
   const int qpos = query_pos(row, L, S_b);
   const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
   const float slope = distance_slope(h, Hs);
@@ -110,64 +118,89 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
       }
       __syncthreads();
       if (!active) continue;
+      // this thread's keys of the chunk: j = sub, sub + R, ...
+      const int mine = nk > sub ? (nk - sub + R - 1) / R : 0;
       float s[kChunk];
       float cmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kChunk; ++j) {
-        float val = -INFINITY;
-        if (j < nk) {
-          float dot = 0.0f;
-          for (int e = 0; e < E; ++e) dot = fmaf(sq[t * qst + e], sk[j * E + e], dot);
-          const int kv = cc + j;
-          const float g = score_apply<true>(a.score, dot * a.scale, b, qpos, kv, S, slope);
-          const bool vis = is_full ? (kv < S_b) : mask_visible(a.mask, b, h, qpos, kv, S_b, S);
-          val = vis ? g : -INFINITY;
+      for (int u = 0; u < kChunk; ++u) {
+        s[u] = -INFINITY;
+        if (u >= mine) continue;
+        const int j = sub + u * R;
+        const float* krow = sk + j * E;
+        float d0 = 0.0f, d1 = 0.0f, d2 = 0.0f, d3 = 0.0f;  // four chains
+        int e = 0;
+        for (; e + 4 <= E; e += 4) {
+          d0 = fmaf(qrow[e], krow[e], d0);
+          d1 = fmaf(qrow[e + 1], krow[e + 1], d1);
+          d2 = fmaf(qrow[e + 2], krow[e + 2], d2);
+          d3 = fmaf(qrow[e + 3], krow[e + 3], d3);
         }
-        s[j] = val;
-        cmax = fmaxf(cmax, val);
+        for (; e < E; ++e) d0 = fmaf(qrow[e], krow[e], d0);
+        const float dot = (d0 + d1) + (d2 + d3);
+        const int kv = cc + j;
+        const float g = score_apply<true>(a.score, dot * a.scale, b, qpos, kv, S, slope);
+        const bool vis = is_full ? (kv < S_b) : mask_visible(a.mask, b, h, qpos, kv, S_b, S);
+        s[u] = vis ? g : -INFINITY;
+        cmax = fmaxf(cmax, s[u]);
       }
       const float m_new = fmaxf(m_run, cmax);
       const float alpha = expf(m_run - m_new);
       float psum = 0.0f;
 #pragma unroll
-      for (int j = 0; j < kChunk; ++j) {
-        s[j] = expf(s[j] - m_new);
-        psum += s[j];
+      for (int u = 0; u < kChunk; ++u) {
+        s[u] = u < mine ? expf(s[u] - m_new) : 0.0f;
+        psum += s[u];
       }
       l_run = l_run * alpha + psum;
       for (int d = 0; d < Ev; ++d) {
-        float acc = so[t * ost + d] * alpha;
+        float acc[2] = {orow[d] * alpha, 0.0f};
 #pragma unroll
-        for (int j = 0; j < kChunk; ++j) acc = fmaf(s[j], (j < nk) ? sv[j * Ev + d] : 0.0f, acc);
-        so[t * ost + d] = acc;
+        for (int u = 0; u < kChunk; ++u)
+          if (u < mine) acc[u & 1] = fmaf(s[u], sv[(sub + u * R) * Ev + d], acc[u & 1]);
+        orow[d] = acc[0] + acc[1];
       }
       m_run = m_new;
     }
   }
-  if (!active) return;
+  // merge the R partials of each row: thread sub 0 of the row writes it
+  __syncthreads();
+  if (sub < R) {
+    sml[sub * BM + rr] = m_run;
+    sml[(R + sub) * BM + rr] = l_run;
+  }
+  __syncthreads();
+  if (!active || sub != 0) return;
+  float m = sml[rr];
+  for (int r = 1; r < R; ++r) m = fmaxf(m, sml[r * BM + rr]);
+  float l = 0.0f;
+  for (int r = 0; r < R; ++r) l += sml[(R + r) * BM + rr] * expf(sml[r * BM + rr] - m);
   const int64_t ooff = b * a.o_stride[0] + h * a.o_stride[1] + row * a.o_stride[2];
-  // a row without a visible key has l_run = 0: out 0 and lse -inf, unless the
+  // a row without a visible key has l = 0: out 0 and lse -inf, unless the
   // caller promised there is none (rows_safe), which drops this guard
-  const bool live = a.rows_safe || l_run > 0.0f;
-  const float inv = live ? 1.0f / l_run : 0.0f;
-  if (a.out_f32) {
-    float* ob = static_cast<float*>(a.out) + ooff;
-    for (int d = 0; d < Ev; ++d) ob[d] = live ? so[t * ost + d] * inv : 0.0f;
-  } else {
-    T* ob = static_cast<T*>(a.out) + ooff;
-    for (int d = 0; d < Ev; ++d) store_out<T>(ob + d, live ? so[t * ost + d] * inv : 0.0f);
+  const bool live = a.rows_safe || l > 0.0f;
+  const float inv = live ? 1.0f / l : 0.0f;
+  for (int d = 0; d < Ev; ++d) {
+    float o = 0.0f;
+    for (int r = 0; r < R; ++r) o += so[(r * BM + rr) * ost + d] * expf(sml[r * BM + rr] - m);
+    const float val = live ? o * inv : 0.0f;
+    if (a.out_f32)
+      static_cast<float*>(a.out)[ooff + d] = val;
+    else
+      store_out<T>(static_cast<T*>(a.out) + ooff + d, val);
   }
   const int64_t rid = (static_cast<int64_t>(b) * a.Hq + h) * L + row;
-  if (a.lse) a.lse[rid] = live ? m_run + logf(l_run) : -INFINITY;
-  if (a.max_scores) a.max_scores[rid] = m_run > kNoKeyMaxS ? m_run : -INFINITY;  // the exact running maximum
+  if (a.lse) a.lse[rid] = live ? m + logf(l) : -INFINITY;
+  if (a.max_scores) a.max_scores[rid] = m > kNoKeyMaxS ? m : -INFINITY;  // the exact running maximum
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream) {
   const int BM = a.bm.BM;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(BM) * ((a.E | 1) + (a.Ev | 1)) +
-                                       static_cast<size_t>(kChunk) * (a.E + a.Ev));
+  const int R = BM >= kSimtThreads ? 1 : kSimtThreads / BM;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(BM) * ((a.E | 1) + R * (a.Ev | 1)) +
+                                       static_cast<size_t>(kChunk) * (a.E + a.Ev) + 2 * R * BM);
   dim3 grid(a.bm.Mb, a.Hq, a.B);
   cudaError_t e;
   if (a.dtype == FA_DTYPE_F32) {

@@ -66,5 +66,22 @@ def test_backward_items_and_their_oracle_sample():
     work, el = s.block(0)
     c = s.c
     b, h = divmod(0, c["Hq"])
-    assert work == float(s.counts[b][:s.rows].sum()) * (6 * c["E"] + 4 * c["Ev"])
+    assert work == float(s.visible(b, h)[:s.rows].sum()) * (6 * c["E"] + 4 * c["Ev"])
     assert el > 0
+
+
+def test_composed_rule_counts():
+    """The bench's closed forms for its composed-rule items (a sliver of every
+    fourth key; half the heads global, half a 256-key window) against the
+    oracle's visibility, head by head."""
+    for label in ("sliver_every_fourth_key", "half_heads_global"):
+        _, name, over = bench.item(label)
+        c = wl.config(name, **bench.config_over(over), B=2, L=700, S=700, Hq=16, Hkv=16)
+        want = 0
+        for b in range(c["B"]):
+            for h in range(c["Hq"]):
+                vis = o.visible(c["mask"], b, h, o.query_positions(c["L"], c["S"]), np.arange(c["S"]), c["S"])
+                got = bench.visible_counts_rows(c, b, h=h)
+                assert np.array_equal(got, vis.sum(axis=1)), (label, b, h)
+                want += int(vis.sum())
+        assert bench.visible_pairs_all_heads(c) == want
