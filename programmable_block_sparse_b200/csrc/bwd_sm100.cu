@@ -74,13 +74,32 @@ constexpr int kInfoFullB = 1 << 30;
 // (tanh_poly2, error under 1.5e-6 relative), else 1 - 2 / (e^{2|y|} + 1)
 // with its sign.  The gradients sum P and dg/ds = 1 - tanh^2 over many cells
 // whose products partly cancel, so the hardware tanh's relative error of
-// about 2^-11 would show in them; both forms are computed and one selected.
-__device__ __forceinline__ float tanh_acc(float y) {
-  float2 u;
-  const float p = tanh_poly2(make_float2(y, y), u).x;
+// about 2^-11 would show in them.
+__device__ __forceinline__ float tanh_big(float y) {
   const float e = ex2_approx(2.0f * kLog2eB * fminf(fabsf(y), 15.0f));  // tanh(15) is 1 in fp32
-  const float big = copysignf(1.0f - __fdividef(2.0f, e + 1.0f), y);
-  return fabsf(y) <= kTanhPolyMax ? p : big;
+  return copysignf(1.0f - __fdividef(2.0f, e + 1.0f), y);
+}
+// tanh(s c_in) of 32 raw scores: the series on the FMA pipe; the exponential
+// form only for arguments beyond kTanhPolyMax, and only when some lane of
+// the warp has one, so the common case issues no MUFU operation for it.
+__device__ __forceinline__ void tanh32(const uint32_t (&sr)[32], float c_in, float (&th)[32]) {
+  float umax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    float2 u;
+    const float2 v =
+        tanh_poly2(make_float2(__uint_as_float(sr[i]) * c_in, __uint_as_float(sr[i + 1]) * c_in), u);
+    th[i] = v.x;
+    th[i + 1] = v.y;
+    umax = max3f(umax, u.x, u.y);
+  }
+  if (__any_sync(0xffffffffu, !(umax <= kTanhPolyMax * kTanhPolyMax))) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float y = __uint_as_float(sr[i]) * c_in;
+      if (!(fabsf(y) <= kTanhPolyMax)) th[i] = tanh_big(y);
+    }
+  }
 }
 
 // Loads tiles into smem boxes of 64 columns x 128 rows (128-byte swizzle).
@@ -90,11 +109,11 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
   for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (kBT * 128), map, bar, c * 64, row, h, b);
 }
 
-// Score rule in log2 units and its slope dg/ds for one cell.
+// Score rule in log2 units and its slope dg/ds for one cell; th is
+// tanh(s c_in) under a soft-cap (unused otherwise).
 template <int SCORE>
-__device__ __forceinline__ void score_and_slope(float s, float c_in, float c_out, float bias, float& t, float& gp) {
+__device__ __forceinline__ void score_and_slope(float s, float th, float c_out, float bias, float& t, float& gp) {
   if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) {
-    const float th = tanh_acc(s * c_in);
     t = fmaf(c_out, th, bias);
     gp = fmaf(-th, th, 1.0f);
   } else {
@@ -292,6 +311,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float bias0 = (SCORE == FA_SCORE_ALIBI || (SCORE == FA_SCORE_CAP_THEN_BIAS && !has_pos))
                                 ? slope2 * static_cast<float>(base - qpos) : 0.0f;
+        float th[32];
+        if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) tanh32(sr, c_in, th);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -304,7 +325,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
               bias = has_pos ? s_pos[cnt & 1][32 * j + c] - pq_scaled : fmaf(slope2, static_cast<float>(c), bias0);
             float t, gp;
-            score_and_slope<SCORE>(__uint_as_float(sr[c]), c_in, c_out, bias, t, gp);
+            score_and_slope<SCORE>(__uint_as_float(sr[c]), th[c], c_out, bias, t, gp);
             const float p = ((bits >> c) & 1u) ? ex2_approx(t - lse2) : 0.0f;
             ds2[e] = p * (__uint_as_float(dp[c]) - dsum) * gp;
           }
@@ -591,6 +612,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float* lq = s_lse[cnt & 1] + 32 * j;
         const float* dq = s_dsum[cnt & 1] + 32 * j;
         const float bias0 = slope2 * static_cast<float>(kv - qbase);  // slope2 (kv - q) at c = 0
+        float th[32];
+        if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) tanh32(sr, c_in, th);
         uint32_t ppk[16], dpk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -603,7 +626,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
               bias = has_pos ? slope2 * (pk_raw - s_pq[cnt & 1][32 * j + c]) : fmaf(-slope2, static_cast<float>(c), bias0);
             float t, gp;
-            score_and_slope<SCORE>(__uint_as_float(sr[c]), c_in, c_out, bias, t, gp);
+            score_and_slope<SCORE>(__uint_as_float(sr[c]), th[c], c_out, bias, t, gp);
             const float p = ((bits >> c) & 1u) ? ex2_approx(t - lq[c]) : 0.0f;
             p2[e] = p;
             d2[e] = p * (__uint_as_float(dp[c]) - dq[c]) * gp;

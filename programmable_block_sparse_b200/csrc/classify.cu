@@ -8,10 +8,11 @@
 // "flexattention-score-mod-block-mask" (charlestar.github.io), section
 // "mask_mod defines legal connections, BlockMask defines block work".
 //
-// How: no dense (L, S) temporary.  One CTA per (b, m) row of tiles; each warp
-// classifies whole tiles.  For the interval-shaped rules (none, causal,
-// sliding window with sinks, prefix-LM, chunked) every query row sees a union
-// of at most two key intervals, so a tile is classified from per-row
+// How: no dense (L, S) temporary.  One CTA per (b, m) row of tiles (and per
+// head for a rule that reads the head); each warp classifies whole tiles.
+// For the interval-shaped rules (none, causal, sliding window with sinks,
+// prefix-LM, chunked) every query row sees a union of at most two key
+// intervals, so a tile is classified from per-row
 // intersection counts (BM work per tile instead of BM x BN).  The document
 // rule counts the same way over runs of equal document id (see
 // classify_tile_document).  A composed rule (FA_MASK_PROGRAM) is decided per
@@ -171,11 +172,13 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs
   const bool causal_family = a.mask.kind == FA_MASK_CAUSAL || a.mask.kind == FA_MASK_SLIDING_WINDOW ||
                              a.mask.kind == FA_MASK_DOCUMENT || a.mask.kind == FA_MASK_CHUNKED;
 
-  // a rule that reads the query head is classified for each head row; any
-  // other is classified once and its lists written to every head row
+  // a rule that reads the query head is classified for each head row (one
+  // CTA per head: blockIdx.z); any other is classified once and its lists
+  // written to every head row
   const bool per_head = a.mask.kind == FA_MASK_PROGRAM && a.mask.reads_head && a.H > 1;
   __shared__ int s_counts[2];
-  for (int hc = 0; hc < (per_head ? a.H : 1); ++hc) {
+  {
+    const int hc = per_head ? static_cast<int>(blockIdx.z) : 0;
     for (int n = warp; n < a.Nb; n += nwarps) {
       const int c0 = n * a.BN;
       const int c1 = min(a.S, c0 + a.BN) - 1;        // inclusive
@@ -230,14 +233,14 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs
         if (i >= npart) a.kv_indices[row * a.Nb + i] = 0;
       }
     }
-    __syncthreads();  // cls and s_counts are rewritten for the next head
   }
 }
 
 }  // namespace
 
 cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream) {
-  dim3 grid(a.Mb, a.B);
+  const bool per_head = a.mask.kind == FA_MASK_PROGRAM && a.mask.reads_head && a.H > 1;
+  dim3 grid(a.Mb, a.B, per_head ? a.H : 1);
   size_t smem = (static_cast<size_t>(a.Nb) + 15) & ~static_cast<size_t>(15);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

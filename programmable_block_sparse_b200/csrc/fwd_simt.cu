@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
   float* sk = so + R * BM * ost;
   float* sv = sk + kChunk * E;
   float* sml = sv + kChunk * Ev;          // [R][BM] partial max, then [R][BM] partial sum
+  float* ss = sml + 2 * R * BM;           // [128][kChunk + 1] each thread's chunk scores
 
   const int hk = h / a.G;
   const int S = a.S, L = a.L;
@@ -120,16 +121,18 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
       if (!active) continue;
       // this thread's keys of the chunk: j = sub, sub + R, ...
       const int mine = nk > sub ? (nk - sub + R - 1) / R : 0;
-      float s[kChunk];
+      // the scores live in shared memory, so the loops stay rolled (this
+      // kernel is bound by latency, and unrolled it overflows the
+      // instruction cache)
+      float* s = ss + t * (kChunk + 1);
       float cmax = -INFINITY;
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        s[u] = -INFINITY;
-        if (u >= mine) continue;
+#pragma unroll 1
+      for (int u = 0; u < mine; ++u) {
         const int j = sub + u * R;
         const float* krow = sk + j * E;
         float d0 = 0.0f, d1 = 0.0f, d2 = 0.0f, d3 = 0.0f;  // four chains
         int e = 0;
+#pragma unroll 1
         for (; e + 4 <= E; e += 4) {
           d0 = fmaf(qrow[e], krow[e], d0);
           d1 = fmaf(qrow[e + 1], krow[e + 1], d1);
@@ -147,18 +150,22 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
       const float m_new = fmaxf(m_run, cmax);
       const float alpha = expf(m_run - m_new);
       float psum = 0.0f;
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        s[u] = u < mine ? expf(s[u] - m_new) : 0.0f;
+#pragma unroll 1
+      for (int u = 0; u < mine; ++u) {
+        s[u] = expf(s[u] - m_new);
         psum += s[u];
       }
       l_run = l_run * alpha + psum;
       for (int d = 0; d < Ev; ++d) {
-        float acc[2] = {orow[d] * alpha, 0.0f};
-#pragma unroll
-        for (int u = 0; u < kChunk; ++u)
-          if (u < mine) acc[u & 1] = fmaf(s[u], sv[(sub + u * R) * Ev + d], acc[u & 1]);
-        orow[d] = acc[0] + acc[1];
+        float acc0 = orow[d] * alpha, acc1 = 0.0f;
+        int u = 0;
+#pragma unroll 1
+        for (; u + 2 <= mine; u += 2) {
+          acc0 = fmaf(s[u], sv[(sub + u * R) * Ev + d], acc0);
+          acc1 = fmaf(s[u + 1], sv[(sub + (u + 1) * R) * Ev + d], acc1);
+        }
+        if (u < mine) acc0 = fmaf(s[u], sv[(sub + u * R) * Ev + d], acc0);
+        orow[d] = acc0 + acc1;
       }
       m_run = m_new;
     }
@@ -200,7 +207,8 @@ cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream) {
   const int BM = a.bm.BM;
   const int R = BM >= kSimtThreads ? 1 : kSimtThreads / BM;
   const size_t smem = sizeof(float) * (static_cast<size_t>(BM) * ((a.E | 1) + R * (a.Ev | 1)) +
-                                       static_cast<size_t>(kChunk) * (a.E + a.Ev) + 2 * R * BM);
+                                       static_cast<size_t>(kChunk) * (a.E + a.Ev) + 2 * R * BM +
+                                       static_cast<size_t>(kSimtThreads) * (kChunk + 1));
   dim3 grid(a.bm.Mb, a.Hq, a.B);
   cudaError_t e;
   if (a.dtype == FA_DTYPE_F32) {

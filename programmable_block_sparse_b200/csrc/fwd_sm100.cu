@@ -196,18 +196,6 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   }
   const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
   const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
-  // c log2(e) tanh(s c_in) as an odd polynomial in the raw score s:
-  // s (k1 + v (k3 + v (k5 + v k7))), v = s^2, k_n = c log2(e) c_in^n c_n with
-  // the series' coefficients c_n; it holds while |s c_in| <= kTanhPolyMax,
-  // that is v <= v_lim.  (A cap so small that c_in^7 could overflow always
-  // takes the hardware tanh.)
-  const bool poly_ok = c_in <= 1.0e4f;
-  const float ci2 = c_in * c_in;
-  const float k1 = poly_ok ? c_out * c_in : 0.0f;
-  const float k3 = poly_ok ? k1 * ci2 * kTanhC3 : 0.0f;
-  const float k5 = poly_ok ? k1 * ci2 * ci2 * kTanhC5 : 0.0f;
-  const float k7 = poly_ok ? k1 * ci2 * ci2 * ci2 * kTanhC7 : 0.0f;
-  const float v_lim = poly_ok ? (kTanhPolyMax * kTanhPolyMax) / ci2 : -1.0f;
   const bool is_prog = a.mask.kind == FA_MASK_PROGRAM;
   // document ids are staged for the document rule and for composed rules
   // that compare documents
@@ -284,39 +272,39 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
           t2[i] = fma2(t2[i], splat2(c_out), fma2(splat2(slope2), col, b0));
         }
       } else {
-        // soft-cap on the FMA pipe: the odd polynomial in s above, then the
-        // bias; a half whose largest |s c_in| is beyond kTanhPolyMax is redone
-        // with the hardware tanh
-        // bias of pair i: -m_fold, plus slope2 (p[kv] - p[q]) (p[kv] staged
-        // in smem) or slope2 (kv - q) under cap-then-bias
-        const float2* pk = reinterpret_cast<const float2*>(s_pos[cnt & 1] + c0);
-        const float2 bq = splat2(has_pos ? -pq_scaled - m_fold : -m_fold);
-        const float2 b0 = splat2(slope2 * static_cast<float>(kv0 + c0 - qpos) - m_fold);
-        auto bias = [&](int i) -> float2 {
-          if constexpr (SCORE == FA_SCORE_SOFTCAP) return bq;
-          if (has_pos) return add2(pk[i], bq);
-          return fma2(splat2(slope2),
-                      make_float2(static_cast<float>(2 * i), static_cast<float>(2 * i + 1)), b0);
-        };
-        float vmax = 0.0f;
+        // soft-cap on the FMA pipe: c tanh(s / c) with tanh's odd series,
+        // exact enough for |s / c| <= kTanhPolyMax; a half whose largest
+        // argument is beyond that is redone with the hardware tanh
+        float2* th = t2;  // tanh(s / c), computed in place
+        float umax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float2 v0 = mul2(t2[i], t2[i]), v1 = mul2(t2[i + 1], t2[i + 1]);
-          float2 p0 = fma2(v0, splat2(k7), splat2(k5)), p1 = fma2(v1, splat2(k7), splat2(k5));
-          p0 = fma2(v0, p0, splat2(k3));
-          p1 = fma2(v1, p1, splat2(k3));
-          p0 = fma2(v0, p0, splat2(k1));
-          p1 = fma2(v1, p1, splat2(k1));
-          vmax = max3f(vmax, fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y));
-          t2[i] = fma2(t2[i], p0, bias(i));
-          t2[i + 1] = fma2(t2[i + 1], p1, bias(i + 1));
+          float2 u0, u1;
+          th[i] = tanh_poly2(mul2(t2[i], splat2(c_in)), u0);
+          th[i + 1] = tanh_poly2(mul2(t2[i + 1], splat2(c_in)), u1);
+          umax = max3f(umax, fmaxf(u0.x, u0.y), fmaxf(u1.x, u1.y));
         }
-        if (__any_sync(0xffffffffu, !(vmax <= v_lim))) {
+        if (__any_sync(0xffffffffu, !(umax <= kTanhPolyMax * kTanhPolyMax))) {
           // rare: reload the raw scores (still in TMEM) for the hardware tanh
           tanh_hw_tmem(tbase + lane_base + col_s + c0, c_in);
           tmem_load64(tbase + lane_base + col_s + c0, t);
+        }
+        if constexpr (SCORE == FA_SCORE_SOFTCAP) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) t2[i] = fma2(t2[i], splat2(c_out), bias(i));
+          for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), splat2(-m_fold));
+        } else if (has_pos) {
+          // bias of column c: slope2 (p[kv] - p[q]) - m_fold, p[kv] staged in smem
+          const float2* pk = reinterpret_cast<const float2*>(s_pos[cnt & 1] + c0);
+          const float2 b0 = splat2(-pq_scaled - m_fold);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), add2(pk[i], b0));
+        } else {
+          const float2 b0 = splat2(slope2 * static_cast<float>(kv0 + c0 - qpos) - m_fold);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 col = make_float2(static_cast<float>(2 * i), static_cast<float>(2 * i + 1));
+            t2[i] = fma2(th[i], splat2(c_out), fma2(splat2(slope2), col, b0));
+          }
         }
       }
       if (need_mask) {
