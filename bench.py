@@ -84,7 +84,23 @@ HEADLINE = BENCH_ITEMS[0][0]
 # label; valid only while that kernel's sources hash to the recorded value
 # (the hash ignores comments).  The scaling of each capture to the full
 # workload is stated in the profile it comes from.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # fwd_sm100_kernel<128, 0>, captured at batch 1 (profiles/fwd_sm100_gqa_sliding_window.md): x 2 sequences
+    "gqa_sliding_window": {"bytes": 2 * (201787392 + 96543232), "source_hash": "e9e8eb8d91dff766"},
+    # fwd_sm100_kernel<64, 3> / <128, 3>, full size (profiles/fwd_sm100_causal_packed_sliver.md)
+    "causal_softcap_alibi": {"bytes": 50412800 + 1033472, "source_hash": "e9e8eb8d91dff766"},
+    "packed_docs": {"bytes": 100861696 + 12390656, "source_hash": "e9e8eb8d91dff766"},
+    "sliver_every_fourth_key": {"bytes": 50420480 + 708864, "source_hash": "e9e8eb8d91dff766"},
+    # decode_tc_kernel<128, 1>, captured at batch 16 (profiles/decode_tc_kernel_decode_kv_cache.md):
+    # x 614602 / 296926 cached tokens
+    "decode_kv_cache": {"bytes": round((1221946880 + 8642816) * 614602 / 296926), "source_hash": "e054904aaeb2d24a"},
+    "decode_kv_cache_q1": {"bytes": round((1220857344 + 4764928) * 614602 / 296926),
+                           "source_hash": "e054904aaeb2d24a"},
+    # bwd_dkdv_kernel (the larger of the two backward kernels), full size
+    # (profiles/bwd_dkdv_dq_backward.md)
+    "backward_causal_softcap_alibi": {"bytes": 69195776 + 7536896, "source_hash": "11fa386a7150b63d"},
+    "backward_packed_docs": {"bytes": 136113152 + 37091328, "source_hash": "11fa386a7150b63d"},
+}
 
 KERNEL_SOURCES = {
     "prefill": ("fwd_sm100.cu", "mods.cuh", "common.cuh", "fastmath.cuh"),

@@ -44,6 +44,17 @@ design notes too):
 * ALiBi / distance slope for head h is 2^(-8 (h + 1) / H), h from 0.
 * Tiles at a ragged edge are classified over their in-range cells only.
   Index lists are ascending; unused slots hold 0.
+* max_scores (the guide's per-row maximum, section 2) is the largest
+  transformed score among the visible keys, in lse's units; -inf for a row
+  with no visible key.
+* Composed rules (guide section 4.3, and_masks / or_masks; "Attention
+  expressions", Examples): the predicates carry no causal bound of their own;
+  same-chunk divides by floor; stride means q = kv (mod a); head-below reads
+  the query head; NOT complements over in-range keys.
+* A paged cache holds logical key j of sequence b in slot j % page_size of
+  page page_table[b][j // page_size]; every rule sees logical positions.
+* The backward is the chain rule of the forward definition; D is formed from
+  the output the backward receives (the stored output when one is given).
 
 Rows are computed in groups of whole rows purely to bound memory; every row
 is evaluated in full, exactly as the definition states.
