@@ -109,19 +109,6 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, 
   for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (kBT * 128), map, bar, c * 64, row, h, b);
 }
 
-// Score rule in log2 units and its slope dg/ds for one cell; th is
-// tanh(s c_in) under a soft-cap (unused otherwise).
-template <int SCORE>
-__device__ __forceinline__ void score_and_slope(float s, float th, float c_out, float bias, float& t, float& gp) {
-  if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) {
-    t = fmaf(c_out, th, bias);
-    gp = fmaf(-th, th, 1.0f);
-  } else {
-    t = fmaf(s, c_out, bias);
-    gp = 1.0f;
-  }
-}
-
 // ---------------------------------------------------------------------------
 // dQ: one query tile, walking its key-side list
 // ---------------------------------------------------------------------------
@@ -134,7 +121,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdBars bars;
-  __shared__ float s_pos[2][kBT];
+  __shared__ __align__(16) float s_pos[2][kBT];
   __shared__ int s_doc[2][kBT];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -245,9 +232,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
     const float slope2 = distance_slope(h, Hs) * kLog2eB;
-    const bool capped = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS;
-    const float c_in = capped ? a.scale / a.score.cap : 0.0f;
-    const float c_out = capped ? a.score.cap * kLog2eB : a.scale * kLog2eB;
+    constexpr bool kCapped = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS;
+    const float c_in = kCapped ? a.scale / a.score.cap : 0.0f;
+    const float c_out = kCapped ? a.score.cap * kLog2eB : a.scale * kLog2eB;
     const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
     const float pq_scaled = has_pos ? slope2 * static_cast<float>(pos_at(a.score, b, qpos, a.S)) : 0.0f;
     const bool is_prog = a.mask.kind == FA_MASK_PROGRAM;
@@ -312,24 +299,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float bias0 = (SCORE == FA_SCORE_ALIBI || (SCORE == FA_SCORE_CAP_THEN_BIAS && !has_pos))
                                 ? slope2 * static_cast<float>(base - qpos) : 0.0f;
         float th[32];
-        if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) tanh32(sr, c_in, th);
+        if constexpr (kCapped) tanh32(sr, c_in, th);
+        // two columns per step in f32x2 arithmetic
+        const float* spos = s_pos[cnt & 1] + 32 * j;
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float ds2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = i + e;
-            float bias = 0.0f;
-            if constexpr (SCORE == FA_SCORE_ALIBI) bias = fmaf(slope2, static_cast<float>(c), bias0);
-            if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
-              bias = has_pos ? s_pos[cnt & 1][32 * j + c] - pq_scaled : fmaf(slope2, static_cast<float>(c), bias0);
-            float t, gp;
-            score_and_slope<SCORE>(__uint_as_float(sr[c]), th[c], c_out, bias, t, gp);
-            const float p = ((bits >> c) & 1u) ? ex2_approx(t - lse2) : 0.0f;
-            ds2[e] = p * (__uint_as_float(dp[c]) - dsum) * gp;
+          const float2 col = make_float2(static_cast<float>(i), static_cast<float>(i + 1));
+          float2 bias = splat2(0.0f);
+          if constexpr (SCORE == FA_SCORE_ALIBI) bias = fma2(splat2(slope2), col, splat2(bias0));
+          if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
+            bias = has_pos ? add2(*reinterpret_cast<const float2*>(spos + i), splat2(-pq_scaled))
+                           : fma2(splat2(slope2), col, splat2(bias0));
+          float2 t, gp = splat2(1.0f);
+          if constexpr (kCapped) {
+            const float2 th2 = make_float2(th[i], th[i + 1]);
+            t = fma2(th2, splat2(c_out), bias);
+            gp = fma2(make_float2(-th2.x, -th2.y), th2, splat2(1.0f));
+          } else {
+            t = fma2(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), splat2(c_out), bias);
           }
-          pk[i >> 1] = pack_bf16x2(ds2[0], ds2[1]);
+          const float2 e = add2(t, splat2(-lse2));
+          const float2 p = make_float2(((bits >> i) & 1u) ? ex2_approx(e.x) : 0.0f,
+                                       ((bits >> (i + 1)) & 1u) ? ex2_approx(e.y) : 0.0f);
+          float2 ds = mul2(p, add2(make_float2(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])), splat2(-dsum)));
+          if constexpr (kCapped) ds = mul2(ds, gp);
+          pk[i >> 1] = pack_bf16x2(ds.x, ds.y);
         }
         // dS of these 32 keys as bf16 pairs over S columns already read
         tmem_st16(tbase + lane_base + 32 * j, pk);
@@ -427,7 +422,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   __shared__ BwdBars bars;
-  __shared__ float s_lse[2][kBT], s_dsum[2][kBT], s_pq[2][kBT];
+  __shared__ __align__(16) float s_lse[2][kBT];
+  __shared__ __align__(16) float s_dsum[2][kBT];
+  __shared__ __align__(16) float s_pq[2][kBT];
   __shared__ int s_doc[2][kBT];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
@@ -543,9 +540,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = kv < S_b;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
-    const bool capped = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS;
-    const float c_in = capped ? a.scale / a.score.cap : 0.0f;
-    const float c_out = capped ? a.score.cap * kLog2eB : a.scale * kLog2eB;
+    constexpr bool kCapped = SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS;
+    const float c_in = kCapped ? a.scale / a.score.cap : 0.0f;
+    const float c_out = kCapped ? a.score.cap * kLog2eB : a.scale * kLog2eB;
     const bool has_pos = SCORE == FA_SCORE_CAP_THEN_BIAS && a.score.pos != nullptr;
     const float pk_raw = has_pos ? static_cast<float>(pos_at(a.score, b, kv, a.S)) : 0.0f;
     const bool is_prog = a.mask.kind == FA_MASK_PROGRAM;
@@ -611,28 +608,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float* lq = s_lse[cnt & 1] + 32 * j;
         const float* dq = s_dsum[cnt & 1] + 32 * j;
+        const float* pqv = s_pq[cnt & 1] + 32 * j;
         const float bias0 = slope2 * static_cast<float>(kv - qbase);  // slope2 (kv - q) at c = 0
         float th[32];
-        if constexpr (SCORE == FA_SCORE_SOFTCAP || SCORE == FA_SCORE_CAP_THEN_BIAS) tanh32(sr, c_in, th);
+        if constexpr (kCapped) tanh32(sr, c_in, th);
+        // four columns per step: their query-side values in one 16-byte load
+        // each, the arithmetic in f32x2 pairs
         uint32_t ppk[16], dpk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p2[2], d2[2];
+        for (int i = 0; i < 32; i += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lq + i);
+          const float4 d4 = *reinterpret_cast<const float4*>(dq + i);
+          float4 q4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
+            if (has_pos) q4 = *reinterpret_cast<const float4*>(pqv + i);
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = i + e;
-            float bias = 0.0f;
-            if constexpr (SCORE == FA_SCORE_ALIBI) bias = fmaf(-slope2, static_cast<float>(c), bias0);
-            if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS)
-              bias = has_pos ? slope2 * (pk_raw - s_pq[cnt & 1][32 * j + c]) : fmaf(-slope2, static_cast<float>(c), bias0);
-            float t, gp;
-            score_and_slope<SCORE>(__uint_as_float(sr[c]), th[c], c_out, bias, t, gp);
-            const float p = ((bits >> c) & 1u) ? ex2_approx(t - lq[c]) : 0.0f;
-            p2[e] = p;
-            d2[e] = p * (__uint_as_float(dp[c]) - dq[c]) * gp;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int c = i + 2 * hh;
+            const float2 lq2 = hh ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+            const float2 dq2 = hh ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+            const float2 col = make_float2(static_cast<float>(c), static_cast<float>(c + 1));
+            float2 bias = splat2(0.0f);
+            if constexpr (SCORE == FA_SCORE_ALIBI) bias = fma2(splat2(-slope2), col, splat2(bias0));
+            if constexpr (SCORE == FA_SCORE_CAP_THEN_BIAS) {
+              const float2 pq2 = hh ? make_float2(q4.z, q4.w) : make_float2(q4.x, q4.y);
+              bias = has_pos ? mul2(splat2(slope2), add2(splat2(pk_raw), make_float2(-pq2.x, -pq2.y)))
+                             : fma2(splat2(-slope2), col, splat2(bias0));
+            }
+            float2 t, gp = splat2(1.0f);
+            if constexpr (kCapped) {
+              const float2 th2 = make_float2(th[c], th[c + 1]);
+              t = fma2(th2, splat2(c_out), bias);
+              gp = fma2(make_float2(-th2.x, -th2.y), th2, splat2(1.0f));
+            } else {
+              t = fma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), splat2(c_out), bias);
+            }
+            const float2 e = add2(t, make_float2(-lq2.x, -lq2.y));
+            const float2 p = make_float2(((bits >> c) & 1u) ? ex2_approx(e.x) : 0.0f,
+                                         ((bits >> (c + 1)) & 1u) ? ex2_approx(e.y) : 0.0f);
+            float2 d = mul2(p, add2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                    make_float2(-dq2.x, -dq2.y)));
+            if constexpr (kCapped) d = mul2(d, gp);
+            ppk[c >> 1] = pack_bf16x2(p.x, p.y);
+            dpk[c >> 1] = pack_bf16x2(d.x, d.y);
           }
-          ppk[i >> 1] = pack_bf16x2(p2[0], p2[1]);
-          dpk[i >> 1] = pack_bf16x2(d2[0], d2[1]);
         }
         // P^T and dS^T of these 32 queries as bf16 pairs over columns already read
         tmem_st16(tbase + lane_base + 32 * j, ppk);
@@ -710,41 +729,47 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const BwdArgs a) {
 
 // Query-side lists: one thread per key tile n of row set (b, h).
 __global__ void __launch_bounds__(128) transpose_kernel(const TransposeArgs a) {
+  // one warp per key tile n: lane l tests rows m = l, l + 32, ... (a binary
+  // search of each ascending list), and ballots keep the rows in order
   const int b = blockIdx.y, h = blockIdx.z;
+  const int lane = threadIdx.x & 31;
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (n >= a.Nb) return;
   const int64_t kv_row0 = (static_cast<int64_t>(b) * a.H + h) * a.Mb;
-  const int64_t q_row0 = (static_cast<int64_t>(b) * a.H + h) * a.Nb;
-  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < a.Nb; n += gridDim.x * blockDim.x) {
-    int np = 0, nf = 0;
-    const int64_t qr = q_row0 + n;
-    for (int m = 0; m < a.Mb; ++m) {
-      const int64_t kr = kv_row0 + m;
-#pragma unroll
-      for (int full = 0; full < 2; ++full) {
-        const int cnt = full ? a.full_kv_num_blocks[kr] : a.kv_num_blocks[kr];
-        const int* lst = (full ? a.full_kv_indices : a.kv_indices) + kr * a.Nb;
-        int lo = 0, hi = cnt - 1;  // the lists are ascending: binary search for n
-        bool found = false;
-        while (lo <= hi) {
-          const int mid = (lo + hi) >> 1;
-          const int x = lst[mid];
-          if (x == n) {
-            found = true;
-            break;
-          }
-          if (x < n) lo = mid + 1;
-          else hi = mid - 1;
-        }
-        if (found) {
-          if (full) a.full_q_indices[qr * a.Mb + nf++] = m;
-          else a.q_indices[qr * a.Mb + np++] = m;
-        }
-      }
+  const int64_t qr = (static_cast<int64_t>(b) * a.H + h) * a.Nb + n;
+  auto listed = [&](const int* idx, int cnt) {
+    int lo = 0, hi = cnt - 1;
+    while (lo <= hi) {
+      const int mid = (lo + hi) >> 1;
+      const int x = idx[mid];
+      if (x == n) return true;
+      if (x < n) lo = mid + 1;
+      else hi = mid - 1;
     }
+    return false;
+  };
+  int np = 0, nf = 0;
+  const unsigned below = (1u << lane) - 1u;
+  for (int m0 = 0; m0 < a.Mb; m0 += 32) {
+    const int m = m0 + lane;
+    bool in_p = false, in_f = false;
+    if (m < a.Mb) {
+      const int64_t kr = kv_row0 + m;
+      in_f = listed(a.full_kv_indices + kr * a.Nb, a.full_kv_num_blocks[kr]);
+      in_p = !in_f && listed(a.kv_indices + kr * a.Nb, a.kv_num_blocks[kr]);
+    }
+    const unsigned bp = __ballot_sync(0xffffffffu, in_p), bf = __ballot_sync(0xffffffffu, in_f);
+    if (in_p) a.q_indices[qr * a.Mb + np + __popc(bp & below)] = m;
+    if (in_f) a.full_q_indices[qr * a.Mb + nf + __popc(bf & below)] = m;
+    np += __popc(bp);
+    nf += __popc(bf);
+  }
+  if (lane == 0) {
     a.q_num_blocks[qr] = np;
     a.full_q_num_blocks[qr] = nf;
-    for (int m = np; m < a.Mb; ++m) a.q_indices[qr * a.Mb + m] = 0;
-    for (int m = nf; m < a.Mb; ++m) a.full_q_indices[qr * a.Mb + m] = 0;
   }
+  for (int m = np + lane; m < a.Mb; m += 32) a.q_indices[qr * a.Mb + m] = 0;
+  for (int m = nf + lane; m < a.Mb; m += 32) a.full_q_indices[qr * a.Mb + m] = 0;
 }
 
 template <int D, int SCORE>
@@ -782,7 +807,7 @@ cudaError_t launch_bwd(const BwdArgs& a, const BwdMaps& maps, cudaStream_t strea
 }
 
 cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t stream) {
-  dim3 grid((a.Nb + 127) / 128, a.B, a.H);
+  dim3 grid((a.Nb + 3) / 4, a.B, a.H);  // four warps (key tiles) per CTA
   transpose_kernel<<<grid, 128, 0, stream>>>(a);
   return cudaGetLastError();
 }
