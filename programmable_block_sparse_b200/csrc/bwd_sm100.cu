@@ -62,7 +62,7 @@ struct BCfg {
 struct BwdBars {
   uint64_t fixed_full;                 // the two tiles loaded once
   uint64_t full[4], empty[4];          // the ring (both tiles of a stage)
-  uint64_t s_full, p_full, o_final;
+  uint64_t s_full[2], p_full[2], o_final;  // per half of the tile's columns
   int info[2];                         // tile index | class bit
   int info_h[2];                       // query head (dK / dV kernel)
   uint32_t tmem_base;
@@ -145,8 +145,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1);
     }
-    mbar_init(&bars.s_full, 2);
-    mbar_init(&bars.p_full, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.s_full[i], 2);  // the MMA thread's arrive (tile info) + the commit
+      mbar_init(&bars.p_full[i], 8);  // every math warp
+    }
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);  // one half of the keys
       constexpr uint32_t idesc_dq = umma_idesc_bf16(128, D, 0, 1);
       const uint64_t dq0 = umma_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t ddo0 = umma_desc_sw128(smem_u32(sDO), 16, 1024);
@@ -201,20 +203,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const int n = list_n(u);
         bars.info[u & 1] = n | (u < nfull ? kInfoFullB : 0);
+        // S and dP in two halves of 64 keys each (columns 64 hf ..), so the
+        // rows' math on the first half overlaps the products of the second,
+        // and dQ over the first half overlaps the math on the second
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * (kBT * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(tbase, dq0 + off, dk0 + s * kStep + off, idesc_s, kk > 0 ? 1u : 0u);
-          umma_ss(tbase + 128, ddo0 + off, dv0 + s * kStep + off, idesc_s, kk > 0 ? 1u : 0u);
+        for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * (kBT * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t koff = s * kStep + off + ((hf * 64 * 128) >> 4);  // key rows 64 hf ..
+            umma_ss(tbase + 64 * hf, dq0 + off, dk0 + koff, idesc_s, kk > 0 ? 1u : 0u);
+            umma_ss(tbase + 128 + 64 * hf, ddo0 + off, dv0 + koff, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mbar_arrive(&bars.s_full[hf]);
+          umma_commit(&bars.s_full[hf]);
         }
-        mbar_arrive(&bars.s_full);
-        umma_commit(&bars.s_full);
-        if (!mbar_wait(&bars.p_full, u & 1, abort, a.status, a.wait_cycles)) break;
-        tc_fence_after();
+        bool half_ok = true;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tbase + 256, tbase + pair_col(kk), dkmn0 + s * kStep + ((kk * 16 * 128) >> 4), idesc_dq,
-                  (u > 0 || kk > 0) ? 1u : 0u);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!(half_ok = mbar_wait(&bars.p_full[hf], u & 1, abort, a.status, a.wait_cycles))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+            umma_ts(tbase + 256, tbase + pair_col(kk), dkmn0 + s * kStep + ((kk * 16 * 128) >> 4), idesc_dq,
+                    (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!half_ok) break;
         umma_commit(&bars.empty[s]);
       }
       umma_commit(&bars.o_final);
@@ -224,7 +238,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ rows
     const int quad = warp & 3;
-    const int jg = (warp - 2) >> 2;  // math group: column chunks 2 jg, 2 jg + 1
+    const int jg = (warp - 2) >> 2;  // math group: chunk jg of each 64-column half
     const int r = quad * 32 + lane;
     const int grow = mt * kBT + r;
     const bool row_ok = grow < a.L;
@@ -250,7 +264,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool alive = true;
     int cnt = 0;
     for (; cnt < total; ++cnt) {
-      bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full, cnt & 1, abort, a.status, a.wait_cycles));
+      bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[0], cnt & 1, abort, a.status, a.wait_cycles));
       const int info = ok ? bars.info[cnt & 1] : 0;
       const int n = info & (kInfoFullB - 1);
       const bool full = (info & kInfoFullB) != 0;
@@ -272,7 +286,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const bool need_mask = !full || edge || !row_ok;
 #pragma unroll 1
-      for (int j = 2 * jg; j < 2 * jg + 2; ++j) {
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf == 1) {
+          // the second half's products land on their own barrier
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[1], cnt & 1, abort, a.status, a.wait_cycles))) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int j = 2 * hf + jg;  // this warp's 32-column chunk of the half
         uint32_t sr[32], dp[32];
         tmem_ld16(tbase + lane_base + 32 * j, *reinterpret_cast<uint32_t(*)[16]>(sr));
         tmem_ld16(tbase + lane_base + 32 * j + 16, *reinterpret_cast<uint32_t(*)[16]>(sr + 16));
@@ -328,11 +351,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // dS of these 32 keys as bf16 pairs over S columns already read
         tmem_st16(tbase + lane_base + 32 * j, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[hf]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
     }
     // epilogue: dq = scale dQ (zero for a row of tiles with no listed key tile)
     if (alive && cnt > 0) {
@@ -449,8 +472,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1);
     }
-    mbar_init(&bars.s_full, 2);
-    mbar_init(&bars.p_full, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.s_full[i], 2);  // the MMA thread's arrive (tile info) + the commit
+      mbar_init(&bars.p_full[i], 8);  // every math warp
+    }
     mbar_init(&bars.o_final, 1);
     bars.abort = 0;
     mbar_fence_init();
@@ -488,7 +513,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = umma_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_s = umma_idesc_bf16(128, 64, 0, 0);  // one half of the queries
       constexpr uint32_t idesc_acc = umma_idesc_bf16(128, D, 0, 1);
       const uint64_t dk0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv0 = umma_desc_sw128(smem_u32(sV), 16, 1024);
@@ -508,23 +533,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         bars.info[u & 1] = m | (f ? kInfoFullB : 0);
         bars.info_h[u & 1] = g;
+        // S^T and dP^T in two halves of 64 queries each (columns 64 hf ..), so
+        // the rows' math on the first half overlaps the products of the
+        // second, and dV / dK over the first half the math on the second
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * (kBT * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(tbase, dk0 + off, dq0 + s * kStep + off, idesc_s, kk > 0 ? 1u : 0u);         // S^T = K Q^T
-          umma_ss(tbase + 128, dv0 + off, ddo0 + s * kStep + off, idesc_s, kk > 0 ? 1u : 0u);  // dP^T = V dout^T
-        }
-        mbar_arrive(&bars.s_full);
-        umma_commit(&bars.s_full);
-        if (!mbar_wait(&bars.p_full, u & 1, abort, a.status, a.wait_cycles)) break;
-        tc_fence_after();
+        for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t boff = s * kStep + ((kk * 16 * 128) >> 4);
-          umma_ts(tbase + 256, tbase + pair_col(kk), ddomn0 + boff, idesc_acc, acc);          // dV += P^T dout
-          umma_ts(tbase + 256 + D, tbase + 128 + pair_col(kk), dqmn0 + boff, idesc_acc, acc); // dK += dS^T Q
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * (kBT * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t qoff = s * kStep + off + ((hf * 64 * 128) >> 4);  // query rows 64 hf ..
+            umma_ss(tbase + 64 * hf, dk0 + off, dq0 + qoff, idesc_s, kk > 0 ? 1u : 0u);         // S^T = K Q^T
+            umma_ss(tbase + 128 + 64 * hf, dv0 + off, ddo0 + qoff, idesc_s, kk > 0 ? 1u : 0u);  // dP^T = V dout^T
+          }
+          mbar_arrive(&bars.s_full[hf]);
+          umma_commit(&bars.s_full[hf]);
         }
+        bool half_ok = true;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!(half_ok = mbar_wait(&bars.p_full[hf], u & 1, abort, a.status, a.wait_cycles))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk) {
+            const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t boff = s * kStep + ((kk * 16 * 128) >> 4);
+            umma_ts(tbase + 256, tbase + pair_col(kk), ddomn0 + boff, idesc_acc, acc);          // dV += P^T dout
+            umma_ts(tbase + 256 + D, tbase + 128 + pair_col(kk), dqmn0 + boff, idesc_acc, acc); // dK += dS^T Q
+          }
+        }
+        if (!half_ok) break;
         umma_commit(&bars.empty[s]);
       }
       umma_commit(&bars.o_final);
@@ -534,7 +571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ key rows
     const int quad = warp & 3;
-    const int jg = (warp - 2) >> 2;  // math group: column chunks 2 jg, 2 jg + 1
+    const int jg = (warp - 2) >> 2;  // math group: chunk jg of each 64-column half
     const int r = quad * 32 + lane;
     const int kv = n * kBT + r;
     const bool key_ok = kv < S_b;
@@ -553,7 +590,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool alive = true;
     int cnt = 0;
     for (; cnt < total; ++cnt) {
-      bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full, cnt & 1, abort, a.status, a.wait_cycles));
+      bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[0], cnt & 1, abort, a.status, a.wait_cycles));
       const int info = ok ? bars.info[cnt & 1] : 0;
       const int mq = info & (kInfoFullB - 1);
       const bool full = (info & kInfoFullB) != 0;
@@ -584,7 +621,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool edge = i0 + kBT > a.L || n * kBT + kBT > S_b;
       const bool need_mask = !full || edge || !key_ok;
 #pragma unroll 1
-      for (int j = 2 * jg; j < 2 * jg + 2; ++j) {
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf == 1) {
+          // the second half's products land on their own barrier
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[1], cnt & 1, abort, a.status, a.wait_cycles))) {
+            alive = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int j = 2 * hf + jg;  // this warp's 32-column chunk of the half
         uint32_t sr[32], dp[32];
         tmem_ld16(tbase + lane_base + 32 * j, *reinterpret_cast<uint32_t(*)[16]>(sr));
         tmem_ld16(tbase + lane_base + 32 * j + 16, *reinterpret_cast<uint32_t(*)[16]>(sr + 16));
@@ -656,11 +702,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // P^T and dS^T of these 32 queries as bf16 pairs over columns already read
         tmem_st16(tbase + lane_base + 32 * j, ppk);
         tmem_st16(tbase + lane_base + 128 + 32 * j, dpk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[hf]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full);
     }
     // epilogue: dv = dV, dk = scale dK (zero for a key tile no query lists)
     if (alive && cnt > 0) {
