@@ -569,26 +569,47 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   };
   auto row_head = [&](int r) { return hk * a.G + hc * p.heads_per_cta + r / a.L; };
 
-  // K (u even) or V (u odd) of tile u / 2 into ring entry u % R
-  auto issue_load = [&](int u) {
-    const int e = u % R, j = u >> 1;
+  // Rows and outer coordinates (batch, or page of a paged pool) of the two
+  // 64-key boxes of tile j; the producer reads them one tile ahead, so the
+  // list and page-table loads are not on its issue path.
+  auto tile_addr = [&](int j, int (&row)[2], int (&outer)[2]) {
     const int n = list_tile(a, brow, nfull, t0 + j / subs);
     const int kv0 = n * a.bm.BN + (j % subs) * kTcKeys;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      // a paged cache keeps each 64-key box in one page
+      row[h2] = kv0 + 64 * h2;
+      outer[h2] = b;
+      if (a.page_table) {
+        outer[h2] = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, row[h2]);
+        row[h2] = row[h2] % a.page_size;
+      }
+    }
+  };
+  int row_c[2], outer_c[2], row_n[2], outer_n[2];  // tile of copy u, and the next tile
+  // K (u even) or V (u odd) of tile u / 2 into ring entry u % R
+  auto issue_load = [&](int u) {
+    if (u == 0) {
+      tile_addr(0, row_c, outer_c);
+      if (nsub > 1) tile_addr(1, row_n, outer_n);
+    } else if ((u & 1) == 0) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        row_c[h2] = row_n[h2];
+        outer_c[h2] = outer_n[h2];
+      }
+      if ((u >> 1) + 1 < nsub) tile_addr((u >> 1) + 1, row_n, outer_n);
+    }
+    const int e = u % R;
     const CUtensorMap* map = (u & 1) ? &map_v : &map_k;
     uint8_t* dst = sKV + e * C::kEntryBytes;
     mbar_expect_tx(&bars.full[e], C::kEntryBytes);
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      // two 64-key boxes per tile; a paged cache keeps each in one page
-      int row = kv0 + 64 * h2, outer = b;
-      if (a.page_table) {
-        outer = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, row);
-        row = row % a.page_size;
-      }
+    for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(dst + c * (kTcKeys * 128) + h2 * (64 * 128), map, &bars.full[e], c * 64, row, hk, outer);
-    }
+        tma_load_4d(dst + c * (kTcKeys * 128) + h2 * (64 * 128), map, &bars.full[e], c * 64, row_c[h2], hk,
+                    outer_c[h2]);
   };
   // The first R copies need no free entry: thread 0 (the producer) issues
   // them right after initialising the barriers, so they are in flight while
