@@ -25,6 +25,7 @@ namespace {
 
 constexpr int kSimtThreads = 128;
 constexpr int kChunk = 32;
+constexpr int kSimtRows = 8;  // query rows per CTA: a query tile spreads over BM / 8 CTAs
 
 template <typename T>
 __device__ __forceinline__ float to_f(T x);
@@ -41,42 +42,47 @@ template <>
 __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(kSimtThreads, 1) fwd_simt_kernel(FwdArgs a) {
   extern __shared__ float smem[];
-  const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int t = threadIdx.x;
   const int BM = a.bm.BM, BN = a.bm.BN;
   const int E = a.E, Ev = a.Ev;
-  // R threads per query row (R = 128 / BM, at least 1): thread t takes row
-  // t % BM and the keys j = sub (mod R) of every chunk, sub = t / BM; the R
-  // partial (max, sum, O) of a row are merged at the end.
-  const int R = BM >= kSimtThreads ? 1 : kSimtThreads / BM;
+  // A CTA takes RB = min(BM, 8) rows of query tile mt; R = 128 / RB threads
+  // per row: thread t takes row t % RB and the keys j = sub (mod R) of every
+  // chunk, sub = t / RB; the R partial (max, sum, O) of a row are merged at
+  // the end.
+  const int RB = BM < kSimtRows ? BM : kSimtRows;
+  const int nsplit = (BM + RB - 1) / RB;
+  const int mt = blockIdx.x / nsplit, part = blockIdx.x % nsplit;
+  const int R = kSimtThreads / RB;
   const int qst = E | 1, ost = Ev | 1;  // odd row strides: no bank conflicts across rows
   float* sq = smem;
-  float* so = sq + BM * qst;             // [R][BM] partial O rows
-  float* sk = so + R * BM * ost;
+  float* so = sq + RB * qst;             // [R][RB] partial O rows
+  float* sk = so + R * RB * ost;
   float* sv = sk + kChunk * E;
-  float* sml = sv + kChunk * Ev;          // [R][BM] partial max, then [R][BM] partial sum
-  float* ss = sml + 2 * R * BM;           // [128][kChunk + 1] each thread's chunk scores
+  float* sml = sv + kChunk * Ev;          // [R][RB] partial max, then [R][RB] partial sum
+  float* ss = sml + 2 * R * RB;           // [128][kChunk + 1] each thread's chunk scores
 
   const int hk = h / a.G;
   const int S = a.S, L = a.L;
   const int S_b = seq_len_b(a.mask, b, S);
-  const int r0 = mt * BM;
+  const int r0 = mt * BM + part * RB;                     // first row of this CTA
+  const int r_end = min(mt * BM + BM, L);                 // end of the tile's rows
   const T* qb = static_cast<const T*>(a.q) + b * a.q_stride[0] + h * a.q_stride[1];
   const T* kb = static_cast<const T*>(a.k) + b * a.k_stride[0] + hk * a.k_stride[1];
   const T* vb = static_cast<const T*>(a.v) + b * a.v_stride[0] + hk * a.v_stride[1];
 
-  for (int i = t; i < BM * E; i += blockDim.x) {
+  for (int i = t; i < RB * E; i += blockDim.x) {
     const int r = i / E, e = i % E;
-    sq[r * qst + e] = (r0 + r < L) ? to_f(qb[(r0 + r) * a.q_stride[2] + e]) : 0.0f;
+    sq[r * qst + e] = (r0 + r < r_end) ? to_f(qb[(r0 + r) * a.q_stride[2] + e]) : 0.0f;
   }
-  for (int i = t; i < R * BM * Ev; i += blockDim.x) so[(i / Ev) * ost + i % Ev] = 0.0f;
+  for (int i = t; i < R * RB * Ev; i += blockDim.x) so[(i / Ev) * ost + i % Ev] = 0.0f;
 
-  const int rr = t % BM, sub = t / BM;
+  const int rr = t % RB, sub = t / RB;
   const int row = r0 + rr;
-  const bool active = sub < R && row < L;
-  float* orow = so + (sub * BM + rr) * ost;
+  const bool active = sub < R && row < r_end;
+  float* orow = so + (sub * RB + rr) * ost;
   const float* qrow = sq + rr * qst;
   const int qpos = query_pos(row, L, S_b);
   const int Hs = a.score.slope_heads > 0 ? a.score.slope_heads : a.Hq;
@@ -173,15 +179,15 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
   // merge the R partials of each row: thread sub 0 of the row writes it
   __syncthreads();
   if (sub < R) {
-    sml[sub * BM + rr] = m_run;
-    sml[(R + sub) * BM + rr] = l_run;
+    sml[sub * RB + rr] = m_run;
+    sml[(R + sub) * RB + rr] = l_run;
   }
   __syncthreads();
   if (!active || sub != 0) return;
   float m = sml[rr];
-  for (int r = 1; r < R; ++r) m = fmaxf(m, sml[r * BM + rr]);
+  for (int r = 1; r < R; ++r) m = fmaxf(m, sml[r * RB + rr]);
   float l = 0.0f;
-  for (int r = 0; r < R; ++r) l += sml[(R + r) * BM + rr] * expf(sml[r * BM + rr] - m);
+  for (int r = 0; r < R; ++r) l += sml[(R + r) * RB + rr] * expf(sml[r * RB + rr] - m);
   const int64_t ooff = b * a.o_stride[0] + h * a.o_stride[1] + row * a.o_stride[2];
   // a row without a visible key has l = 0: out 0 and lse -inf, unless the
   // caller promised there is none (rows_safe), which drops this guard
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
   const float inv = live ? 1.0f / l : 0.0f;
   for (int d = 0; d < Ev; ++d) {
     float o = 0.0f;
-    for (int r = 0; r < R; ++r) o += so[(r * BM + rr) * ost + d] * expf(sml[r * BM + rr] - m);
+    for (int r = 0; r < R; ++r) o += so[(r * RB + rr) * ost + d] * expf(sml[r * RB + rr] - m);
     const float val = live ? o * inv : 0.0f;
     if (a.out_f32)
       static_cast<float*>(a.out)[ooff + d] = val;
@@ -205,11 +211,12 @@ __global__ void __launch_bounds__(kSimtThreads) fwd_simt_kernel(FwdArgs a) {
 
 cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream) {
   const int BM = a.bm.BM;
-  const int R = BM >= kSimtThreads ? 1 : kSimtThreads / BM;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(BM) * ((a.E | 1) + R * (a.Ev | 1)) +
-                                       static_cast<size_t>(kChunk) * (a.E + a.Ev) + 2 * R * BM +
+  const int RB = BM < kSimtRows ? BM : kSimtRows;
+  const int R = kSimtThreads / RB;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(RB) * ((a.E | 1) + R * (a.Ev | 1)) +
+                                       static_cast<size_t>(kChunk) * (a.E + a.Ev) + 2 * R * RB +
                                        static_cast<size_t>(kSimtThreads) * (kChunk + 1));
-  dim3 grid(a.bm.Mb, a.Hq, a.B);
+  dim3 grid(a.bm.Mb * ((BM + RB - 1) / RB), a.Hq, a.B);
   cudaError_t e;
   if (a.dtype == FA_DTYPE_F32) {
     e = cudaFuncSetAttribute(fwd_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
