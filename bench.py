@@ -86,20 +86,20 @@ HEADLINE = BENCH_ITEMS[0][0]
 # workload is stated in the profile it comes from.
 NCU_TRAFFIC = {
     # fwd_sm100_kernel<128, 0>, captured at batch 1 (profiles/fwd_sm100_gqa_sliding_window.md): x 2 sequences
-    "gqa_sliding_window": {"bytes": 2 * (201787392 + 96543232), "source_hash": "e9e8eb8d91dff766"},
+    "gqa_sliding_window": {"bytes": 2 * (201745152 + 94600448), "source_hash": "f65fafb4a06d314c"},
     # fwd_sm100_kernel<64, 3> / <128, 3>, full size (profiles/fwd_sm100_causal_packed_sliver.md)
-    "causal_softcap_alibi": {"bytes": 50412800 + 1033472, "source_hash": "e9e8eb8d91dff766"},
-    "packed_docs": {"bytes": 100861696 + 12390656, "source_hash": "e9e8eb8d91dff766"},
-    "sliver_every_fourth_key": {"bytes": 50420480 + 708864, "source_hash": "e9e8eb8d91dff766"},
+    "causal_softcap_alibi": {"bytes": 50419968 + 782848, "source_hash": "f65fafb4a06d314c"},
+    "packed_docs": {"bytes": 100836352 + 9787648, "source_hash": "f65fafb4a06d314c"},
+    "sliver_every_fourth_key": {"bytes": 50427392 + 771584, "source_hash": "f65fafb4a06d314c"},
     # decode_tc_kernel<128, 1>, captured at batch 16 (profiles/decode_tc_kernel_decode_kv_cache.md):
     # x 614602 / 296926 cached tokens
-    "decode_kv_cache": {"bytes": round((1221946880 + 8642816) * 614602 / 296926), "source_hash": "e054904aaeb2d24a"},
-    "decode_kv_cache_q1": {"bytes": round((1220857344 + 4764928) * 614602 / 296926),
-                           "source_hash": "e054904aaeb2d24a"},
+    "decode_kv_cache": {"bytes": round((1222132224 + 8572672) * 614602 / 296926), "source_hash": "66031533768da397"},
+    "decode_kv_cache_q1": {"bytes": round((1220863488 + 4685568) * 614602 / 296926),
+                           "source_hash": "66031533768da397"},
     # bwd_dkdv_kernel (the larger of the two backward kernels), full size
     # (profiles/bwd_dkdv_dq_backward.md)
-    "backward_causal_softcap_alibi": {"bytes": 69195776 + 7536896, "source_hash": "11fa386a7150b63d"},
-    "backward_packed_docs": {"bytes": 136113152 + 37091328, "source_hash": "11fa386a7150b63d"},
+    "backward_causal_softcap_alibi": {"bytes": 69229056 + 7497984, "source_hash": "fd297535d8b984d1"},
+    "backward_packed_docs": {"bytes": 136204544 + 36972288, "source_hash": "fd297535d8b984d1"},
 }
 
 KERNEL_SOURCES = {

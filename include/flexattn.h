@@ -395,6 +395,7 @@ int flexattn_backward_workspace_size(const fa_tensor* q, size_t* bytes);
  *   block_mask / block_mask_q: 128 x 128 tiles, with the query-side lists
  *       from flexattn_transpose_block_mask.
  *   workspace: flexattn_backward_workspace_size() bytes.
+ * Every tensor's base and strides are 16-byte aligned (else FA_ERR_ALIGN).
  * No paged cache.  Errors: those of flexattn_forward, and FA_ERR_UNSUPPORTED
  * for other dtypes, head dims or tile sizes. */
 int flexattn_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v, const fa_tensor* out,

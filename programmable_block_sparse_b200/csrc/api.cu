@@ -738,8 +738,8 @@ int flexattn_backward(const fa_tensor* q, const fa_tensor* k, const fa_tensor* v
   }
   for (const fa_tensor* g : {dq, dk, dv})
     if (g->dtype != FA_DTYPE_BF16 && g->dtype != FA_DTYPE_F32) return fail(FA_ERR_DTYPE, "gradients are bf16 or fp32");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
     return fail(FA_ERR_ALIGN, "the backward pass needs 16-byte aligned tensors and strides");
   if (qs->B != block_mask->B || qs->H != block_mask->H || qs->Mb != block_mask->Mb || qs->Nb != block_mask->Nb)
     return fail(FA_ERR_MASK_SHAPE, "query-side lists must have the block mask's B, H, Mb, Nb");

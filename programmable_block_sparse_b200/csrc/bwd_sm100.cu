@@ -755,22 +755,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 1) tmem_dealloc(tbase, 512);
 }
 
-// D = rowsum(dout * out) in fp32: one warp per row.
+// D = rowsum(dout * out) in fp32.  Each thread reads 8 elements of a row
+// with one 16-byte load from each tensor, E / 8 neighbouring lanes share a
+// row (8 or 16), and a shuffle tree over those lanes sums it: 256 / (E / 8)
+// rows of one (batch, head) per CTA, grid (row blocks, Hq, B).
 __global__ void __launch_bounds__(256) bwd_dsum_kernel(const BwdArgs a) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
-  if (row >= rows) return;
-  const int i = static_cast<int>(row % a.L);
-  const int h = static_cast<int>((row / a.L) % a.Hq);
-  const int b = static_cast<int>(row / (static_cast<int64_t>(a.L) * a.Hq));
-  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] + i * a.o_stride[2];
-  const __nv_bfloat16* d = static_cast<const __nv_bfloat16*>(a.dout) + b * a.do_stride[0] + h * a.do_stride[1] + i * a.do_stride[2];
+  const int lg = a.E == 64 ? 3 : 4;  // log2 of the threads per row
+  const int tpr = 1 << lg;
+  const int i = blockIdx.x * (256 >> lg) + (threadIdx.x >> lg);
+  const int part = threadIdx.x & (tpr - 1);
+  const int h = blockIdx.y, b = blockIdx.z;
   float acc = 0.0f;
-  for (int e = lane; e < a.E; e += 32) acc = fmaf(__bfloat162float(o[e]), __bfloat162float(d[e]), acc);
+  if (i < a.L) {
+    const __nv_bfloat16* o =
+        static_cast<const __nv_bfloat16*>(a.out) + b * a.o_stride[0] + h * a.o_stride[1] + i * a.o_stride[2];
+    const __nv_bfloat16* d =
+        static_cast<const __nv_bfloat16*>(a.dout) + b * a.do_stride[0] + h * a.do_stride[1] + i * a.do_stride[2];
+    const uint4 ov = __ldg(reinterpret_cast<const uint4*>(o) + part);
+    const uint4 dv = __ldg(reinterpret_cast<const uint4*>(d) + part);
+    const __nv_bfloat162* op = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* dp = reinterpret_cast<const __nv_bfloat162*>(&dv);
+    float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) a.dsum[row] = acc;
+    for (int j = 0; j < 4; ++j) s2 = fma2(__bfloat1622float2(op[j]), __bfloat1622float2(dp[j]), s2);
+    acc = s2.x + s2.y;
+  }
+  for (int off = tpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (i < a.L && part == 0) a.dsum[(static_cast<int64_t>(b) * a.Hq + h) * a.L + i] = acc;
 }
 
 // Query-side lists: one thread per key tile n of row set (b, h).
@@ -845,8 +856,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, const BwdMaps& maps, cudaStream_t str
 }  // namespace
 
 cudaError_t launch_bwd(const BwdArgs& a, const BwdMaps& maps, cudaStream_t stream) {
-  const int64_t rows = static_cast<int64_t>(a.B) * a.Hq * a.L;
-  bwd_dsum_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(a);
+  const int rows_per_cta = 256 / (a.E >> 3);
+  bwd_dsum_kernel<<<dim3((a.L + rows_per_cta - 1) / rows_per_cta, a.Hq, a.B), 256, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return a.E == 64 ? launch_bwd_d<64>(a, maps, stream) : launch_bwd_d<128>(a, maps, stream);

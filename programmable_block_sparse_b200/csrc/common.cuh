@@ -99,6 +99,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Cluster launch control (sm_100): a running CTA asks the hardware to cancel
+// the launch of a CTA that has not started yet (the next one in launch
+// order) and does that CTA's work itself.  The 16-byte answer is written
+// asynchronously to `resp` (16-byte aligned shared memory) and completes
+// `bar`, which must expect 16 bytes.  After an answer that cancelled
+// nothing, no further request may be made.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                   smem_u32(resp)),
+               "r"(smem_u32(bar))
+               : "memory");
+}
+// Reads an answer: true with the cancelled CTA's index (x, y, z), or false.
+__device__ __forceinline__ bool clc_query(const void* resp, int& x, int& y, int& z) {
+  uint32_t ok = 0, cx = 0, cy = 0, cz = 0;
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b128 r;\n ld.shared.b128 r, [%4];\n"
+      " clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n selp.u32 %3, 1, 0, p;\n"
+      " @p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%0, %1, %2, _}, r;\n}\n"
+      : "+r"(cx), "+r"(cy), "+r"(cz), "+r"(ok)
+      : "r"(smem_u32(resp))
+      : "memory");
+  x = static_cast<int>(cx);
+  y = static_cast<int>(cy);
+  z = static_cast<int>(cz);
+  return ok != 0;
+}
+
+// ---------------------------------------------------------------------------
 // TMA (tiled bulk tensor copies, no multicast)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,

@@ -10,9 +10,12 @@
 // first); section "The compiler plugs local rules into the attention template"
 // (online softmax and tiling without materialising the score matrix).
 //
-// One CTA computes two adjacent 128-row query tiles (A = 2p, B = 2p + 1) of one
-// (batch, query head).  The two tiles' BlockMask lists are merged in key order
-// and every K/V tile of the union is loaded once for both:
+// A work item is two adjacent 128-row query tiles (A = 2p, B = 2p + 1) of one
+// (batch, query head).  The kernel is persistent, one CTA per SM, through
+// cluster launch control: a CTA that finishes an item takes over the launch
+// of the next CTA that has not started, longest items first.  The two
+// tiles' BlockMask lists are merged in key order and every K/V tile of the
+// union is loaded once for both:
 //   warp 0       TMA producer: Q_A, Q_B, then K_u, V_u of every union tile u
 //                into NS-stage rings (128 x 64 bf16 boxes, 128-byte swizzle).
 //   warp 1       TMEM allocator and MMA issuer (one elected thread):
@@ -40,6 +43,11 @@
 // second half of the softmax.
 // The running max only moves (and O rescales) when it grows by more than 2^8;
 // P then stays below 2^8 and the final O / l ratio is exact.
+//
+// Barrier phases and ring positions run on across items.  The next item's Q
+// is loaded once the current item's last QK has completed, and its first QKs
+// are issued as soon as the current item's last PVs are, so the next S is
+// computed while the softmax groups write the current item's output.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records FA_ERR_TIMEOUT
 // in the status word, stops issuing work, drains its own copies and MMAs
@@ -78,12 +86,17 @@ enum : uint32_t { kInA = 1, kFullA = 2, kInB = 4, kFullB = 8 };
 constexpr int kInfoFull = 1 << 30;  // class bit in the published tile info
 
 struct Barriers {
+  uint4 clc_resp[2];              // answers of the launch-control requests (16-byte aligned)
+  uint64_t clc_full[2];           // answer r has landed in clc_resp[r & 1]
+  uint64_t clc_empty[2];          // the MMA thread and the 8 softmax warps have read it
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
   uint64_t p_half[2];  // the first 64 keys' P is written: their PV may start
   uint64_t s_free[2], o_done[2];  // head dim 64 only: S read out / PV finished
-  uint64_t o_final;
+  uint64_t q_empty;               // the item's last QK is done: Q may be reloaded
+  uint64_t o_final[2];            // per group: the item's last PV is done
+  uint64_t mma_done;              // every MMA of the CTA has completed
   int info[2][2];  // per group, ring of 2: tile index | kFullA-style class bit
   uint32_t tmem_base;
   int abort;
@@ -139,6 +152,37 @@ struct UnionIter {
   }
 };
 
+// Work items.  A work item is a pair of adjacent query tiles of one (batch,
+// query head), one per CTA of the launch grid (head, batch, pair), with the
+// pair counted down in z: CTAs start in linear order (x fastest, z slowest),
+// so every (batch, head)'s last pairs -- under causal-like rules the longest
+// lists of key tiles -- come first and the short ones fill in at the end.
+// The kernel is persistent through cluster launch control: a running CTA
+// takes its own item, then repeatedly cancels the launch of the next CTA
+// that has not started and does that CTA's item, keeping its TMEM, barriers
+// and pipelines.  Items thus go, longest first, to whichever SM frees up.
+struct Item {
+  int h, b, mtA, mtB;
+  bool has_b;
+  int hk, S_b;
+  int64_t row_a;  // the block mask's list row of tile A
+};
+
+__device__ __forceinline__ Item item_of(const FwdArgs& a, int x, int y, int z) {
+  Item it;
+  const int pair = static_cast<int>(gridDim.z) - 1 - z;
+  it.h = x;
+  it.b = y;
+  it.mtA = 2 * pair;
+  it.mtB = 2 * pair + 1;
+  it.has_b = it.mtB < a.bm.Mb;
+  it.hk = it.h / a.G;
+  it.S_b = seq_len_b(a.mask, it.b, a.S);
+  const int bmb = a.bm.B > 1 ? it.b : 0, bmh = a.bm.H > 1 ? it.h : 0;
+  it.row_a = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb + it.mtA;
+  return it;
+}
+
 // Rarely run paths, kept out of line so the softmax loop stays compact in the
 // instruction cache: a composed mask rule's bits for one 32-key word, and the
 // hardware tanh of 64 columns (for a half whose arguments exceed the
@@ -165,10 +209,13 @@ __device__ __noinline__ void tanh_hw_tmem(uint32_t taddr, float c_in) {
 }
 
 // Softmax and epilogue of one 128-row query tile; runs on one warpgroup.
+// gbase counts the group's tiles of earlier work items and nfin the items in
+// which it had tiles (the phases of its barriers run on across items);
+// returns false once a wait gave up.
 template <int D, int SCORE>
-__device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, float (*s_pos)[kTile],
+__device__ __forceinline__ bool softmax_group(const FwdArgs& a, Barriers& bars, float (*s_pos)[kTile],
                                               int (*s_doc)[kTile], int X, int mt, int h, int b, int S_b,
-                                              int64_t row_a, bool has_b, uint32_t tbase) {
+                                              int64_t row_a, bool has_b, uint32_t tbase, int& gbase, int& nfin) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
@@ -219,23 +266,24 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   // gives up inside a tile marks the warp dead, it skips the rest of the tile
   // and votes false at the next barrier.
   for (; cnt < total; ++cnt) {
+    const int g = gbase + cnt;  // the group's tile count over all items so far
     // a warp-uniform result: the lanes leave the loop together or not at all
-    bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[X], cnt & 1, abort, a.status, a.wait_cycles));
-    const int info = ok ? bars.info[X][cnt & 1] : 0;
+    bool ok = alive && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[X], g & 1, abort, a.status, a.wait_cycles));
+    const int info = ok ? bars.info[X][g & 1] : 0;
     const int n = info & (kInfoFull - 1);
     const bool full = (info & kInfoFull) != 0;
     const int kv0 = n * kTile;
     const bool edge = kv0 + kTile > S_b;
     const bool stage_doc = is_doc && (!full || edge);  // the same for every row of the tile
     if (group_stage) {
-      // this tile's key-side values into smem (double-buffered by cnt & 1);
+      // this tile's key-side values into smem (double-buffered by g & 1);
       // every warp of the group reaches the barrier on every tile, and it
       // also tells each warp whether all four got their S, so that on a
       // timeout the group leaves together and no warp waits for another
       if (ok) {
         const int kv = kv0 + r;
-        if (has_pos) s_pos[cnt & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
-        if (stage_doc) s_doc[cnt & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
+        if (has_pos) s_pos[g & 1][r] = slope2 * static_cast<float>(pos_at(a.score, b, kv, a.S));
+        if (stage_doc) s_doc[g & 1][r] = kv < a.S ? __ldg(doc_row + kv) : -2;
       }
       ok = named_bar_and(1 + X, 128, ok);
     }
@@ -294,7 +342,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
           for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), splat2(-m_fold));
         } else if (has_pos) {
           // bias of column c: slope2 (p[kv] - p[q]) - m_fold, p[kv] staged in smem
-          const float2* pk = reinterpret_cast<const float2*>(s_pos[cnt & 1] + c0);
+          const float2* pk = reinterpret_cast<const float2*>(s_pos[g & 1] + c0);
           const float2 b0 = splat2(-pq_scaled - m_fold);
 #pragma unroll
           for (int i = 0; i < 32; ++i) t2[i] = fma2(th[i], splat2(c_out), add2(pk[i], b0));
@@ -314,7 +362,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
           const int base = kv0 + c0 + 32 * w;
           uint32_t same = 0xFFFFFFFFu;  // same-document bits of the word's keys
           if (stage_doc) {
-            const int* dk = s_doc[cnt & 1] + c0 + 32 * w;
+            const int* dk = s_doc[g & 1] + c0 + 32 * w;
             same = 0u;
 #pragma unroll
             for (int i = 0; i < 32; ++i) same |= (dk[i] == my_doc ? 1u : 0u) << i;
@@ -348,12 +396,14 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
     // O_X holds a sum only after the group's first tile (its first PV
     // overwrites whatever the columns held)
     const bool rescale = grow_max && cnt > 0;
+    // the first tile of an item needs no wait: the previous item's last PV
+    // was covered by that item's o_final
     bool pv_done = !kSepP || cnt == 0;
     auto wait_pv = [&]() {
       // the previous tile's PV reads P and writes O; with separate S columns
       // the S of this tile may have landed before that PV finished
       if (!pv_done) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[X], (cnt - 1) & 1, abort, a.status, a.wait_cycles))) alive = false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[X], (g - 1) & 1, abort, a.status, a.wait_cycles))) alive = false;
         tc_fence_after();
         pv_done = true;
       }
@@ -427,8 +477,10 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
   }
 
   // ------------------------------------------------------------- epilogue
+  gbase += cnt;
   if (alive && cnt > 0) {
-    alive = mbar_wait(&bars.o_final, 0, abort, a.status, a.wait_cycles);
+    alive = mbar_wait(&bars.o_final[X], nfin & 1, abort, a.status, a.wait_cycles);
+    ++nfin;
     tc_fence_after();
   }
   // TMEM loads are warp-collective: every lane takes part, rows past L
@@ -471,6 +523,7 @@ __device__ __forceinline__ void softmax_group(const FwdArgs& a, Barriers& bars, 
       }
     }
   }
+  return alive;
 }
 
 template <int D, int SCORE>
@@ -489,22 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = sK + NS * C::kTileBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Blocks start in linear order (x fastest, z slowest): with the query-tile
-  // pair in z, counted down, every (batch, head)'s last pairs -- the longest
-  // rows of tiles under causal-like rules -- start first and the short ones
-  // fill in at the end, instead of long CTAs starting in the last wave.
-  const int pair = gridDim.z - 1 - blockIdx.z;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int mtA = 2 * pair, mtB = 2 * pair + 1;
-  const bool has_b = mtB < a.bm.Mb;
-  const int hk = h / a.G;
-  const int S_b = seq_len_b(a.mask, b, a.S);
-  const int bmb = a.bm.B > 1 ? b : 0, bmh = a.bm.H > 1 ? h : 0;
-  const int64_t row_a = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb + mtA;
   volatile int* abort = &bars.abort;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
@@ -517,8 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.p_half[i], 4);
       mbar_init(&bars.s_free[i], 4);
       mbar_init(&bars.o_done[i], 1);
+      mbar_init(&bars.o_final[i], 1);
     }
-    mbar_init(&bars.o_final, 1);
+    mbar_init(&bars.mma_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.clc_full[i], 1);   // the producer's arrive with the 16-byte expectation
+      mbar_init(&bars.clc_empty[i], 9);  // the MMA thread + 8 softmax warps
+    }
     bars.abort = 0;
     mbar_fence_init();
   }
@@ -530,33 +577,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA
+    // One ring position u per union tile, counted over all of the CTA's
+    // items; Q of the next item is loaded as soon as the current item's last
+    // QK has completed (q_empty), while its last tiles are still in flight.
+    // This thread also makes the launch-control requests: request r, made
+    // once the loads of item r are issued (a few tiles before the item ends,
+    // so that the next item goes to the SM that frees up first), names item
+    // r + 1.
     if (lane == 0) {
-      UnionIter it;
-      it.init(a, row_a, has_b);
-      int n;
-      uint32_t flags;
-      bool any = it.next(n, flags);
-      if (any) {
-        tma_prefetch_desc(&map_k);
-        tma_prefetch_desc(&map_v);
-        mbar_expect_tx(&bars.q_full, (has_b ? 2 : 1) * C::kTileBytes);
-        for (int c = 0; c < C::kBoxes; ++c) {
-          tma_load_4d(sQ + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mtA * kTile, h, b);
-          if (has_b)
-            tma_load_4d(sQ + C::kTileBytes + c * (kTile * 128), &map_q, &bars.q_full, c * 64, mtB * kTile, h, b);
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      int u = 0, nq = 0, issued_k = 0, issued_v = 0, requests = 0;
+      bool ok = true;
+      int cx = blockIdx.x, cy = blockIdx.y, cz = blockIdx.z;
+      for (int r = 0; ok && !*abort; ++r) {
+        const Item itm = item_of(a, cx, cy, cz);
+        UnionIter it;
+        it.init(a, itm.row_a, itm.has_b);
+        int n;
+        uint32_t flags;
+        bool any = it.next(n, flags);  // false: no tile for either query tile
+        if (any && nq > 0 && !mbar_wait(&bars.q_empty, (nq - 1) & 1, abort, a.status, a.wait_cycles)) break;
+        if (any) {
+          mbar_expect_tx(&bars.q_full, (itm.has_b ? 2 : 1) * C::kTileBytes);
+          for (int c = 0; c < C::kBoxes; ++c) {
+            tma_load_4d(sQ + c * (kTile * 128), &map_q, &bars.q_full, c * 64, itm.mtA * kTile, itm.h, itm.b);
+            if (itm.has_b)
+              tma_load_4d(sQ + C::kTileBytes + c * (kTile * 128), &map_q, &bars.q_full, c * 64, itm.mtB * kTile, itm.h,
+                          itm.b);
+          }
+          ++nq;
         }
-        int u = 0, issued_k = 0, issued_v = 0;
-        for (; any && !*abort; ++u, any = it.next(n, flags)) {
+        for (; any; ++u, any = it.next(n, flags)) {
           const int s = u % NS;
           const uint32_t round = u / NS;
-          if (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
+          if (*abort || (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles))) {
+            ok = false;
+            break;
+          }
           // a paged pool is read in two 64-key boxes per tile, each from its
           // own page (the swizzle follows the smem address, so the halves
           // land exactly as one 128-row box would)
-          int pg0 = b, pg1 = b, row0 = n * kTile, row1 = n * kTile + 64;
+          int pg0 = itm.b, pg1 = itm.b, row0 = n * kTile, row1 = n * kTile + 64;
           if (a.page_table) {
-            pg0 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, n * kTile);
-            pg1 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, b, n * kTile + 64);
+            pg0 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, itm.b, n * kTile);
+            pg1 = cache_page(a.page_table, a.pages_per_seq, a.page_size, a.num_pages, a.status, itm.b, n * kTile + 64);
             row0 = (n * kTile) % a.page_size;
             row1 = (n * kTile + 64) % a.page_size;
           }
@@ -564,38 +630,52 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < C::kBoxes; ++c) {
             uint8_t* dst = sK + s * C::kTileBytes + c * (kTile * 128);
             if (a.page_table) {
-              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, row0, hk, pg0);
-              tma_load_4d(dst + 64 * 128, &map_k, &bars.k_full[s], c * 64, row1, hk, pg1);
+              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, row0, itm.hk, pg0);
+              tma_load_4d(dst + 64 * 128, &map_k, &bars.k_full[s], c * 64, row1, itm.hk, pg1);
             } else {
-              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, n * kTile, hk, b);
+              tma_load_4d(dst, &map_k, &bars.k_full[s], c * 64, n * kTile, itm.hk, itm.b);
             }
           }
           issued_k = u + 1;
-          if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) break;
+          if (u >= NS && !mbar_wait(&bars.v_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(&bars.v_full[s], C::kTileBytes);
           for (int c = 0; c < C::kBoxes; ++c) {
             uint8_t* dst = sV + s * C::kTileBytes + c * (kTile * 128);
             if (a.page_table) {
-              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, row0, hk, pg0);
-              tma_load_4d(dst + 64 * 128, &map_v, &bars.v_full[s], c * 64, row1, hk, pg1);
+              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, row0, itm.hk, pg0);
+              tma_load_4d(dst + 64 * 128, &map_v, &bars.v_full[s], c * 64, row1, itm.hk, pg1);
             } else {
-              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, n * kTile, hk, b);
+              tma_load_4d(dst, &map_v, &bars.v_full[s], c * 64, n * kTile, itm.hk, itm.b);
             }
           }
           issued_v = u + 1;
         }
-        // Drain on every path: each copy this thread issued lands before it
-        // leaves, so the CTA never exits with copies in flight, even when
-        // another warp gives up after this loop has ended.  Only the last NS
-        // of each ring can be pending (earlier slots were waited free before
-        // reuse); on the normal path they have landed already.
-        volatile int never = 0;
-        mbar_wait(&bars.q_full, 0, &never, nullptr);
-        for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
-          mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
-        for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
-          mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
+        if (!ok) break;
+        // request r into answer slot r & 1, once its previous answer is read;
+        // the next item, if it cancelled a CTA
+        if (r >= 2 && !mbar_wait(&bars.clc_empty[r & 1], ((r >> 1) - 1) & 1, abort, a.status, a.wait_cycles)) break;
+        mbar_expect_tx(&bars.clc_full[r & 1], 16);
+        clc_try_cancel(&bars.clc_resp[r & 1], &bars.clc_full[r & 1]);
+        requests = r + 1;
+        if (!mbar_wait(&bars.clc_full[r & 1], (r >> 1) & 1, abort, a.status, a.wait_cycles)) break;
+        if (!clc_query(&bars.clc_resp[r & 1], cx, cy, cz)) break;
       }
+      // Drain on every path: each copy and request this thread issued lands
+      // before it leaves, so the CTA never exits with one in flight, even
+      // when another warp gives up after this loop has ended.  Only the last
+      // request, the last Q and the last NS of each ring can be pending
+      // (earlier ones were waited on before reuse); on the normal path they
+      // have landed already.
+      volatile int never = 0;
+      if (requests > 0) mbar_wait(&bars.clc_full[(requests - 1) & 1], ((requests - 1) >> 1) & 1, &never, nullptr);
+      if (nq > 0) mbar_wait(&bars.q_full, (nq - 1) & 1, &never, nullptr);
+      for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
+        mbar_wait(&bars.k_full[j % NS], (j / NS) & 1, &never, nullptr);
+      for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
+        mbar_wait(&bars.v_full[j % NS], (j / NS) & 1, &never, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
@@ -609,14 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dk0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dv0 = umma_desc_sw128(smem_u32(sV), kTile * 128, 1024);
       constexpr uint32_t kTileStep = C::kTileBytes >> 4;
-      UnionIter it;
-      it.init(a, row_a, has_b);
-      int n_cur, n_nxt = 0;
-      uint32_t f_cur, f_nxt = 0;
-      bool have_cur = it.next(n_cur, f_cur);
-      int pcnt[2] = {0, 0};  // P tiles consumed per group
+      // counters over all of the CTA's items: ring position, P tiles consumed,
+      // QK tiles issued and S tiles read out per group, Q tiles loaded
+      int u = 0, nq = 0;
+      int pcnt[2] = {0, 0}, qcnt[2] = {0, 0}, freed[2] = {0, 0};
       bool acc[2] = {false, false};
-      int qcnt[2] = {0, 0};  // QK tiles issued per group
       auto issue_qk = [&](int X, int s, int n, uint32_t flags) {
         // publish the tile index and class for the softmax group (released by
         // this thread's arrive; the phase completes with the MMA commit below)
@@ -632,9 +709,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(&bars.s_full[X]);
       };
+      // O_X += P_X V (the item's first PV of a group overwrites O_X); head
+      // dim 64 has P and O in columns of their own and signals o_done
       auto issue_pv = [&](int X, int s) -> bool {
         const uint64_t dv = dv0 + s * kTileStep;
-        const uint32_t o_tmem = tbase + 256u * X + 128u, p_tmem = tbase + 256u * X;
+        const uint32_t o_tmem = tbase + 256u * X + (D == 64 ? 192u : 128u);
+        const uint32_t p_tmem = tbase + 256u * X + (D == 64 ? 128u : 0u);
         const uint32_t acc0 = acc[X] ? 1u : 0u;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -645,118 +725,96 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
             umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
         }
+        if (D == 64) umma_commit(&bars.o_done[X]);
         acc[X] = true;
         ++pcnt[X];
         return true;
       };
-      bool ok = have_cur && mbar_wait(&bars.q_full, 0, abort, a.status, a.wait_cycles);
-      if constexpr (D == 64) {
-        // S, P and O in separate columns: the next tile's QK of a group goes
-        // in as soon as its softmax has read S (s_free), ahead of this
-        // tile's PV (p_full), so the next S is ready when the softmax needs it.
-        int freed[2] = {0, 0};  // S tiles of each group read out so far
-        auto issue_pv_sep = [&](int X, int s) -> bool {
-          const uint64_t dv = dv0 + s * kTileStep;
-          const uint32_t o_tmem = tbase + 256u * X + 192u, p_tmem = tbase + 256u * X + 128u;
-          const uint32_t acc0 = acc[X] ? 1u : 0u;
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            if (!mbar_wait(hf == 0 ? &bars.p_half[X] : &bars.p_full[X], pcnt[X] & 1, abort, a.status, a.wait_cycles)) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
-              umma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-          }
-          umma_commit(&bars.o_done[X]);
-          acc[X] = true;
-          ++pcnt[X];
-          return true;
-        };
-        auto qk_after_free = [&](int X, int s, int n, uint32_t flags) -> bool {
-          if (qcnt[X] > 0) {  // the group's previous S must be read out first
-            if (!mbar_wait(&bars.s_free[X], freed[X] & 1, abort, a.status, a.wait_cycles)) return false;
-            ++freed[X];
-            tc_fence_after();
-          }
-          issue_qk(X, s, n, flags);
-          return true;
-        };
-        if (ok) {
-          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status, a.wait_cycles);
+      // head dim 64: a group's QK waits until its softmax has read the
+      // previous S (s_free), possibly of the previous item
+      auto qk_after_free = [&](int X, int s, int n, uint32_t flags) -> bool {
+        if (D == 64 && qcnt[X] > 0) {
+          if (!mbar_wait(&bars.s_free[X], freed[X] & 1, abort, a.status, a.wait_cycles)) return false;
+          ++freed[X];
           tc_fence_after();
-          if (ok && (f_cur & kInA)) ok = qk_after_free(0, 0, n_cur, f_cur);
-          if (ok && (f_cur & kInB)) ok = qk_after_free(1, 0, n_cur, f_cur);
-          if (ok) umma_commit(&bars.k_empty[0]);
         }
-        for (int u = 0; ok && have_cur; ++u) {
+        issue_qk(X, s, n, flags);
+        return true;
+      };
+      bool ok = true;
+      int cx = blockIdx.x, cy = blockIdx.y, cz = blockIdx.z;
+      for (int r = 0; ok && !*abort; ++r) {
+        const Item itm = item_of(a, cx, cy, cz);
+        UnionIter it;
+        it.init(a, itm.row_a, itm.has_b);
+        int n_cur, n_nxt = 0;
+        uint32_t f_cur, f_nxt = 0;
+        bool have_cur = it.next(n_cur, f_cur);  // false: no tile for either query tile
+        acc[0] = acc[1] = false;
+        if (have_cur) {
+          ok = mbar_wait(&bars.q_full, nq & 1, abort, a.status, a.wait_cycles);
+          ++nq;
+          if (ok) ok = mbar_wait(&bars.k_full[u % NS], (u / NS) & 1, abort, a.status, a.wait_cycles);
+          tc_fence_after();
+          if (ok && (f_cur & kInA)) ok = qk_after_free(0, u % NS, n_cur, f_cur);
+          if (ok && (f_cur & kInB)) ok = qk_after_free(1, u % NS, n_cur, f_cur);
+          if (ok) umma_commit(&bars.k_empty[u % NS]);
+        }
+        for (; ok && have_cur; ++u) {
           const int s = u % NS, s1 = (u + 1) % NS;
           const bool have_nxt = it.next(n_nxt, f_nxt);
+          // every QK of the item is issued: Q may be reloaded once they are done
+          if (!have_nxt) umma_commit(&bars.q_empty);
           bool k_ready = false, v_ready = false;
-          for (int X = 0; X < 2 && ok; ++X) {
-            const uint32_t in_x = X == 0 ? kInA : kInB;
-            if (have_nxt && (f_nxt & in_x)) {
-              if (!k_ready) {
-                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
-                tc_fence_after();
-                k_ready = true;
+          if constexpr (D == 64) {
+            // S, P and O in separate columns: the next tile's QK of a group
+            // goes in as soon as its softmax has read S, ahead of this
+            // tile's PV, so the next S is ready when the softmax needs it.
+            for (int X = 0; X < 2 && ok; ++X) {
+              const uint32_t in_x = X == 0 ? kInA : kInB;
+              if (have_nxt && (f_nxt & in_x)) {
+                if (!k_ready) {
+                  ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
+                  tc_fence_after();
+                  k_ready = true;
+                }
+                if (ok) ok = qk_after_free(X, s1, n_nxt, f_nxt);
               }
-              if (ok) ok = qk_after_free(X, s1, n_nxt, f_nxt);
+              if (ok && (f_cur & in_x)) {
+                if (!v_ready) {
+                  ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles);
+                  tc_fence_after();
+                  v_ready = true;
+                }
+                if (ok) ok = issue_pv(X, s);
+              }
             }
-            if (ok && (f_cur & in_x)) {
-              if (!v_ready) {
-                ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles);
-                tc_fence_after();
-                v_ready = true;
+          } else {
+            // P_X shares the S columns: PV_X of this tile, then QK_X of the next
+            ok = mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles);
+            tc_fence_after();
+            for (int X = 0; X < 2 && ok; ++X) {
+              const uint32_t in_x = X == 0 ? kInA : kInB;
+              if (f_cur & in_x) ok = issue_pv(X, s);
+              if (ok && have_nxt && (f_nxt & in_x)) {
+                if (!k_ready) {
+                  ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
+                  tc_fence_after();
+                  k_ready = true;
+                }
+                if (ok) issue_qk(X, s1, n_nxt, f_nxt);
               }
-              if (ok) ok = issue_pv_sep(X, s);
             }
           }
           if (!ok) break;
           // every union tile is some group's tile, and so is the next one
           umma_commit(&bars.v_empty[s]);
           if (have_nxt) {
-            if (!k_ready && !mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles)) break;
-            umma_commit(&bars.k_empty[s1]);
-          }
-          have_cur = have_nxt;
-          n_cur = n_nxt;
-          f_cur = f_nxt;
-        }
-      } else {
-        if (ok) {
-          ok = mbar_wait(&bars.k_full[0], 0, abort, a.status, a.wait_cycles);
-          tc_fence_after();
-          if (ok) {
-            if (f_cur & kInA) issue_qk(0, 0, n_cur, f_cur);
-            if (f_cur & kInB) issue_qk(1, 0, n_cur, f_cur);
-            umma_commit(&bars.k_empty[0]);
-          }
-        }
-        for (int u = 0; ok && have_cur; ++u) {
-          const int s = u % NS, s1 = (u + 1) % NS;
-          const bool have_nxt = it.next(n_nxt, f_nxt);
-          bool k_nxt_ready = false;
-          if (!mbar_wait(&bars.v_full[s], (u / NS) & 1, abort, a.status, a.wait_cycles)) break;
-          for (int X = 0; X < 2 && ok; ++X) {
-            const uint32_t in_x = X == 0 ? kInA : kInB;
-            if (f_cur & in_x) ok = issue_pv(X, s);
-            if (ok && have_nxt && (f_nxt & in_x)) {
-              if (!k_nxt_ready) {
-                ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
-                tc_fence_after();
-                k_nxt_ready = true;
-              }
-              if (ok) issue_qk(X, s1, n_nxt, f_nxt);
-            }
-          }
-          if (!ok) break;
-          umma_commit(&bars.v_empty[s]);
-          if (have_nxt) {
-            if (!k_nxt_ready) {
-              // K_{u+1} is listed for neither group's next QK only if a group
-              // skips it; it still has to be consumed before its slot is reused
-              ok = mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles);
-              if (!ok) break;
+            // K_{u+1} is listed for neither group's next QK only if a group
+            // skips it; it still has to be consumed before its slot is reused
+            if (!k_ready && !mbar_wait(&bars.k_full[s1], ((u + 1) / NS) & 1, abort, a.status, a.wait_cycles)) {
+              ok = false;
+              break;
             }
             umma_commit(&bars.k_empty[s1]);
           }
@@ -764,18 +822,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           n_cur = n_nxt;
           f_cur = f_nxt;
         }
+        // the item's O of each group with tiles is complete once these land
+        if (!ok) break;
+        if (acc[0]) umma_commit(&bars.o_final[0]);
+        if (acc[1]) umma_commit(&bars.o_final[1]);
+        // the next item, if request r cancelled a CTA
+        if (!mbar_wait(&bars.clc_full[r & 1], (r >> 1) & 1, abort, a.status, a.wait_cycles)) break;
+        const bool more = clc_query(&bars.clc_resp[r & 1], cx, cy, cz);
+        mbar_arrive(&bars.clc_empty[r & 1]);
+        if (!more) break;
       }
-      (void)n_cur;
-      // every MMA issued above completes before the epilogue or TMEM release
-      umma_commit(&bars.o_final);
+      // every MMA issued above completes before TMEM is released
+      umma_commit(&bars.mma_done);
       volatile int never = 0;
-      mbar_wait(&bars.o_final, 0, &never, nullptr);
+      mbar_wait(&bars.mma_done, 0, &never, nullptr);
     }
   } else {
     // -------------------------------------------------------------- softmax
-    // warps 2-5: tile A, warps 6-9: tile B; warp % 4 is the TMEM lane quadrant
+    // warps 2-5: tile A, warps 6-9: tile B; warp % 4 is the TMEM lane quadrant.
+    // The group's four warps agree at each item whether to go on (a warp
+    // that gave up inside an item leaves with its group).
     const int X = (warp - 2) >> 2;
-    softmax_group<D, SCORE>(a, bars, s_pos[X], s_doc[X], X, X == 0 ? mtA : mtB, h, b, S_b, row_a, has_b, tbase);
+    int gbase = 0, nfin = 0;
+    bool go = true;
+    int cx = blockIdx.x, cy = blockIdx.y, cz = blockIdx.z;
+    for (int r = 0; named_bar_and(1 + X, 128, go); ++r) {
+      const Item itm = item_of(a, cx, cy, cz);
+      const bool alive = softmax_group<D, SCORE>(a, bars, s_pos[X], s_doc[X], X, X == 0 ? itm.mtA : itm.mtB, itm.h,
+                                                 itm.b, itm.S_b, itm.row_a, itm.has_b, tbase, gbase, nfin);
+      // the next item, if request r cancelled a CTA (the answer is the same
+      // for all four warps, so they go on or stop together)
+      bool more = false;
+      if (alive && __all_sync(0xffffffffu, mbar_wait(&bars.clc_full[r & 1], (r >> 1) & 1, abort, a.status, a.wait_cycles))) {
+        more = clc_query(&bars.clc_resp[r & 1], cx, cy, cz);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.clc_empty[r & 1]);
+      }
+      go = alive && more;
+    }
   }
 
   tc_fence_before();
@@ -789,6 +873,8 @@ cudaError_t launch_one(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t str
   auto kern = fwd_sm100_kernel<D, SCORE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // one CTA per work item; the CTAs that start first (one per SM: shared
+  // memory and TMEM allow no second) take over the launches of the rest
   dim3 grid(a.Hq, a.B, (a.bm.Mb + 1) / 2);
   kern<<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(a, maps.q, maps.k, maps.v);
   return cudaGetLastError();

@@ -61,6 +61,7 @@ cudaError_t launch_fwd_simt(const FwdArgs& a, cudaStream_t stream);
 struct Sm100Maps {
   CUtensorMap q, k, v;
 };
+// One CTA per pair of query tiles, persistent through cluster launch control.
 cudaError_t launch_fwd_sm100(const FwdArgs& a, const Sm100Maps& maps, cudaStream_t stream);
 
 // Split-KV decode for short queries (bf16, E = Ev in {64, 128}, L <= 16) and

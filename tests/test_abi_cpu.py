@@ -275,6 +275,8 @@ def test_backward_checked_on_the_host(lib):
     assert call(ws_bytes=16) == 10                                          # workspace
     assert call(lse=None) == 1
     assert call(dk=_t(2, 4, 256, 64, stride=(4 * 256 * 64, 256 * 64, 64, 2))) == 8
+    assert call(o=_t(2, 4, 256, 64, addr=FAKE + 2)) == 8                    # out read with 16-byte loads
+    assert call(o=_t(2, 4, 256, 64, stride=(4 * 256 * 68, 256 * 68, 68 + 1, 1))) == 8
     n = C.c_size_t()
     assert lib.flexattn_backward_workspace_size(C.byref(q), C.byref(n)) == 0 and n.value == 2 * 4 * 256 * 4
 
