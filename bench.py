@@ -86,11 +86,11 @@ HEADLINE = BENCH_ITEMS[0][0]
 # workload is stated in the profile it comes from.
 NCU_TRAFFIC = {
     # fwd_sm100_kernel<128, 0>, captured at batch 1 (profiles/fwd_sm100_gqa_sliding_window.md): x 2 sequences
-    "gqa_sliding_window": {"bytes": 2 * (201745152 + 94600448), "source_hash": "f65fafb4a06d314c"},
+    "gqa_sliding_window": {"bytes": 2 * (201698816 + 94893312), "source_hash": "7a8c170bdf2d59bb"},
     # fwd_sm100_kernel<64, 3> / <128, 3>, full size (profiles/fwd_sm100_causal_packed_sliver.md)
-    "causal_softcap_alibi": {"bytes": 50419968 + 782848, "source_hash": "f65fafb4a06d314c"},
-    "packed_docs": {"bytes": 100836352 + 9787648, "source_hash": "f65fafb4a06d314c"},
-    "sliver_every_fourth_key": {"bytes": 50427392 + 771584, "source_hash": "f65fafb4a06d314c"},
+    "causal_softcap_alibi": {"bytes": 50420480 + 684288, "source_hash": "7a8c170bdf2d59bb"},
+    "packed_docs": {"bytes": 100907776 + 10119424, "source_hash": "7a8c170bdf2d59bb"},
+    "sliver_every_fourth_key": {"bytes": 50427392 + 745216, "source_hash": "7a8c170bdf2d59bb"},
     # decode_tc_kernel<128, 1>, captured at batch 16 (profiles/decode_tc_kernel_decode_kv_cache.md):
     # x 614602 / 296926 cached tokens
     "decode_kv_cache": {"bytes": round((1222132224 + 8572672) * 614602 / 296926), "source_hash": "66031533768da397"},

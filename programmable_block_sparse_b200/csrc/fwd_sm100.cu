@@ -494,31 +494,36 @@ __device__ __forceinline__ bool softmax_group(const FwdArgs& a, Barriers& bars, 
     const int64_t rid = (static_cast<int64_t>(b) * a.Hq + h) * a.L + grow;
     if (row_ok && a.lse) a.lse[rid] = live ? (m_ref + log2f(l_sum)) * kLn2 : -INFINITY;
     if (row_ok && a.max_scores) a.max_scores[rid] = m_true * kLn2;
+    // O comes out of TMEM 64 columns per wait (four loads in flight)
 #pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t rr[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) rr[i] = 0u;
+    for (int cb = 0; cb < D / 64; ++cb) {
+      float o64[64];
       if (cnt > 0) {
-        tmem_ld16(tbase + lane_base + col_o + c * 16, rr);
-        tmem_wait_ld();
+        tmem_load64(tbase + lane_base + col_o + cb * 64, o64);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) o64[i] = 0.0f;
       }
-      if (row_ok) {
-        if (a.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow_off + c * 16);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = live ? make_float4(__uint_as_float(rr[4 * i]) * inv, __uint_as_float(rr[4 * i + 1]) * inv,
-                                        __uint_as_float(rr[4 * i + 2]) * inv, __uint_as_float(rr[4 * i + 3]) * inv)
-                          : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        } else {
-          uint32_t pk[8];
+      for (int c = 4 * cb; c < 4 * cb + 4; ++c) {
+        const uint32_t* rr = reinterpret_cast<const uint32_t*>(o64) + 16 * (c - 4 * cb);
+        if (row_ok) {
+          if (a.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow_off + c * 16);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow_off + c * 16);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int i = 0; i < 4; ++i)
+              dst[i] = live ? make_float4(__uint_as_float(rr[4 * i]) * inv, __uint_as_float(rr[4 * i + 1]) * inv,
+                                          __uint_as_float(rr[4 * i + 2]) * inv, __uint_as_float(rr[4 * i + 3]) * inv)
+                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          } else {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = live ? pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv) : 0u;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow_off + c * 16);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
       }
     }
@@ -581,9 +586,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // items; Q of the next item is loaded as soon as the current item's last
     // QK has completed (q_empty), while its last tiles are still in flight.
     // This thread also makes the launch-control requests: request r, made
-    // once the loads of item r are issued (a few tiles before the item ends,
-    // so that the next item goes to the SM that frees up first), names item
-    // r + 1.
+    // just before the last tile of item r is loaded (a few tiles before the
+    // item ends, so that the next item goes to the SM that frees up first),
+    // names item r + 1.
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
@@ -609,10 +614,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++nq;
         }
-        for (; any; ++u, any = it.next(n, flags)) {
+        // request r, into answer slot r & 1 once its previous answer is read,
+        // is made just before the item's last tile is loaded
+        bool requested = false;
+        auto request = [&]() -> bool {
+          if (r >= 2 && !mbar_wait(&bars.clc_empty[r & 1], ((r >> 1) - 1) & 1, abort, a.status, a.wait_cycles))
+            return false;
+          mbar_expect_tx(&bars.clc_full[r & 1], 16);
+          clc_try_cancel(&bars.clc_resp[r & 1], &bars.clc_full[r & 1]);
+          requests = r + 1;
+          requested = true;
+          return true;
+        };
+        for (; any; ++u) {
+          int n_nxt = 0;
+          uint32_t f_nxt = 0;
+          const bool have_nxt = it.next(n_nxt, f_nxt);
           const int s = u % NS;
           const uint32_t round = u / NS;
-          if (*abort || (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles))) {
+          if (*abort || (!have_nxt && !request()) ||
+              (u >= NS && !mbar_wait(&bars.k_empty[s], (round - 1) & 1, abort, a.status, a.wait_cycles))) {
             ok = false;
             break;
           }
@@ -652,14 +673,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           issued_v = u + 1;
+          n = n_nxt;
+          flags = f_nxt;
+          any = have_nxt;
         }
         if (!ok) break;
-        // request r into answer slot r & 1, once its previous answer is read;
-        // the next item, if it cancelled a CTA
-        if (r >= 2 && !mbar_wait(&bars.clc_empty[r & 1], ((r >> 1) - 1) & 1, abort, a.status, a.wait_cycles)) break;
-        mbar_expect_tx(&bars.clc_full[r & 1], 16);
-        clc_try_cancel(&bars.clc_resp[r & 1], &bars.clc_full[r & 1]);
-        requests = r + 1;
+        if (!requested && !request()) break;  // an item without tiles
+        // the next item, if request r cancelled a CTA
         if (!mbar_wait(&bars.clc_full[r & 1], (r >> 1) & 1, abort, a.status, a.wait_cycles)) break;
         if (!clc_query(&bars.clc_resp[r & 1], cx, cy, cz)) break;
       }

@@ -152,6 +152,20 @@ def test_fully_masked_rows_give_zero_and_neg_inf():
     _status_ok()
 
 
+@pytest.mark.parametrize("E", [64, 128])
+def test_persistent_prefill_with_empty_items(E):
+    """More pairs of query tiles than SMs (384), so running CTAs take over
+    the launches of the rest, and some pairs without a single key tile: a
+    sequence with no valid key, and, under bottom-right causal with L > S,
+    the query tiles before the first visible key."""
+    case = Case(4, 16, 8, 1300, 1000, E, E, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 30.0}, seed=21,
+                kv_len=[1000, 0, 513, 777], sentinel_tail=True)
+    out, lse = case.run(128, 128, split_kv=1)
+    assert torch.all(out[1] == 0) and torch.all(lse[1] == -math.inf)
+    assert_close(case, out, lse, *case.oracle())
+    _status_ok()
+
+
 def test_kv_len_tails_never_leak():
     """Cache positions past the valid length hold +-1e4; they must not reach the output."""
     for dtype in ("fp32", "bf16"):
