@@ -98,8 +98,8 @@ NCU_TRAFFIC = {
                            "source_hash": "66031533768da397"},
     # bwd_dkdv_kernel (the larger of the two backward kernels), full size
     # (profiles/bwd_dkdv_dq_backward.md)
-    "backward_causal_softcap_alibi": {"bytes": 69229056 + 7497984, "source_hash": "fd297535d8b984d1"},
-    "backward_packed_docs": {"bytes": 136204544 + 36972288, "source_hash": "fd297535d8b984d1"},
+    "backward_causal_softcap_alibi": {"bytes": 68308736 + 7811072, "source_hash": "6a65fba814bf1a59"},
+    "backward_packed_docs": {"bytes": 135514112 + 36383488, "source_hash": "6a65fba814bf1a59"},
 }
 
 KERNEL_SOURCES = {

@@ -102,6 +102,32 @@ __device__ __forceinline__ void tanh32(const uint32_t (&sr)[32], float c_in, flo
   }
 }
 
+// Ties 16 registers written by tcgen05.ld to a point after tcgen05.wait::ld,
+// so that no use of them is scheduled before the wait.
+__device__ __forceinline__ void hold16(uint32_t (&x)[16]) {
+  asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7]),
+               "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]));
+}
+
+// Writes 16 fp32 accumulator columns of a row, times `mul`, as fp32 or bf16
+// with 16-byte stores (the gradient tensors are 16-byte aligned).
+__device__ __forceinline__ void store16(void* base, int64_t off, bool f32, const uint32_t* rr, float mul) {
+  if (f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = make_float4(__uint_as_float(rr[4 * i]) * mul, __uint_as_float(rr[4 * i + 1]) * mul,
+                           __uint_as_float(rr[4 * i + 2]) * mul, __uint_as_float(rr[4 * i + 3]) * mul);
+  } else {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * mul, __uint_as_float(rr[2 * i + 1]) * mul);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + off);
+    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  }
+}
+
 // Loads tiles into smem boxes of 64 columns x 128 rows (128-byte swizzle).
 template <int D>
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int h, int b) {
@@ -364,28 +390,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (__all_sync(0xffffffffu, alive)) {
       const int64_t off = b * a.dq_stride[0] + h * a.dq_stride[1] + static_cast<int64_t>(row_ok ? grow : 0) * a.dq_stride[2];
+      // this group's D / 2 columns of dQ, all loads in flight before one wait
+      constexpr int kChunks = D / 32;
+      uint32_t rr[kChunks][16];
+      if (total > 0) {
 #pragma unroll
-      for (int c = jg * (D / 32); c < (jg + 1) * (D / 32); ++c) {
-        uint32_t rr[16];
+        for (int i = 0; i < kChunks; ++i) tmem_ld16(tbase + lane_base + 256 + (jg * kChunks + i) * 16, rr[i]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) rr[i] = 0u;
-        if (total > 0) {
-          tmem_ld16(tbase + lane_base + 256 + c * 16, rr);
-          tmem_wait_ld();
-        }
-        if (row_ok) {
-          if (a.dq_f32) {
-            float* dst = static_cast<float*>(a.dq) + off + c * 16;
+        for (int i = 0; i < kChunks; ++i) hold16(rr[i]);
+      } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) dst[i] = __uint_as_float(rr[i]) * a.scale;
-          } else {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.dq) + off + c * 16;
+        for (int i = 0; i < kChunks; ++i)
 #pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              *reinterpret_cast<uint32_t*>(dst + i) =
-                  pack_bf16x2(__uint_as_float(rr[i]) * a.scale, __uint_as_float(rr[i + 1]) * a.scale);
-          }
-        }
+          for (int e = 0; e < 16; ++e) rr[i][e] = 0u;
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) store16(a.dq, off + (jg * kChunks + i) * 16, a.dq_f32, rr[i], a.scale);
       }
     }
   }
@@ -723,27 +745,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool f32 = which ? a.dk_f32 : a.dv_f32;
         const float mul = which ? a.scale : 1.0f;
         const int64_t off = b * st[0] + hk * st[1] + static_cast<int64_t>(kvr) * st[2];
+        // 64 columns per wait (four loads in flight)
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t rr[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rr[i] = 0u;
+        for (int cb = 0; cb < D / 64; ++cb) {
+          uint32_t rr[4][16];
           if (total > 0) {
-            tmem_ld16(tbase + lane_base + 256 + which * D + c * 16, rr);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tmem_ld16(tbase + lane_base + 256 + which * D + (4 * cb + i) * 16, rr[i]);
             tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hold16(rr[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int e = 0; e < 16; ++e) rr[i][e] = 0u;
           }
           if (row_ok) {
-            if (f32) {
-              float* dst = static_cast<float*>(base) + off + c * 16;
 #pragma unroll
-              for (int i = 0; i < 16; ++i) dst[i] = __uint_as_float(rr[i]) * mul;
-            } else {
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(base) + off + c * 16;
-#pragma unroll
-              for (int i = 0; i < 16; i += 2)
-                *reinterpret_cast<uint32_t*>(dst + i) =
-                    pack_bf16x2(__uint_as_float(rr[i]) * mul, __uint_as_float(rr[i + 1]) * mul);
-            }
+            for (int i = 0; i < 4; ++i) store16(base, off + (4 * cb + i) * 16, f32, rr[i], mul);
           }
         }
       }
