@@ -127,3 +127,17 @@ def test_head_dependent_rule_needs_per_head_block_mask():
     with pytest.raises(fa.FlexAttnError) as e:
         case.run(128, 128, bm=bm)
     assert e.value.status == 5
+
+
+@pytest.mark.parametrize("name", ["half_heads_global", "every_fourth_key"])
+def test_persistent_kernel_with_composed_rules(name):
+    """256 pairs of query tiles, more than the SMs, so running CTAs take over
+    the launches of the rest; the head-dependent rule with a block mask per
+    head, whose items alternate long and short along the head index."""
+    B, H, L = 2, 16, 2048
+    case, reads_head = _case(name, B, H, H, L, L, 128, "bf16", seed=31)
+    bm = case.block_mask(128, 128, B_mask=1, H_mask=H if reads_head else 1)
+    out, lse, mx = case.run(128, 128, bm=bm, split_kv=1, max_scores=True)
+    ro, rl, rm = case.oracle(aux=True)
+    assert_close(case, out, lse, ro, rl, mx, rm)
+    _status_ok()

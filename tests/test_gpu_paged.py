@@ -110,6 +110,13 @@ def test_prefill_paged_tensor_cores(E):
          {"kind": "cap_then_bias", "cap": 30.0, "slope_heads": 0, "pos": "global"}, [704, 650], 128, 1, seed=E)
 
 
+def test_prefill_paged_persistent():
+    # 256 pairs of query tiles over a pool of shuffled 64-key pages: the
+    # persistent tensor-core kernel reads each key tile from two pages
+    _run(2, 16, 4, 2048, 64, 32, 128, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 30.0}, [2048, 1500],
+         128, 1, seed=41)
+
+
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_paged_general_kernel(dtype):
     # pages of 48 keys: not a multiple of 64, so the general kernel reads them
