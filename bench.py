@@ -659,6 +659,26 @@ def measure(wk, args, dev, world, flush, peaks, peak_src):
     if fa.flexattn_poll_device_status() != 0:
         raise RuntimeError(f"{wk.label}: device status word set during warm-up")
     graphs, launch = (None, "eager") if args.eager else wk.capture_graphs()
+    # the step (block-mask build + timed call) as one graph: its replay times
+    # the step; the two per-call graphs time each part
+    g_step = None
+    if graphs:
+        try:
+            outs = wk.grads if wk.backward else (wk.out, wk.lse)
+            ref = [t.clone() for t in outs]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                wk.build()
+                wk.forward()
+            for t in outs:
+                t.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            if all(torch.equal(a, b) for a, b in zip(ref, outs)) and fa.flexattn_poll_device_status() == 0:
+                g_step = g
+                launch = "CUDA graph replay: one graph per step (one per call for the split timings)"
+        except Exception:  # keep the per-call graphs for the step as well
+            torch.cuda.synchronize()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -681,17 +701,25 @@ def measure(wk, args, dev, world, flush, peaks, peak_src):
                 wk.forward()
             e2.record(stream)
             flush.zero_()
+        step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)] if g_step else []
+        for s0, s1 in step_ev:
+            s0.record(stream)
+            g_step.replay()
+            s1.record(stream)
+            flush.zero_()
         torch.cuda.synchronize()
         time.sleep(0.15)
     if world > 1:
         dist.barrier()
     mask_ms = [a.elapsed_time(b) for a, b, _ in ev]
     fwd_ms = [b.elapsed_time(c_) for _, b, c_ in ev]
-    step_ms = [a.elapsed_time(c_) for a, _, c_ in ev]
+    step_ms = ([a.elapsed_time(b) for a, b in step_ev] if step_ev else
+               [a.elapsed_time(c_) for a, _, c_ in ev])
     total_ms = max_over_ranks(sum(step_ms), dev, world)
     if fa.flexattn_poll_device_status() != 0:
         raise RuntimeError(f"{wk.label}: device status word set during the timed region")
-    del graphs
+    del graphs, g_step
 
     ms_per_step = total_ms / args.steps
     fwd_mean = statistics.mean(fwd_ms)

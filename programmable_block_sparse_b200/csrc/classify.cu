@@ -157,10 +157,17 @@ __device__ uint8_t classify_tile_program(const MaskParams& m, int b, int h, int 
   return all_full ? kFull : (any_vis ? kPartial : kEmpty);
 }
 
+// One instantiation per family of rules, so that each launch carries only the
+// code its rule needs (the kernel runs once per call, its instructions are
+// fetched cold): kIntervals for the interval-shaped rules, kDocument,
+// kProgram for composed rules.
+enum RuleFamily { kIntervals = 0, kDocument = 1, kProgram = 2 };
+
+template <int FAMILY>
 __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs a) {
   extern __shared__ uint8_t cls[];
-  __shared__ int s_run_a[kClassifyThreads / 32][129];
-  __shared__ int s_run_id[kClassifyThreads / 32][128];
+  __shared__ int s_run_a[FAMILY == kDocument ? kClassifyThreads / 32 : 1][129];
+  __shared__ int s_run_id[FAMILY == kIntervals ? 1 : kClassifyThreads / 32][128];
   const int mt = blockIdx.x;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,9 +192,9 @@ __global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs
       uint8_t k;
       if (c0 >= S_b || (causal_family && c0 > q_hi)) {
         k = kEmpty;
-      } else if (a.mask.kind == FA_MASK_DOCUMENT) {
+      } else if constexpr (FAMILY == kDocument) {
         k = classify_tile_document(a.mask, b, r0, r1, c0, c1, a.L, a.S, S_b, s_run_a[warp], s_run_id[warp]);
-      } else if (a.mask.kind == FA_MASK_PROGRAM) {
+      } else if constexpr (FAMILY == kProgram) {
         k = classify_tile_program(a.mask, b, hc, r0, r1, c0, c1, a.L, a.S, S_b, s_run_id[warp]);
       } else {
         k = classify_tile_intervals(a.mask, r0, r1, c0, c1, a.L, S_b);
@@ -242,12 +249,14 @@ cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream) {
   const bool per_head = a.mask.kind == FA_MASK_PROGRAM && a.mask.reads_head && a.H > 1;
   dim3 grid(a.Mb, a.B, per_head ? a.H : 1);
   size_t smem = (static_cast<size_t>(a.Nb) + 15) & ~static_cast<size_t>(15);
+  auto kern = a.mask.kind == FA_MASK_DOCUMENT  ? classify_kernel<kDocument>
+              : a.mask.kind == FA_MASK_PROGRAM ? classify_kernel<kProgram>
+                                               : classify_kernel<kIntervals>;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(classify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  classify_kernel<<<grid, kClassifyThreads, smem, stream>>>(a);
+  kern<<<grid, kClassifyThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
