@@ -27,7 +27,11 @@ namespace fa {
 
 namespace {
 
+// threads per CTA: the composed-rule family needs about 120 registers per
+// thread; the others fit 64, so a CTA of 32 warps takes a row of tiles in
+// fewer rounds (the work is a chain of dependent loads per tile)
 constexpr int kClassifyThreads = 256;
+constexpr int kClassifyThreadsWide = 1024;
 enum : uint8_t { kEmpty = 0, kPartial = 1, kFull = 2 };
 
 // |[lo, hi] intersect [c0, c1]| for inclusive bounds.
@@ -164,10 +168,12 @@ __device__ uint8_t classify_tile_program(const MaskParams& m, int b, int h, int 
 enum RuleFamily { kIntervals = 0, kDocument = 1, kProgram = 2 };
 
 template <int FAMILY>
-__global__ void __launch_bounds__(kClassifyThreads) classify_kernel(ClassifyArgs a) {
+__global__ void __launch_bounds__(FAMILY == kProgram ? kClassifyThreads : kClassifyThreadsWide)
+    classify_kernel(ClassifyArgs a) {
+  constexpr int kWarps = (FAMILY == kProgram ? kClassifyThreads : kClassifyThreadsWide) / 32;
   extern __shared__ uint8_t cls[];
-  __shared__ int s_run_a[FAMILY == kDocument ? kClassifyThreads / 32 : 1][129];
-  __shared__ int s_run_id[FAMILY == kIntervals ? 1 : kClassifyThreads / 32][128];
+  __shared__ int s_run_a[FAMILY == kDocument ? kWarps : 1][129];
+  __shared__ int s_run_id[FAMILY == kIntervals ? 1 : kWarps][128];
   const int mt = blockIdx.x;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -252,11 +258,12 @@ cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream) {
   auto kern = a.mask.kind == FA_MASK_DOCUMENT  ? classify_kernel<kDocument>
               : a.mask.kind == FA_MASK_PROGRAM ? classify_kernel<kProgram>
                                                : classify_kernel<kIntervals>;
-  if (smem > 48 * 1024) {
+  // the document family also holds 33 KB of static shared memory
+  if (smem + (a.mask.kind == FA_MASK_DOCUMENT ? 33 * 1024 : 5 * 1024) > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, kClassifyThreads, smem, stream>>>(a);
+  kern<<<grid, a.mask.kind == FA_MASK_PROGRAM ? kClassifyThreads : kClassifyThreadsWide, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
