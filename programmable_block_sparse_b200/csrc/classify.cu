@@ -27,10 +27,10 @@ namespace fa {
 
 namespace {
 
-// threads per CTA: the composed-rule family needs about 120 registers per
-// thread; the others fit 64, so a CTA of 32 warps takes a row of tiles in
-// fewer rounds (the work is a chain of dependent loads per tile)
-constexpr int kClassifyThreads = 256;
+// threads per CTA: 16 warps for composed rules, 32 for the other families,
+// so that a row of tiles is taken in few rounds (a tile's classification is
+// a chain of dependent loads)
+constexpr int kClassifyThreads = 512;
 constexpr int kClassifyThreadsWide = 1024;
 enum : uint8_t { kEmpty = 0, kPartial = 1, kFull = 2 };
 
@@ -258,8 +258,8 @@ cudaError_t launch_classify(const ClassifyArgs& a, cudaStream_t stream) {
   auto kern = a.mask.kind == FA_MASK_DOCUMENT  ? classify_kernel<kDocument>
               : a.mask.kind == FA_MASK_PROGRAM ? classify_kernel<kProgram>
                                                : classify_kernel<kIntervals>;
-  // the document family also holds 33 KB of static shared memory
-  if (smem + (a.mask.kind == FA_MASK_DOCUMENT ? 33 * 1024 : 5 * 1024) > 48 * 1024) {
+  // static shared memory: 33 KB in the document family, 9 KB in the composed
+  if (smem + (a.mask.kind == FA_MASK_DOCUMENT ? 33 * 1024 : 9 * 1024) > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
