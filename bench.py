@@ -86,11 +86,11 @@ HEADLINE = BENCH_ITEMS[0][0]
 # workload is stated in the profile it comes from.
 NCU_TRAFFIC = {
     # fwd_sm100_kernel<128, 0>, captured at batch 1 (profiles/fwd_sm100_gqa_sliding_window.md): x 2 sequences
-    "gqa_sliding_window": {"bytes": 2 * (201698816 + 94893312), "source_hash": "7a8c170bdf2d59bb"},
+    "gqa_sliding_window": {"bytes": 2 * (201789696 + 94654464), "source_hash": "e563253dfa69d1e2"},
     # fwd_sm100_kernel<64, 3> / <128, 3>, full size (profiles/fwd_sm100_causal_packed_sliver.md)
-    "causal_softcap_alibi": {"bytes": 50420480 + 684288, "source_hash": "7a8c170bdf2d59bb"},
-    "packed_docs": {"bytes": 100907776 + 10119424, "source_hash": "7a8c170bdf2d59bb"},
-    "sliver_every_fourth_key": {"bytes": 50427392 + 745216, "source_hash": "7a8c170bdf2d59bb"},
+    "causal_softcap_alibi": {"bytes": 50418944 + 882688, "source_hash": "e563253dfa69d1e2"},
+    "packed_docs": {"bytes": 100893440 + 10517248, "source_hash": "e563253dfa69d1e2"},
+    "sliver_every_fourth_key": {"bytes": 50424320 + 783360, "source_hash": "e563253dfa69d1e2"},
     # decode_tc_kernel<128, 1>, captured at batch 16 (profiles/decode_tc_kernel_decode_kv_cache.md):
     # x 614602 / 296926 cached tokens
     "decode_kv_cache": {"bytes": round((1222132224 + 8572672) * 614602 / 296926), "source_hash": "66031533768da397"},

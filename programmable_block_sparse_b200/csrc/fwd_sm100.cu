@@ -208,6 +208,29 @@ __device__ __noinline__ void tanh_hw_tmem(uint32_t taddr, float c_in) {
   tmem_wait_st();
 }
 
+// The same-document bits of a tile's four 32-key words for the calling row
+// (document id `mine`; `none` clears them): lane l reads the ids of keys
+// 32 w + l from the staged row, and each distinct document among the warp's
+// rows takes one round of ballots (one or two rounds on a packed batch).
+// Called by all 32 lanes of a warp.
+__device__ __noinline__ uint4 doc_words(const int* keys_doc, int mine, bool none) {
+  const int lane = threadIdx.x & 31;
+  int kd[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) kd[w] = keys_doc[32 * w + lane];
+  uint4 r = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t pending = 0xFFFFFFFFu;
+  while (pending) {
+    const int d = __shfl_sync(0xffffffffu, mine, __ffs(pending) - 1);
+    const uint32_t m0 = __ballot_sync(0xffffffffu, kd[0] == d), m1 = __ballot_sync(0xffffffffu, kd[1] == d);
+    const uint32_t m2 = __ballot_sync(0xffffffffu, kd[2] == d), m3 = __ballot_sync(0xffffffffu, kd[3] == d);
+    const bool take = mine == d;
+    if (take) r = make_uint4(m0, m1, m2, m3);
+    pending &= ~__ballot_sync(0xffffffffu, take);
+  }
+  return none ? make_uint4(0u, 0u, 0u, 0u) : r;
+}
+
 // Softmax and epilogue of one 128-row query tile; runs on one warpgroup.
 // gbase counts the group's tiles of earlier work items and nfin the items in
 // which it had tiles (the phases of its barriers run on across items);
@@ -300,6 +323,9 @@ __device__ __forceinline__ bool softmax_group(const FwdArgs& a, Barriers& bars, 
     // that pass 2 subtracts nothing unless the maximum moves.  Arithmetic in
     // f32x2 pairs; maxima as trees of three-input maxima.
     const bool need_mask = !full || edge || !row_ok;
+    // same-document bits of the tile's four 32-key words for this row
+    uint4 doc_bits = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+    if (stage_doc) doc_bits = doc_words(s_doc[g & 1], my_doc, qpos < 0);  // the same for every row of the tile
     const float m_fold = (m_ref == kNoKeyMax) ? 0.0f : m_ref;
     float mx = -INFINITY;  // maximum of t - m_fold over this tile
 #pragma unroll 1
@@ -360,14 +386,9 @@ __device__ __forceinline__ bool softmax_group(const FwdArgs& a, Barriers& bars, 
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const int base = kv0 + c0 + 32 * w;
-          uint32_t same = 0xFFFFFFFFu;  // same-document bits of the word's keys
-          if (stage_doc) {
-            const int* dk = s_doc[g & 1] + c0 + 32 * w;
-            same = 0u;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) same |= (dk[i] == my_doc ? 1u : 0u) << i;
-            if (qpos < 0) same = 0u;
-          }
+          // same-document bits of the word's keys (half is a rolled loop: a
+          // select, not an index, keeps doc_bits in registers)
+          const uint32_t same = half == 0 ? (w == 0 ? doc_bits.x : doc_bits.y) : (w == 0 ? doc_bits.z : doc_bits.w);
           if (is_prog) {
             bits[w] = row_ok ? program_word(&a.mask, h, qpos, base, same, S_b) : 0u;
           } else {
