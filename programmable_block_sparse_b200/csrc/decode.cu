@@ -526,6 +526,28 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16], int lane) {
   return op(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
+// The sequence with the given rank when sequences are ordered by the length
+// of their list of key tiles, longest first (ties by index), for up to 32
+// sequences with lists of their own; otherwise the batch order.  Called by
+// every lane of a warp.
+__device__ __forceinline__ int sequence_of_rank(const FwdArgs& a, int rank) {
+  if (a.B > 32 || a.bm.B == 1) return rank;
+  const int lane = threadIdx.x & 31;
+  int cnt = -1;
+  if (lane < a.B) {
+    const int64_t row = static_cast<int64_t>(lane) * a.bm.H * a.bm.Mb;  // head row 0, query tile 0
+    cnt = __ldg(a.bm.full_kv_num_blocks + row) + __ldg(a.bm.kv_num_blocks + row);
+  }
+  int r = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int cj = __shfl_sync(0xffffffffu, cnt, j);
+    r += (cj > cnt || (cj == cnt && j < lane)) ? 1 : 0;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < a.B && r == rank);
+  return hit ? __ffs(hit) - 1 : rank;
+}
+
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kTcThreads, 2)
     decode_tc_kernel(const __grid_constant__ FwdArgs a, const DecodePlan p,
@@ -543,21 +565,23 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   uint8_t* sQ = smem + C::kRingBytes;
   uint8_t* sP = sQ + C::kQBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // split-major grid (KV head x head chunk, batch, split): every CTA of split 0
-  // (the longest runs of tiles) is dispatched before any of split 1, so the
-  // last CTAs to start are the short remainders
-  const int split = blockIdx.z;
+  // grid (KV head x head chunk, split, rank): CTAs start in linear order, so
+  // the sequences are taken from the longest list of tiles to the shortest,
+  // and each sequence's tiles are cut into p.splits equal chunks: the longest
+  // chunks start first and the last CTAs to start are the shortest
+  const int split = blockIdx.y;
   const int head_chunks = (a.G + p.heads_per_cta - 1) / p.heads_per_cta;
   const int hk = blockIdx.x / head_chunks, hc = blockIdx.x % head_chunks;
-  const int b = blockIdx.y;
+  const int b = sequence_of_rank(a, static_cast<int>(blockIdx.z));
   const int S_b = seq_len_b(a.mask, b, a.S);
   const int bmb = a.bm.B > 1 ? b : 0;
   const int bmh = a.bm.H > 1 ? hk * a.G + hc * p.heads_per_cta : 0;  // per-head lists: one head per CTA
   const int64_t brow = (static_cast<int64_t>(bmb) * a.bm.H + bmh) * a.bm.Mb;
   const int nfull = __ldg(a.bm.full_kv_num_blocks + brow);
   const int ntiles = nfull + __ldg(a.bm.kv_num_blocks + brow);
-  const int t0 = split * p.tiles_per_split;
-  const int t1 = min(ntiles, t0 + p.tiles_per_split);
+  const int chunk = (ntiles + p.splits - 1) / p.splits;  // this sequence's tiles per split
+  const int t0 = split * chunk;
+  const int t1 = min(ntiles, t0 + chunk);
   const int subs = a.bm.BN / kTcKeys;  // 128-key tiles per listed block
   const int nsub = t1 > t0 ? (t1 - t0) * subs : 0;
   volatile int* abort = &bars.abort;
@@ -985,7 +1009,7 @@ cudaError_t launch_decode_d(const FwdArgs& a, const DecodePlan& p, const Sm100Ma
                                                    : decode_tc_kernel<DT, FA_SCORE_CAP_THEN_BIAS>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<DT>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid_tc(a.Hkv * head_chunks, a.B, p.splits);
+    dim3 grid_tc(a.Hkv * head_chunks, p.splits, a.B);
     kern<<<grid_tc, kTcThreads, TcCfg<DT>::kSmemBytes, stream>>>(a, p, maps.k, maps.v, ws_o, ws_lse, ws_max);
   } else {
     auto kern = a.score.kind == FA_SCORE_NONE      ? decode_kernel<D, FA_SCORE_NONE>
