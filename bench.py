@@ -91,11 +91,15 @@ NCU_TRAFFIC = {
     "causal_softcap_alibi": {"bytes": 50418944 + 882688, "source_hash": "e563253dfa69d1e2"},
     "packed_docs": {"bytes": 100893440 + 10517248, "source_hash": "e563253dfa69d1e2"},
     "sliver_every_fourth_key": {"bytes": 50424320 + 783360, "source_hash": "e563253dfa69d1e2"},
+    "half_heads_global": {"bytes": 50460928 + 648448, "source_hash": "e563253dfa69d1e2"},
     # decode_tc_kernel<128, 1>, captured at batch 16 (profiles/decode_tc_kernel_decode_kv_cache.md):
     # x 614602 / 296926 cached tokens
     "decode_kv_cache": {"bytes": round((1220940800 + 7898368) * 614602 / 296926), "source_hash": "ffab78b4d4eb3af3"},
     "decode_kv_cache_q1": {"bytes": round((1220451328 + 4600320) * 614602 / 296926),
                            "source_hash": "ffab78b4d4eb3af3"},
+    # the same kernel over the shuffled 64-key page pool, at batch 16
+    "decode_kv_cache_paged": {"bytes": round((1220960512 + 7605248) * 614602 / 296926),
+                              "source_hash": "ffab78b4d4eb3af3"},
     # bwd_dkdv_kernel (the larger of the two backward kernels), full size
     # (profiles/bwd_dkdv_dq_backward.md)
     "backward_causal_softcap_alibi": {"bytes": 68308736 + 7811072, "source_hash": "6a65fba814bf1a59"},
