@@ -79,6 +79,22 @@ def test_decode_rows_without_keys():
     _status_ok()
 
 
+@pytest.mark.parametrize("kv_len", [[64, 700, 1500, 129, 700], [300] * 3 + [1200] + [5] * 2,
+                                    [(37 * i) % 900 + 40 for i in range(40)]],
+                         ids=["ascending_and_ties", "equal_runs", "forty_sequences"])
+@pytest.mark.parametrize("split_kv", [0, 3])
+def test_decode_sequence_order(kv_len, split_kv):
+    """The tensor-core decode takes sequences longest list first and cuts
+    each into equal chunks: lengths out of order, ties, and more than 32
+    sequences (then taken in batch order)."""
+    case = Case(len(kv_len), 8, 2, 4, 1500, 128, 128, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0},
+                seed=len(kv_len), kv_len=kv_len, sentinel_tail=True)
+    ro, rl, rm = case.oracle(aux=True)
+    out, lse, mx = case.run(128, 128, split_kv=split_kv, max_scores=True)
+    assert_close(case, out, lse, ro, rl, mx, rm)
+    _status_ok()
+
+
 def test_split_counts_agree():
     import programmable_block_sparse_b200 as fa
     case = Case(2, 8, 2, 4, 4096, 128, 128, "bf16", {"kind": "causal"}, {"kind": "softcap", "cap": 50.0}, seed=1,
